@@ -1,0 +1,210 @@
+"""fp64 CPU oracle for the HySparse / HySparse2 hot path (ctypes wrapper).
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` are the only callers.  The product package
+never imports this module, and this module never imports the product package:
+the two share no code.  The arithmetic lives in ``hs_oracle.c`` (plain C,
+double precision, one query row at a time); this file only marshals numpy
+arrays and compiles the C file with gcc on first use.
+
+Function map (titles of the pages the method is described on):
+  full_attn_index  -- "HySparse 混合稀疏注意力（一）" sections on block-level
+                      scores, GQA group max and TopKBlocks; "HySparse: A Hybrid
+                      Sparse Attention Architecture ..." 3.2 / Algorithm 1;
+                      "HySparse2 ..." 4.2 (token-level top-k, forced window).
+  sparse_attn      -- "HySparse 混合稀疏注意力（一）" sections on cross-layer KV
+                      reuse and the two memories of one query; "HySparse ..." 3.3.
+"""
+from __future__ import annotations
+
+import contextlib
+import ctypes
+import os
+import subprocess
+import threading
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "hs_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+_lock = threading.Lock()
+
+
+def build(force: bool = False) -> str:
+    """Compile hs_oracle.c into liboracle.so (gcc, -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("hq", ctypes.c_int), ("hkv", ctypes.c_int),
+                ("head_dim", ctypes.c_int), ("t_q", ctypes.c_int), ("t_kv", ctypes.c_int),
+                ("q_offset", ctypes.c_int), ("mode", ctypes.c_int),
+                ("block_size", ctypes.c_int), ("k", ctypes.c_int), ("window", ctypes.c_int),
+                ("scale", ctypes.c_double)]
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = _bind(ctypes.CDLL(build()))
+    return _lib
+
+
+def _bind(lib):
+    P = ctypes.c_void_p
+    lib.orc_full_attn_index.argtypes = [ctypes.POINTER(_Params), P, P, P, P, ctypes.c_int,
+                                        P, P, P, P, P, P, P, ctypes.c_int]
+    lib.orc_full_attn_index.restype = ctypes.c_int
+    lib.orc_sparse_attn.argtypes = [ctypes.POINTER(_Params), P, P, P, P, ctypes.c_int, P,
+                                    P, P, P, P, P, P, P, P]
+    lib.orc_sparse_attn.restype = ctypes.c_int
+    lib.orc_num_threads.restype = ctypes.c_int
+    return lib
+
+
+@contextlib.contextmanager
+def use_library(path: str):
+    """Temporarily route every oracle call to another build of hs_oracle.c.
+
+    Used only by the mutation tests, which compile deliberately broken copies
+    of the oracle and check that the pins reject them.
+    """
+    global _lib
+    with _lock:
+        old = _lib
+        _lib = _bind(ctypes.CDLL(path))
+    try:
+        yield
+    finally:
+        with _lock:
+            _lib = old
+
+
+@dataclass
+class Params:
+    """Shapes and the method's knobs.  mode: "block" (HySparse) or "token" (HySparse2)."""
+    batch: int
+    hq: int
+    hkv: int
+    head_dim: int
+    t_q: int
+    t_kv: int
+    mode: str = "block"
+    block_size: int = 64
+    k: int = 1024
+    window: int = 128
+    q_offset: int = 0
+    scale: float = 0.0  # 0 -> 1/sqrt(head_dim)
+
+    @property
+    def group(self) -> int:
+        return self.hq // self.hkv
+
+    @property
+    def ksel(self) -> int:
+        return self.k // self.block_size if self.mode == "block" else self.k
+
+    def _c(self) -> _Params:
+        s = self.scale if self.scale > 0 else 1.0 / np.sqrt(self.head_dim)
+        return _Params(self.batch, self.hq, self.hkv, self.head_dim, self.t_q, self.t_kv,
+                       self.q_offset, 0 if self.mode == "block" else 1, self.block_size,
+                       self.k, self.window, float(s))
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _rows_array(p: Params, rows, decode: bool) -> np.ndarray:
+    if rows is None:
+        tq = 1 if decode else p.t_q
+        b, u, j = np.meshgrid(np.arange(p.batch), np.arange(p.hkv), np.arange(tq), indexing="ij")
+        rows = np.stack([b.ravel(), u.ravel(), j.ravel()], axis=1)
+    return np.ascontiguousarray(np.asarray(rows, dtype=np.int32).reshape(-1, 3))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    return int(_load().orc_num_threads())
+
+
+def full_attn_index(p: Params, q, k, v, rows=None, kv_len=None, want_scores: bool = False):
+    """Full attention + oracle index for the listed rows (default: all rows).
+
+    rows: int array [n, 3] of (batch, kv group, query row).  kv_len: per-batch
+    cache length for decode (the query is then the newest token).
+    Returns dict with o [n, g, d], lse [n, g], idx [n, ksel], cnt [n],
+    sel_score [n, ksel] and, if asked, scores [n, n_cand] (-1 beyond the row's
+    candidates).
+    """
+    lib = _load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    assert q.shape == (p.batch, p.hq, p.t_q, p.head_dim), q.shape
+    assert k.shape == v.shape == (p.batch, p.hkv, p.t_kv, p.head_dim), k.shape
+    rws = _rows_array(p, rows, kv_len is not None)
+    kvl = None if kv_len is None else np.ascontiguousarray(np.asarray(kv_len, dtype=np.int32))
+    n, g, d, ks = len(rws), p.group, p.head_dim, p.ksel
+    o = np.zeros((n, g, d)); lse = np.zeros((n, g))
+    idx = np.zeros((n, ks), dtype=np.int32); cnt = np.zeros(n, dtype=np.int32)
+    sel = np.zeros((n, ks))
+    stride = 0
+    scores = None
+    if want_scores:
+        stride = (-(-p.t_kv // p.block_size)) if p.mode == "block" else p.t_kv
+        scores = np.zeros((n, stride))
+    c = p._c()
+    rc = lib.orc_full_attn_index(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), _ptr(kvl), n,
+                                 _ptr(rws), _ptr(o), _ptr(lse), _ptr(idx), _ptr(cnt), _ptr(sel),
+                                 _ptr(scores), stride)
+    if rc != 0:
+        raise ValueError("oracle: invalid arguments")
+    out = dict(rows=rws, o=o, lse=lse, idx=idx, cnt=cnt, sel_score=sel)
+    if want_scores:
+        out["scores"] = scores
+    return out
+
+
+def sparse_attn(p: Params, q, kf, vf, idx_rows, cnt_rows, rows=None, kv_len=None,
+                k_loc=None, v_loc=None):
+    """Sparse layer over the listed rows, reusing K^F/V^F and the given index sets.
+
+    idx_rows [n, ksel] / cnt_rows [n] are the index sets of the listed rows.
+    Returns dict with o_g [n, g, d], lse_g [n, g] and, when k_loc is given,
+    o_l / lse_l of the local (own K'/V') window branch.
+    """
+    lib = _load()
+    q, kf, vf = _f64(q), _f64(kf), _f64(vf)
+    rws = _rows_array(p, rows, kv_len is not None)
+    n, g, d, ks = len(rws), p.group, p.head_dim, p.ksel
+    idx_rows = np.ascontiguousarray(np.asarray(idx_rows, dtype=np.int32).reshape(n, ks))
+    cnt_rows = np.ascontiguousarray(np.asarray(cnt_rows, dtype=np.int32).reshape(n))
+    for r in range(n):  # the oracle sums over the list as given: it must be a set
+        ids = idx_rows[r, :cnt_rows[r]]
+        assert len(np.unique(ids)) == len(ids), "index set has duplicates"
+    kvl = None if kv_len is None else np.ascontiguousarray(np.asarray(kv_len, dtype=np.int32))
+    kl = None if k_loc is None else _f64(k_loc)
+    vl = None if v_loc is None else _f64(v_loc)
+    o_g = np.zeros((n, g, d)); lse_g = np.zeros((n, g))
+    o_l = np.zeros((n, g, d)); lse_l = np.zeros((n, g))
+    c = p._c()
+    rc = lib.orc_sparse_attn(ctypes.byref(c), _ptr(q), _ptr(kf), _ptr(vf), _ptr(kvl), n,
+                             _ptr(rws), _ptr(idx_rows), _ptr(cnt_rows), _ptr(kl), _ptr(vl),
+                             _ptr(o_g), _ptr(lse_g), _ptr(o_l), _ptr(lse_l))
+    if rc != 0:
+        raise ValueError("oracle: invalid arguments")
+    out = dict(rows=rws, o_g=o_g, lse_g=lse_g)
+    if k_loc is not None:
+        out.update(o_l=o_l, lse_l=lse_l)
+    return out

@@ -61,10 +61,10 @@ def _load():
 
 def _bind(lib):
     P = ctypes.c_void_p
-    lib.orc_full_attn_index.argtypes = [ctypes.POINTER(_Params), P, P, P, P, ctypes.c_int,
+    lib.orc_full_attn_index.argtypes = [ctypes.POINTER(_Params), P, P, P, P, P, ctypes.c_int,
                                         P, P, P, P, P, P, P, ctypes.c_int]
     lib.orc_full_attn_index.restype = ctypes.c_int
-    lib.orc_sparse_attn.argtypes = [ctypes.POINTER(_Params), P, P, P, P, ctypes.c_int, P,
+    lib.orc_sparse_attn.argtypes = [ctypes.POINTER(_Params), P, P, P, P, P, ctypes.c_int, P,
                                     P, P, P, P, P, P, P, P]
     lib.orc_sparse_attn.restype = ctypes.c_int
     lib.orc_num_threads.restype = ctypes.c_int
@@ -140,11 +140,21 @@ def num_threads() -> int:
     return int(_load().orc_num_threads())
 
 
-def full_attn_index(p: Params, q, k, v, rows=None, kv_len=None, want_scores: bool = False):
+def _pos(q_pos, n):
+    if q_pos is None:
+        return None
+    a = np.ascontiguousarray(np.asarray(q_pos, dtype=np.int32).reshape(-1))
+    assert len(a) == n
+    return a
+
+
+def full_attn_index(p: Params, q, k, v, rows=None, kv_len=None, want_scores: bool = False,
+                    q_pos=None):
     """Full attention + oracle index for the listed rows (default: all rows).
 
     rows: int array [n, 3] of (batch, kv group, query row).  kv_len: per-batch
-    cache length for decode (the query is then the newest token).
+    cache length for decode (the query is then the newest token).  q_pos:
+    optional explicit position of each listed row.
     Returns dict with o [n, g, d], lse [n, g], idx [n, ksel], cnt [n],
     sel_score [n, ksel] and, if asked, scores [n, n_cand] (-1 beyond the row's
     candidates).
@@ -165,7 +175,8 @@ def full_attn_index(p: Params, q, k, v, rows=None, kv_len=None, want_scores: boo
         stride = (-(-p.t_kv // p.block_size)) if p.mode == "block" else p.t_kv
         scores = np.zeros((n, stride))
     c = p._c()
-    rc = lib.orc_full_attn_index(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), _ptr(kvl), n,
+    qp = _pos(q_pos, n)
+    rc = lib.orc_full_attn_index(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), _ptr(kvl), _ptr(qp), n,
                                  _ptr(rws), _ptr(o), _ptr(lse), _ptr(idx), _ptr(cnt), _ptr(sel),
                                  _ptr(scores), stride)
     if rc != 0:
@@ -177,7 +188,7 @@ def full_attn_index(p: Params, q, k, v, rows=None, kv_len=None, want_scores: boo
 
 
 def sparse_attn(p: Params, q, kf, vf, idx_rows, cnt_rows, rows=None, kv_len=None,
-                k_loc=None, v_loc=None):
+                k_loc=None, v_loc=None, q_pos=None):
     """Sparse layer over the listed rows, reusing K^F/V^F and the given index sets.
 
     idx_rows [n, ksel] / cnt_rows [n] are the index sets of the listed rows.
@@ -199,7 +210,8 @@ def sparse_attn(p: Params, q, kf, vf, idx_rows, cnt_rows, rows=None, kv_len=None
     o_g = np.zeros((n, g, d)); lse_g = np.zeros((n, g))
     o_l = np.zeros((n, g, d)); lse_l = np.zeros((n, g))
     c = p._c()
-    rc = lib.orc_sparse_attn(ctypes.byref(c), _ptr(q), _ptr(kf), _ptr(vf), _ptr(kvl), n,
+    qp = _pos(q_pos, n)
+    rc = lib.orc_sparse_attn(ctypes.byref(c), _ptr(q), _ptr(kf), _ptr(vf), _ptr(kvl), _ptr(qp), n,
                              _ptr(rws), _ptr(idx_rows), _ptr(cnt_rows), _ptr(kl), _ptr(vl),
                              _ptr(o_g), _ptr(lse_g), _ptr(o_l), _ptr(lse_l))
     if rc != 0:
@@ -207,4 +219,96 @@ def sparse_attn(p: Params, q, kf, vf, idx_rows, cnt_rows, rows=None, kv_len=None
     out = dict(rows=rws, o_g=o_g, lse_g=lse_g)
     if k_loc is not None:
         out.update(o_l=o_l, lse_l=lse_l)
+    return out
+
+
+# ------------------------------------------------------------ sampled rows
+def _units(rows):
+    order = {}
+    for n, (b, u, _) in enumerate(rows):
+        order.setdefault((int(b), int(u)), []).append(n)
+    return order
+
+
+def _f64_any(t):
+    """float64 numpy copy of a numpy array or a (CPU or CUDA) torch tensor."""
+    if hasattr(t, "detach"):
+        import torch
+        return t.detach().to("cpu", torch.float64).numpy()
+    return _f64(t)
+
+
+def _take_rows(q, b, h0, h1, js):
+    if hasattr(q, "index_select"):
+        import torch
+        return q[b, h0:h1].index_select(1, torch.as_tensor(js, device=q.device))[None]
+    return q[b, h0:h1][:, js][None]
+
+
+def full_attn_rows(q, k, v, rows, pos, mode, block_size, k_budget, window):
+    """full_attn_index on the listed rows (b, u, j) at positions pos only.
+
+    q [b, hq, tq, d], k/v [b, hkv, T, d] (numpy or torch, any device).  Per
+    (batch, group) only the rows' query vectors and the group's K/V prefix
+    0..max(pos) are converted to float64, so rows of very long contexts can be
+    evaluated without a float64 copy of the whole cache.  Returns o, lse, idx,
+    cnt and the per-row candidate scores (list of arrays) in row order.
+    """
+    rows = np.asarray(rows, dtype=np.int32).reshape(-1, 3)
+    pos = np.asarray(pos, dtype=np.int64).reshape(-1)
+    hq, d = q.shape[1], q.shape[3]
+    hkv = k.shape[1]
+    g = hq // hkv
+    ksel = k_budget // block_size if mode == "block" else k_budget
+    n = len(rows)
+    out = dict(rows=rows, o=np.zeros((n, g, d)), lse=np.zeros((n, g)),
+               idx=np.zeros((n, ksel), np.int32), cnt=np.zeros(n, np.int32),
+               scores=[None] * n, _t=pos)
+    for (b, u), ns in _units(rows).items():
+        ns = np.array(ns)
+        ts = pos[ns]
+        tmax = int(ts.max())
+        qs = _take_rows(q, b, u * g, (u + 1) * g, rows[ns, 2].astype(np.int64))
+        p = Params(1, g, 1, d, len(ns), tmax + 1, mode=mode, block_size=block_size,
+                   k=k_budget, window=window)
+        r = full_attn_index(p, _f64_any(qs), _f64_any(k[b, u, :tmax + 1][None, None]),
+                            _f64_any(v[b, u, :tmax + 1][None, None]),
+                            rows=[(0, 0, x) for x in range(len(ns))], q_pos=ts, want_scores=True)
+        out["o"][ns] = r["o"]
+        out["lse"][ns] = r["lse"]
+        out["idx"][ns] = r["idx"]
+        out["cnt"][ns] = r["cnt"]
+        for x, nn in enumerate(ns):
+            out["scores"][nn] = r["scores"][x]
+    return out
+
+
+def sparse_attn_rows(q, kf, vf, idx_rows, cnt_rows, rows, pos, mode, block_size, k_budget,
+                     window, k_loc=None, v_loc=None):
+    """sparse_attn on the listed rows only (same conventions as full_attn_rows)."""
+    rows = np.asarray(rows, dtype=np.int32).reshape(-1, 3)
+    pos = np.asarray(pos, dtype=np.int64).reshape(-1)
+    idx_rows = np.asarray(idx_rows)
+    cnt_rows = np.asarray(cnt_rows)
+    hq, d = q.shape[1], q.shape[3]
+    g = hq // kf.shape[1]
+    n = len(rows)
+    out = dict(o_g=np.zeros((n, g, d)), lse_g=np.zeros((n, g)), o_l=np.zeros((n, g, d)),
+               lse_l=np.zeros((n, g)))
+    for (b, u), ns in _units(rows).items():
+        ns = np.array(ns)
+        ts = pos[ns]
+        tmax = int(ts.max())
+        q1 = _take_rows(q, b, u * g, (u + 1) * g, rows[ns, 2].astype(np.int64))
+        p = Params(1, g, 1, d, len(ns), tmax + 1, mode=mode, block_size=block_size,
+                   k=k_budget, window=window)
+        sl = lambda t: None if t is None else _f64_any(t[b, u, :tmax + 1][None, None])  # noqa
+        r = sparse_attn(p, _f64_any(q1), sl(kf), sl(vf), idx_rows[ns], cnt_rows[ns],
+                        rows=[(0, 0, x) for x in range(len(ns))], q_pos=ts, k_loc=sl(k_loc),
+                        v_loc=sl(v_loc))
+        out["o_g"][ns] = r["o_g"]
+        out["lse_g"][ns] = r["lse_g"]
+        if k_loc is not None:
+            out["o_l"][ns] = r["o_l"]
+            out["lse_l"][ns] = r["lse_l"]
     return out

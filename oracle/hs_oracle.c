@@ -64,10 +64,14 @@ int orc_ksel(const orc_params* p) {
     return p->mode == 0 ? p->k / p->block_size : p->k;
 }
 
-/* Query position and number of visible keys for a row.
- * Prefill: t = q_offset + j, keys 0..t.  Decode (kv_len given): the single
- * query is the newest token, t = kv_len[b]-1.                               */
-static int orc_position(const orc_params* p, const int* kv_len, const orc_row* r) {
+/* Query position of listed row number n; the row sees keys 0..t.
+ * Prefill: t = q_offset + j.  Decode (kv_len given): the single query is the
+ * newest token, t = kv_len[b]-1.  q_pos (nullable) gives each listed row its
+ * position explicitly, so a caller can pass just the query vectors it wants
+ * evaluated (row j of q is then only storage, not a position).            */
+static int orc_position(const orc_params* p, const int* kv_len, const int* q_pos, int n,
+                        const orc_row* r) {
+    if (q_pos) return q_pos[n];
     if (kv_len) return kv_len[r->b] - 1;
     return p->q_offset + r->j;
 }
@@ -150,7 +154,7 @@ static int int_cmp(const void* a, const void* b) {
  *             (blocks 0..nb-1 or tokens 0..t), -1 beyond
  */
 int orc_full_attn_index(const orc_params* p, const double* q, const double* k,
-                        const double* v, const int* kv_len, int n_rows,
+                        const double* v, const int* kv_len, const int* q_pos, int n_rows,
                         const orc_row* rows, double* o, double* lse, int* idx,
                         int* cnt, double* sel_score, double* scores,
                         int scores_stride) {
@@ -163,7 +167,7 @@ int orc_full_attn_index(const orc_params* p, const double* q, const double* k,
 #pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
     for (int r = 0; r < n_rows; ++r) {
         const orc_row* row = &rows[r];
-        const int t = orc_position(p, kv_len, row);
+        const int t = orc_position(p, kv_len, q_pos, r, row);
         const int n = t + 1; /* visible keys 0..t */
         if (t < 0 || t >= p->t_kv) { bad = 1; continue; }
         int* keys = (int*)malloc(sizeof(int) * n);
@@ -262,7 +266,8 @@ int orc_full_attn_index(const orc_params* p, const double* q, const double* k,
  * (only written when k_loc != NULL).
  */
 int orc_sparse_attn(const orc_params* p, const double* q, const double* kf,
-                    const double* vf, const int* kv_len, int n_rows, const orc_row* rows,
+                    const double* vf, const int* kv_len, const int* q_pos, int n_rows,
+                    const orc_row* rows,
                     const int* idx_rows, const int* cnt_rows, const double* k_loc,
                     const double* v_loc, double* o_g, double* lse_g, double* o_l,
                     double* lse_l) {
@@ -273,7 +278,7 @@ int orc_sparse_attn(const orc_params* p, const double* q, const double* kf,
 #pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
     for (int r = 0; r < n_rows; ++r) {
         const orc_row* row = &rows[r];
-        const int t = orc_position(p, kv_len, row);
+        const int t = orc_position(p, kv_len, q_pos, r, row);
         const int c = cnt_rows[r];
         const int B = p->mode == 0 ? p->block_size : 1;
         if (t < 0 || t >= p->t_kv || c < 0 || c > ksel) { bad = 1; continue; }

@@ -1,0 +1,451 @@
+#!/usr/bin/env python
+"""Benchmark of the HySparse hybrid block on one B200 per process.
+
+A step is one pass of the hot path over one batch of synthetic input: the
+full-attention layer with its oracle indexer, then the block's sparse layers
+reusing its K^F/V^F and index set (HySparse 7B-dense-shaped block-level
+prefill by default: b=2, T=16384, 32/8 heads, d=128, bf16, B=64, k=1024,
+1 full : 3 sparse, each sparse layer with its own 128-token window K'/V').
+
+Printed value (rank 0, one JSON line): the step's peak-normalised throughput,
+    (F_full / P_tensor + B_sparse / P_hbm) / t_step, summed over ranks,
+i.e. the fraction of one B200's roofline the step achieves (N x that for N
+replicas).  The line also carries the two halves of the metric separately:
+full+index TFLOP/s and sparse-reuse K/V GB/s, each with its fraction of peak.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload (the only place besides the cpu_baseline field
+where this script runs the oracle).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from oracle_top_kv_b200 import accounting as A  # noqa: E402
+from oracle_top_kv_b200 import workloads as wl  # noqa: E402
+
+METRIC = "full+index prefill TFLOP/s and sparse-reuse KV GB/s (fraction of B200 peak)"
+UNIT = "fraction of one B200 roofline (step)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples of this GPU's clocks while the timed region runs."""
+
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.rows, self.proc, self.err = [], None, None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.gpu_id = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception as e:  # pragma: no cover
+            self.gpu_id, self.err = None, repr(e)
+
+    def start(self):
+        if self.gpu_id is None:
+            return
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception as e:
+            self.err = repr(e)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) == 7:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                    "note": self.err or "no nvidia-smi samples"}
+        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4)
+                          if r[3 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+# ------------------------------------------------------------------ our arm
+class HybridBlock:
+    """Device buffers and C-ABI calls of one full layer + its sparse layers."""
+
+    def __init__(self, w, device):
+        from oracle_top_kv_b200 import hs
+        self.hs = hs
+        self.w = w
+        self.dev = device
+        q, k, v, _ = wl.full_layer_inputs(w, device=device)
+        self.q, self.k, self.v = q, k, v
+        self.p = hs.make_params(w.batch, w.hq, w.hkv, w.head_dim, w.tq, w.t, w.q_offset, w.dtype,
+                                w.mode, w.block_size, w.k, w.window)
+        self.o, self.lse, self.idx, self.cnt, _ = hs.full_outputs(self.p, device)
+        self.qs, self.kl, self.vl, self.og, self.lg, self.ol, self.ll = [], [], [], [], [], [], []
+        for layer in range(w.n_sparse):
+            qs = wl.sparse_layer_query(w, layer, device=device)
+            self.qs.append(qs)
+            self.og.append(torch.empty_like(qs))
+            self.lg.append(torch.empty(w.batch, w.hq, w.tq, dtype=torch.float32, device=device))
+            if w.swa_branch:
+                kl, vl = wl.sparse_layer_local_kv(w, layer, device=device)
+                self.kl.append(kl)
+                self.vl.append(vl)
+                self.ol.append(torch.empty_like(qs))
+                self.ll.append(torch.empty_like(self.lg[-1]))
+            else:
+                self.kl.append(None); self.vl.append(None); self.ol.append(None); self.ll.append(None)
+
+    def full(self, stream):
+        self.hs.hs_full_attn_index(self.p, self.q, self.k, self.v, self.o, self.lse, self.idx,
+                                   self.cnt, None, None, stream)
+
+    def sparse(self, layer, stream):
+        self.hs.hs_sparse_attn_reuse(self.p, self.qs[layer], self.k, self.v, self.idx, self.cnt,
+                                     self.kl[layer], self.vl[layer], self.og[layer],
+                                     self.lg[layer], self.ol[layer], self.ll[layer], None, stream)
+
+    def inputs(self):
+        t = [self.q, self.k, self.v] + self.qs
+        if self.w.swa_branch:
+            t += self.kl + self.vl
+        return t
+
+    def outputs(self):
+        t = [self.o, self.lse, self.idx, self.cnt] + self.og + self.lg
+        if self.w.swa_branch:
+            t += self.ol + self.ll
+        return t
+
+
+def work(w, blk):
+    """Algorithmic FLOPs of the full layer and bytes of each sparse layer."""
+    flops = A.full_layer_flops(w.batch, w.hq, w.head_dim, w.tq, w.q_offset)
+    rows = A.sparse_rows_from_index(blk.idx, blk.cnt, w.mode, w.block_size, w.q_offset)
+    local = A.window_rows(w.batch, w.hkv, w.tq, w.window, w.q_offset) if w.swa_branch else 0
+    elt = 2 if w.dtype == "bf16" else 4
+    sbytes = A.sparse_layer_bytes(rows, w.batch, w.hq, w.tq, w.head_dim, elt, w.ksel, w.hkv, local)
+    return flops, sbytes
+
+
+def traffic_for(kernel, workload):
+    """Per-launch DRAM bytes from the committed ncu summary, if the kernel's
+    source is unchanged since the capture; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path)).get(kernel)
+    if not d or d.get("workload") != workload:
+        return None
+    h = hashlib.sha256()
+    for f in d.get("sources", []):
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return d["bytes_per_launch"] if h.hexdigest() == d.get("sha256") else None
+
+
+def run_ours(args, rank, world, device):
+    from oracle_top_kv_b200 import hs
+    hs.load()
+    w = wl.WORKLOADS[args.workload]
+    peaks, peak_kind = load_peaks()
+    blk = HybridBlock(w, device)
+    stream = torch.cuda.current_stream(device)
+    sh = stream.cuda_stream
+
+    def step():
+        blk.full(sh)
+        for layer in range(w.n_sparse):
+            blk.sparse(layer, sh)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    assert hs.hs_device_status(sh) == 0
+    flops, sbytes = work(w, blk)
+
+    n_ev = 1 + w.n_sparse
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev + 1)]
+           for _ in range(args.steps)]
+    clocks = ClockSampler(device)
+    clocks.start()
+    time.sleep(0.5)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    launches0 = hs.hs_launch_count()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s in range(args.steps):
+        evs[s][0].record(stream)
+        blk.full(sh)
+        evs[s][1].record(stream)
+        for layer in range(w.n_sparse):
+            blk.sparse(layer, sh)
+            evs[s][2 + layer].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    launches = hs.hs_launch_count() - launches0
+    if world > 1:
+        torch.distributed.barrier()
+    clocks.stop()
+    total_ms = t0.elapsed_time(t1)
+    if world > 1:
+        tt = torch.tensor([total_ms], device=device)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    assert hs.hs_device_status(sh) == 0
+    full_ms = [evs[s][0].elapsed_time(evs[s][1]) for s in range(args.steps)]
+    sparse_ms = [evs[s][1 + l].elapsed_time(evs[s][2 + l]) for s in range(args.steps)
+                 for l in range(w.n_sparse)]
+    ms_step = total_ms / args.steps
+
+    p_tensor = peaks["bf16_tflops_sustained"] * 1e12
+    p_hbm = peaks["hbm_gbs"] * 1e9
+    full_s = statistics.mean(full_ms) / 1e3
+    sparse_s = statistics.mean(sparse_ms) / 1e3
+    ideal = flops / p_tensor + w.n_sparse * sbytes / p_hbm
+    value = world * ideal / (ms_step / 1e3)
+    full_tflops = flops / full_s / 1e12
+    sparse_gbs = sbytes / sparse_s / 1e9
+    tokens = w.batch * w.tq
+    # dominant kernel: the one with the larger share of the step
+    if sum(full_ms) >= sum(sparse_ms):
+        roof = {"kernel": "full_attn_index", "bound": "tensor", "achieved": full_tflops,
+                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": full_tflops / peaks["bf16_tflops_sustained"],
+                "traffic": traffic_for("full_attn_index", w.name),
+                "peak_source": f"{peak_kind} bf16_tflops_sustained",
+                "work_per_launch": flops, "avg_launch_ms": full_s * 1e3}
+    else:
+        roof = {"kernel": "sparse_attn_reuse", "bound": "hbm", "achieved": sparse_gbs,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": sparse_gbs / peaks["hbm_gbs"],
+                "traffic": traffic_for("sparse_attn_reuse", w.name),
+                "peak_source": f"{peak_kind} hbm_gbs",
+                "work_per_launch": sbytes, "avg_launch_ms": sparse_s * 1e3}
+
+    e2e = run_e2e(args, blk, w, stream, ideal, world, device) if not args.no_e2e else None
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seq_len": w.t, "hq": w.hq,
+                   "hkv": w.hkv, "head_dim": w.head_dim, "mode": w.mode,
+                   "block_size": w.block_size, "k": w.k, "window": w.window,
+                   "sparse_layers": w.n_sparse, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (step reads > 1 GB; K^F+V^F alone 134 MB)"},
+        "full_index_tflops": full_tflops * world,
+        "full_index_frac_of_peak": full_tflops / peaks["bf16_tflops_sustained"],
+        "sparse_kv_gbs": sparse_gbs * world,
+        "sparse_frac_of_hbm_peak": sparse_gbs / peaks["hbm_gbs"],
+        "full_ms": full_s * 1e3, "sparse_ms_per_layer": sparse_s * 1e3,
+        "tokens_per_s": world * tokens / (ms_step / 1e3),
+        "peaks": {"bf16_tflops_sustained": peaks["bf16_tflops_sustained"],
+                  "hbm_gbs": peaks["hbm_gbs"], "source": peak_kind},
+        "roofline": roof, "gpu_launches": launches, "clocks": clocks.summary(),
+        "e2e": e2e,
+    }
+    return line
+
+
+def run_e2e(args, blk, w, stream, ideal, world, device):
+    """Same step through the C ABI with inputs in pinned host memory: every
+    step copies its inputs host->device and its results device->host."""
+    host_in = [t.cpu().pin_memory() for t in blk.inputs()]
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in blk.outputs()]
+    dev_in, dev_out = blk.inputs(), blk.outputs()
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    sh = stream.cuda_stream
+
+    def step():
+        for d, h in zip(dev_in, host_in):
+            d.copy_(h, non_blocking=True)
+        blk.full(sh)
+        for layer in range(w.n_sparse):
+            blk.sparse(layer, sh)
+        for h, d in zip(host_out, dev_out):
+            h.copy_(d, non_blocking=True)
+
+    n = max(1, min(args.steps, 3))
+    step()
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = e0.elapsed_time(e1) / n
+    if world > 1:
+        tt = torch.tensor([ms], device=device)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        ms = float(tt.item())
+    return {"value": world * ideal / (ms / 1e3), "unit": UNIT, "ms_per_step": ms,
+            "steps": n, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+# --------------------------------------------------------------- oracle arm
+def oracle_inputs(w):
+    q, k, v, _ = wl.full_layer_inputs(w, device="cpu")
+    layers = []
+    for layer in range(w.n_sparse):
+        qs = wl.sparse_layer_query(w, layer, device="cpu")
+        kl, vl = wl.sparse_layer_local_kv(w, layer, device="cpu") if w.swa_branch else (None, None)
+        layers.append((qs, kl, vl))
+    return q, k, v, layers
+
+
+def oracle_sample_time(w, inputs, budget_rows=48, seed=0):
+    """Time the fp64 oracle on a bounded sample of the step and extrapolate.
+
+    Sample: `budget_rows` query rows spread over positions (and over batch and
+    kv groups), each through the full layer and every sparse layer.  The full
+    layer's cost grows with the row's position, the sparse layers' does not,
+    so the extrapolation weights rows by visible keys and by count respectively.
+    """
+    import oracle
+    q, k, v, layers = inputs
+    rng = np.random.default_rng(seed)
+    js = np.unique(np.linspace(0, w.tq - 1, budget_rows).astype(int))
+    rows = np.array([(int(rng.integers(0, w.batch)), int(rng.integers(0, w.hkv)), int(j))
+                     for j in js], np.int32)
+    pos = w.q_offset + rows[:, 2]
+    t0 = time.perf_counter()
+    orc = oracle.full_attn_rows(q, k, v, rows, pos, w.mode, w.block_size, w.k, w.window)
+    t_full = time.perf_counter() - t0
+    t_sp = 0.0
+    for (qs, kl, vl) in layers:
+        t0 = time.perf_counter()
+        oracle.sparse_attn_rows(qs, k, v, orc["idx"], orc["cnt"], rows, pos, w.mode,
+                                w.block_size, w.k, w.window, kl, vl)
+        t_sp += time.perf_counter() - t0
+    n_all = w.batch * w.hkv * w.tq
+    all_pairs = w.batch * w.hkv * A.causal_pairs(w.tq, w.q_offset)
+    est_full = t_full * all_pairs / float((pos + 1).sum())
+    est_sparse = t_sp * n_all / len(rows)
+    sample = (f"{len(rows)} query rows (all heads of their group) through the full layer and "
+              f"{w.n_sparse} sparse layers, timed {t_full + t_sp:.2f} s, extrapolated to the "
+              f"whole step by visible keys (full layer) and by row count (sparse layers)")
+    return est_full + est_sparse, sample, oracle.num_threads()
+
+
+def cpu_value(w, t_step):
+    peaks, _ = load_peaks()
+    flops = A.full_layer_flops(w.batch, w.hq, w.head_dim, w.tq, w.q_offset)
+    rows = w.batch * w.hkv * sum(min(w.k, w.q_offset + j + 1) for j in range(w.tq))
+    local = A.window_rows(w.batch, w.hkv, w.tq, w.window, w.q_offset) if w.swa_branch else 0
+    sbytes = A.sparse_layer_bytes(rows, w.batch, w.hq, w.tq, w.head_dim, 2, w.ksel, w.hkv, local)
+    ideal = (flops / (peaks["bf16_tflops_sustained"] * 1e12) +
+             w.n_sparse * sbytes / (peaks["hbm_gbs"] * 1e9))
+    return ideal / t_step
+
+
+def run_reference(args, w):
+    inputs = oracle_inputs(w)
+    for s in range(args.warmup):
+        oracle_sample_time(w, inputs, budget_rows=12, seed=1000 + s)
+    times = []
+    sample = cores = None
+    for s in range(max(1, args.steps)):
+        t, sample, cores = oracle_sample_time(w, inputs, budget_rows=12, seed=s)
+        times.append(t)
+    t_step = statistics.mean(times)
+    v = cpu_value(w, t_step)
+    return {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": 0, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": w.name, "batch": w.batch, "seq_len": w.t},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": "per step: " + sample},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="hysparse_7b_block", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = wl.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, w)), flush=True)
+        return
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    line = run_ours(args, rank, world, device)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t, sample, cores = oracle_sample_time(w, oracle_inputs(w))
+        line["cpu_baseline"] = {"value": cpu_value(w, t), "unit": UNIT, "cores": cores,
+                                "kind": "oracle", "sample": sample,
+                                "ms_per_step_extrapolated": t * 1e3}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

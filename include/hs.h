@@ -1,0 +1,179 @@
+/*
+ * hs.h -- C ABI of the B200 (sm_100a) HySparse / HySparse2 hot path.
+ *
+ * Two halves of one hybrid block, as the pages describe them:
+ *   1. a full-attention layer that is also the oracle indexer: exact causal
+ *      GQA softmax attention that, besides O, emits per query and KV group the
+ *      index set of the best keys ("HySparse 混合稀疏注意力（一）", sections
+ *      "从精确注意力里提取块级分数" and "GQA 下为什么要组内共享索引";
+ *      "HySparse: A Hybrid Sparse Attention Architecture ...", 3.2 and
+ *      Algorithm 1; "HySparse2: Hybrid Sparse Attention with Two-Level KV
+ *      Sharing", 4.2 "改造一"/"改造二");
+ *   2. the sparse layers that follow it, which reuse that layer's K^F/V^F and
+ *      index set and run attention over only the selected keys, with their own
+ *      query ("HySparse 混合稀疏注意力（一）", "跨层 KV Cache 复用怎样成立" and
+ *      "同一个 Query，查询两种记忆"; "HySparse ..." 3.3).
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates or frees device memory.  Scratch is passed in through
+ *    `workspace` (size from hs_workspace_size; NULL allowed when that is 0).
+ *  - Every pointer must be 16-byte aligned.  Tensors are dense, row-major,
+ *    with the innermost dimension = head_dim:
+ *        q, o, q_sparse, o_global, o_local   [batch][hq ][t_q ][head_dim]
+ *        k, v, k_f, v_f, k_local, v_local     [batch][hkv][t_kv][head_dim]
+ *        lse, lse_global, lse_local          [batch][hq ][t_q ]            fp32 (natural log)
+ *        idx                                 [batch][hkv][t_q ][ksel]      int32
+ *        idx_count                           [batch][hkv][t_q ]            int32
+ *    where ksel = k / block_size (block mode) or k (token mode).  Query head h
+ *    belongs to KV group u = h / (hq / hkv).  Decode uses t_q = 1 and
+ *    t_kv = cache capacity (the row stride of the cache).
+ *  - Positions are 0-based and causal: query row j sits at position
+ *    t = q_offset + j and sees keys 0..t (t < t_kv required).
+ *  - Index sets are written in ascending order and padded with -1;
+ *    idx_count holds the number of valid entries.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream).  Argument errors are detected on the host before any
+ *    launch and returned synchronously; nothing is launched then.  A failed
+ *    launch returns HS_ERR_CUDA.  Errors found on the device (an index or
+ *    sequence length out of range) skip the offending row and set a sticky
+ *    per-device status word that hs_device_status reads.  No kernel traps.
+ *  - Supported: head_dim in {64, 128}; hq % hkv == 0 with hq/hkv <= 16;
+ *    block mode: block_size in {16, 32, 64, 128}, k % block_size == 0,
+ *    k/block_size <= 64; token mode: 0 <= window <= k <= 4096;
+ *    dtype fp32 or bf16 (decode: bf16 only).
+ */
+#ifndef HS_H_
+#define HS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HS_OK = 0,
+    HS_ERR_INVALID_ARG = 1, /* a pointer, shape or knob is out of range        */
+    HS_ERR_UNSUPPORTED = 2, /* valid, but not a shape this build implements   */
+    HS_ERR_CUDA = 3,        /* a CUDA launch or runtime call failed           */
+    HS_ERR_TIMEOUT = 4,     /* a bounded device wait gave up                  */
+    HS_ERR_BOUNDS = 5,      /* a device-side index / length was out of range  */
+    HS_ERR_WORKSPACE = 6    /* workspace missing or smaller than required     */
+} hs_status;
+
+typedef enum { HS_BF16 = 0, HS_FP32 = 1 } hs_dtype;
+
+/* Selection granularity: HySparse blocks of B keys, or HySparse2 tokens with
+ * the most recent `window` tokens always selected. */
+typedef enum { HS_SEL_BLOCK = 0, HS_SEL_TOKEN = 1 } hs_sel_mode;
+
+typedef struct {
+    int32_t batch;      /* b                                                   */
+    int32_t hq;         /* query heads                                         */
+    int32_t hkv;        /* key/value heads (GQA groups)                        */
+    int32_t head_dim;   /* d                                                   */
+    int32_t t_q;        /* query rows per (batch, head)                        */
+    int32_t t_kv;       /* key rows per (batch, kv head); decode: capacity     */
+    int32_t q_offset;   /* position of query row 0 (chunked prefill)           */
+    int32_t dtype;      /* hs_dtype of q, k, v and of the outputs o            */
+    int32_t mode;       /* hs_sel_mode                                         */
+    int32_t block_size; /* B (block mode)                                      */
+    int32_t k;          /* token budget; token mode: total, window included    */
+    int32_t window;     /* w (token mode: forced window; block mode: SWA width) */
+    float scale;        /* softmax scale; 0 -> 1/sqrt(head_dim)                */
+} hs_params;
+
+/*
+ * Full-attention layer + oracle indexer (prefill, or a prefill chunk).
+ *
+ * For every query row and head:  o = softmax(scale q K^T, causal) V and
+ * lse = log sum exp(scale q K^T).  For every query row and KV group u it
+ * writes the index set I_t:
+ *   block mode: the k/B blocks with the largest group score
+ *               S_bar_{t,r} = max_{h in u} max_{i in block r, i<=t} p_{h,t,i};
+ *   token mode: {max(0,t-w+1)..t} plus the k-w keys of 0..t-w with the largest
+ *               S_bar_{t,i} = max_{h in u} p_{h,t,i}.
+ * When every candidate fits in the budget, all of them are selected.  Equal
+ * scores go to the lower index.  No T x T (or T x T/B) matrix is written.
+ *
+ * q, k, v:    inputs (layouts above).  o, lse: outputs.
+ * idx, idx_count: outputs (ascending, -1 padded).
+ * sel_scores: optional output [batch][hkv][t_q][ksel] fp32, the S_bar of each
+ *             selected entry (0 in the padding); NULL to skip.
+ * workspace:  hs_workspace_size(p, HS_WS_FULL) bytes (may be 0 / NULL).
+ */
+hs_status hs_full_attn_index(const hs_params* p, const void* q, const void* k,
+                             const void* v, void* o, float* lse, int32_t* idx,
+                             int32_t* idx_count, float* sel_scores, void* workspace,
+                             size_t ws_bytes, void* stream);
+
+/*
+ * Sparse layer reusing the full layer's K^F, V^F and index set, with its own
+ * query q_sparse:  o_global = softmax over R_t of (scale q' k_i) v_i, where R_t is
+ * the selected tokens (token mode) or the keys of the selected blocks clipped
+ * to i <= t (block mode).
+ * When k_local / v_local are non-NULL (block mode), the local branch is also
+ * computed: causal softmax attention of q' over the layer's OWN k_local,
+ * v_local restricted to keys max(0,t-w+1)..t, into o_local / lse_local.
+ * The two branches are returned unfused (the sigmoid gate needs trained
+ * weights and is the caller's).  A row whose index set is empty gets o = 0 and
+ * lse = -inf.  idx entries out of range set HS_ERR_BOUNDS on the device.
+ */
+hs_status hs_sparse_attn_reuse(const hs_params* p, const void* q_sparse, const void* k_f,
+                               const void* v_f, const int32_t* idx,
+                               const int32_t* idx_count, const void* k_local,
+                               const void* v_local, void* o_global, float* lse_global,
+                               void* o_local, float* lse_local, void* workspace,
+                               size_t ws_bytes, void* stream);
+
+typedef enum { HS_DECODE_FULL_INDEX = 0, HS_DECODE_SPARSE = 1 } hs_decode_kind;
+
+/*
+ * One decode step for a batch of sequences, bf16, token mode
+ * ("HySparse 混合稀疏注意力（一）": at step t the new token first passes the full
+ * layer, which selects for position t, then the block's sparse layers).
+ *
+ * q:        [batch][hq][1][head_dim], the new token's query.
+ * k_cache, v_cache: [batch][hkv][t_kv][head_dim]; the caller has already
+ *           written the new token's k/v at row seq_len[b]-1.
+ * seq_len:  DEVICE int32 [batch], 1 <= seq_len[b] <= t_kv (new token included).
+ * HS_DECODE_FULL_INDEX: writes o, lse and idx/idx_count [batch][hkv][ksel]
+ *           for position seq_len[b]-1 (same rule as hs_full_attn_index).
+ * HS_DECODE_SPARSE: reads idx/idx_count and writes o (and lse) of the sparse
+ *           layer with query q over K^F = k_cache, V^F = v_cache.
+ * sel_scores: optional (FULL_INDEX only), as in hs_full_attn_index.
+ * workspace: hs_workspace_size(p, HS_WS_DECODE_FULL / HS_WS_DECODE_SPARSE).
+ * The caller keeps k_cache, v_cache and idx alive until the last sparse layer
+ * of the block has run.
+ */
+hs_status hs_decode_step(const hs_params* p, int32_t kind, const void* q,
+                         const void* k_cache, const void* v_cache, const int32_t* seq_len,
+                         int32_t* idx, int32_t* idx_count, void* o, float* lse,
+                         float* sel_scores, void* workspace, size_t ws_bytes, void* stream);
+
+enum { HS_WS_FULL = 0, HS_WS_SPARSE = 1, HS_WS_DECODE_FULL = 2, HS_WS_DECODE_SPARSE = 3 };
+
+/* Bytes of workspace the matching entry point needs for these parameters
+ * (0 when none).  Returns (size_t)-1 for invalid parameters. */
+size_t hs_workspace_size(const hs_params* p, int32_t which);
+
+/* Waits for `stream`, then returns in *out the sticky device status word of
+ * the current device (an hs_status value, HS_OK if nothing went wrong) and
+ * clears it.  Returns HS_ERR_CUDA if the wait or the read failed. */
+hs_status hs_device_status(void* stream, int32_t* out);
+
+/* Static, human-readable name of a status code. */
+const char* hs_status_string(int32_t status);
+
+/* Number of kernels this library has launched in this process so far (all
+ * devices, all streams).  A diagnostic for callers that account for launches;
+ * it counts successful launch calls, not completed kernels. */
+uint64_t hs_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HS_H_ */

@@ -1,0 +1,222 @@
+// decode_full.cu -- decode step of the full-attention layer acting as the
+// oracle indexer ("HySparse 混合稀疏注意力（一）": at decode step t the new token
+// first passes the full layer, which selects for position t; cost model
+// "Decode：关键收益来自少读 KV": the full layer streams the whole cache).
+//
+// Three launches per step:
+//  1. decode_full_split_kernel: one warp per (sequence, kv group, 2048-key
+//     split) streams its slice of the cache once; the group's heads are the
+//     16 MMA rows.  It keeps an online-softmax partial (m, l, O) per head and
+//     exports every scaled logit a2_{h,i} (log2 domain) to the workspace,
+//     because the group score max_h (a2_{h,i} - lse2_h) needs every head's
+//     final lse, known only after all splits;
+//  2. the exact log-sum-exp merge of the splits (shared with the sparse
+//     decode) -> o, lse, and lse2 for the selector;
+//  3. decode_select_kernel: one CTA per (sequence, group) ranks keys
+//     0..t-w by max_h (a2_{h,i} - lse2_h) (= log2 of max_h p_{h,t,i}) with the
+//     exact streaming top-k and appends the forced window t-w+1..t
+//     ("HySparse2 ..." 4.2).
+#include "attend_mma.cuh"
+#include "block_topk.cuh"
+#include "hs_common.cuh"
+#include "hs_kernels.cuh"
+
+namespace hs {
+
+cudaError_t launch_decode_combine(const KParams& p, const float* part, int n_split,
+                                  const int32_t* seq_len, void* o, float* lse, float* lse2,
+                                  cudaStream_t st);
+
+constexpr int kDecodeKeys = 2048;  // cache keys per split
+constexpr int kDecodeWarps = 4;
+constexpr int kSelectThreads = 512;
+
+struct DecodeWs {
+    float* logits;  // [batch*hkv][t_kv][16]
+    float* part;    // [batch*hkv][n_split][16][D+2]
+    float* lse2;    // [batch*hq]
+    int n_split;
+};
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+static DecodeWs decode_ws_layout(const KParams& p, void* base) {
+    DecodeWs w;
+    w.n_split = (p.t_kv + kDecodeKeys - 1) / kDecodeKeys;
+    const size_t units = (size_t)p.batch * p.hkv;
+    const size_t logits_b = align256(units * p.t_kv * 16 * sizeof(float));
+    const size_t part_b = align256(units * w.n_split * 16 * (p.head_dim + 2) * sizeof(float));
+    char* c = static_cast<char*>(base);
+    w.logits = reinterpret_cast<float*>(c);
+    w.part = reinterpret_cast<float*>(c + logits_b);
+    w.lse2 = reinterpret_cast<float*>(c + logits_b + part_b);
+    return w;
+}
+
+size_t decode_full_workspace(const KParams& p) {
+    const int n_split = (p.t_kv + kDecodeKeys - 1) / kDecodeKeys;
+    const size_t units = (size_t)p.batch * p.hkv;
+    return align256(units * p.t_kv * 16 * sizeof(float)) +
+           align256(units * n_split * 16 * (p.head_dim + 2) * sizeof(float)) +
+           align256((size_t)p.batch * p.hq * sizeof(float));
+}
+
+template <int D>
+struct LogitExport {
+    float* logits;  // this unit's [t_kv][16]
+    int first, last, g;
+    __device__ __forceinline__ void operator()(int c, float (&s)[4][4], int) const {
+        const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int h = gid + 8 * (e >> 1);
+                const int key = first + c * kChunk + n * 8 + tig * 2 + (e & 1);
+                if (h < g && key <= last) logits[(size_t)key * 16 + h] = s[n][e];
+            }
+        }
+    }
+};
+
+template <int D>
+__global__ void __launch_bounds__(kDecodeWarps * 32)
+    decode_full_split_kernel(KParams p, const __nv_bfloat16* __restrict__ q,
+                             const __nv_bfloat16* __restrict__ kc,
+                             const __nv_bfloat16* __restrict__ vc,
+                             const int32_t* __restrict__ seq_len, DecodeWs ws) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    const int warp = threadIdx.x >> 5;
+    const int task = blockIdx.x * kDecodeWarps + warp;
+    if (task >= p.batch * p.hkv * ws.n_split) return;
+    const int sp = task % ws.n_split;
+    const int unit = task / ws.n_split;
+    const int u = unit % p.hkv, b = unit / p.hkv;
+    const int g = p.group;
+    const int L = seq_len[b];
+    AttnState<D> st;
+    st.init();
+    const int first = sp * kDecodeKeys;
+    if (L >= 1 && L <= p.t_kv && first < L) {
+        const int last = min(L - 1, first + kDecodeKeys - 1);
+        const uint32_t sbase = smem_u32(smem_raw) + warp * WarpSmem<D>::kBytes;
+        uint32_t qf[D / 16][4];
+        load_q_frags<D>(qf, q + ((size_t)b * p.hq + u * g) * D, D, g);
+        const size_t kvoff = (size_t)unit * p.t_kv * D;
+        LogitExport<D> hook{ws.logits + (size_t)unit * p.t_kv * 16, first, last, g};
+        attend_rows<D>(st, qf, kc + kvoff, vc + kvoff, last - first + 1,
+                       ContiguousKeys{first, last}, sbase, p.scale_log2, hook);
+    }
+    store_partial<D>(st, ws.part + (size_t)task * 16 * (D + 2), g);
+}
+
+__global__ void __launch_bounds__(kSelectThreads)
+    decode_select_kernel(KParams p, const int32_t* __restrict__ seq_len, DecodeWs ws,
+                         int32_t* __restrict__ idx, int32_t* __restrict__ cnt,
+                         float* __restrict__ sel) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    __shared__ int s_count;
+    __shared__ unsigned long long s_thresh;
+    __shared__ float s_lse2[16];
+    const int unit = blockIdx.x;
+    const int u = unit % p.hkv, b = unit / p.hkv;
+    const int g = p.group;
+    const int L = seq_len[b];
+    int32_t* irow = idx + (size_t)unit * p.ksel;
+    float* srow = sel ? sel + (size_t)unit * p.ksel : nullptr;
+    if (L < 1 || L > p.t_kv) {
+        for (int x = threadIdx.x; x < p.ksel; x += blockDim.x) {
+            irow[x] = -1;
+            if (srow) srow[x] = 0.f;
+        }
+        if (threadIdx.x == 0) { cnt[unit] = 0; set_status(HS_ERR_BOUNDS); }
+        return;
+    }
+    const int t = L - 1;
+    const int Kc = p.k - p.window;
+    BlockTopK topk;
+    topk.setup(smem_raw, Kc, blockDim.x, &s_count, &s_thresh);
+    if (threadIdx.x < 16) s_lse2[threadIdx.x] = threadIdx.x < g ? ws.lse2[b * p.hq + u * g + threadIdx.x] : 0.f;
+    __syncthreads();
+
+    const bool select_all = t + 1 <= p.k;
+    const int lo = t - p.window + 1;
+    const bool ranked = !select_all && Kc > 0;
+    int n_scored;
+    if (select_all) n_scored = srow ? t + 1 : 0;
+    else n_scored = srow ? t + 1 : lo;
+    const float* lg = ws.logits + (size_t)unit * p.t_kv * 16;
+
+    for (int c0 = 0; c0 < n_scored; c0 += blockDim.x) {
+        const int i = c0 + threadIdx.x;
+        if (i < n_scored) {
+            const float4* r4 = reinterpret_cast<const float4*>(lg + (size_t)i * 16);
+            float s = -INFINITY;
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                if (q4 * 4 >= g) break;
+                const float4 a = r4[q4];
+                const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (q4 * 4 + e < g) s = fmaxf(s, av[e] - s_lse2[q4 * 4 + e]);
+            }
+            if (select_all) srow[i] = exp2f(s);
+            else if (i >= lo) { if (srow) srow[Kc + (i - lo)] = exp2f(s); }
+            else if (ranked) topk.offer(s, (uint32_t)i);
+        }
+        if (ranked) topk.end_round();
+    }
+    __syncthreads();
+    if (threadIdx.x >= 32) return;
+    int n_out;
+    if (select_all) {
+        n_out = t + 1;
+        for (int x = threadIdx.x; x < n_out; x += 32) irow[x] = x;
+        for (int x = n_out + threadIdx.x; x < p.ksel; x += 32) {
+            irow[x] = -1;
+            if (srow) srow[x] = 0.f;
+        }
+    } else {
+        n_out = topk.finish(irow, srow, p.ksel, lo, t);
+    }
+    if (threadIdx.x == 0) cnt[unit] = n_out;
+}
+
+template <int D>
+static cudaError_t launch_decode_full_t(const KParams& p, const void* q, const void* kc,
+                                        const void* vc, const int32_t* seq_len, int32_t* idx,
+                                        int32_t* cnt, void* o, float* lse, float* sel, void* ws,
+                                        cudaStream_t st) {
+    DecodeWs w = decode_ws_layout(p, ws);
+    const size_t smem = (size_t)kDecodeWarps * WarpSmem<D>::kBytes;
+    auto kern = decode_full_split_kernel<D>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int n_tasks = p.batch * p.hkv * w.n_split;
+    kern<<<(n_tasks + kDecodeWarps - 1) / kDecodeWarps, kDecodeWarps * 32, smem, st>>>(
+        p, (const __nv_bfloat16*)q, (const __nv_bfloat16*)kc, (const __nv_bfloat16*)vc, seq_len,
+        w);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_decode_combine(p, w.part, w.n_split, seq_len, o, lse, w.lse2, st)) !=
+        cudaSuccess)
+        return e;
+    const size_t sel_smem = BlockTopK::smem_bytes(p.k - p.window, kSelectThreads);
+    e = cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sel_smem);
+    if (e != cudaSuccess) return e;
+    decode_select_kernel<<<p.batch * p.hkv, kSelectThreads, sel_smem, st>>>(p, seq_len, w, idx,
+                                                                           cnt, sel);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_full(const KParams& p, const void* q, const void* kc, const void* vc,
+                               const int32_t* seq_len, int32_t* idx, int32_t* cnt, void* o,
+                               float* lse, float* sel, void* ws, cudaStream_t st) {
+    if (p.head_dim == 64)
+        return launch_decode_full_t<64>(p, q, kc, vc, seq_len, idx, cnt, o, lse, sel, ws, st);
+    return launch_decode_full_t<128>(p, q, kc, vc, seq_len, idx, cnt, o, lse, sel, ws, st);
+}
+
+}  // namespace hs

@@ -1,0 +1,223 @@
+// hs_api.cu -- the C ABI declared in include/hs.h: argument validation,
+// kernel selection and launch, workspace sizing and the device status word.
+//
+// The whole library is one translation unit (the kernel files are included
+// below), so the sticky status word defined in hs_common.cuh is a single
+// __device__ symbol without relocatable device code.
+#include <math.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "../../include/hs.h"
+#include "hs_common.cuh"
+#include "hs_kernels.cuh"
+
+#include "decode_full.cu"
+#include "full_simt.cu"
+#include "sparse.cu"
+
+namespace hs {
+static std::atomic<uint64_t> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace hs
+
+namespace {
+
+using hs::KParams;
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+bool ok_ptr(const void* ptr) { return ptr != nullptr && aligned16(ptr); }
+bool ok_opt(const void* ptr) { return ptr == nullptr || aligned16(ptr); }
+
+// Common shape / knob checks.  Returns HS_OK and fills kp on success.
+hs_status resolve(const hs_params* p, bool decode, KParams* kp) {
+    if (!p) return HS_ERR_INVALID_ARG;
+    if (p->batch < 1 || p->hq < 1 || p->hkv < 1 || p->t_q < 0 || p->t_kv < 1 || p->q_offset < 0)
+        return HS_ERR_INVALID_ARG;
+    if (p->hq % p->hkv != 0) return HS_ERR_INVALID_ARG;
+    if (p->dtype != HS_BF16 && p->dtype != HS_FP32) return HS_ERR_INVALID_ARG;
+    if (p->mode != HS_SEL_BLOCK && p->mode != HS_SEL_TOKEN) return HS_ERR_INVALID_ARG;
+    if (!(p->scale >= 0.f) || !isfinite(p->scale)) return HS_ERR_INVALID_ARG;
+    if (p->k < 1 || p->window < 0) return HS_ERR_INVALID_ARG;
+    int ksel;
+    if (p->mode == HS_SEL_BLOCK) {
+        if (p->block_size < 1 || p->k % p->block_size != 0) return HS_ERR_INVALID_ARG;
+        ksel = p->k / p->block_size;
+    } else {
+        if (p->window > p->k) return HS_ERR_INVALID_ARG;
+        ksel = p->k;
+    }
+    if (decode) {
+        if (p->t_q != 1) return HS_ERR_INVALID_ARG;
+    } else if ((long long)p->q_offset + p->t_q > p->t_kv) {
+        return HS_ERR_INVALID_ARG;
+    }
+    // element counts must stay far from overflow
+    const double big = (double)p->batch * p->hq * (double)(p->t_kv > p->t_q ? p->t_kv : p->t_q) *
+                       (p->head_dim > 0 ? p->head_dim : 1);
+    if (big > 4.0e15) return HS_ERR_INVALID_ARG;
+    // what this build implements
+    const int g = p->hq / p->hkv;
+    if (p->head_dim != 64 && p->head_dim != 128) return HS_ERR_UNSUPPORTED;
+    if (g > 16) return HS_ERR_UNSUPPORTED;
+    if (p->mode == HS_SEL_BLOCK) {
+        const int B = p->block_size;
+        if (B != 16 && B != 32 && B != 64 && B != 128) return HS_ERR_UNSUPPORTED;
+        if (ksel > 64) return HS_ERR_UNSUPPORTED;
+    } else if (p->k > 4096) {
+        return HS_ERR_UNSUPPORTED;
+    }
+    kp->batch = p->batch;
+    kp->hq = p->hq;
+    kp->hkv = p->hkv;
+    kp->group = g;
+    kp->head_dim = p->head_dim;
+    kp->t_q = p->t_q;
+    kp->t_kv = p->t_kv;
+    kp->q_offset = decode ? 0 : p->q_offset;
+    kp->mode = p->mode;
+    kp->block_size = p->mode == HS_SEL_BLOCK ? p->block_size : 1;
+    kp->k = p->k;
+    kp->window = p->window;
+    kp->ksel = ksel;
+    const float scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->head_dim);
+    kp->scale_log2 = scale * hs::kLog2e;
+    return HS_OK;
+}
+
+hs_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HS_OK : HS_ERR_CUDA; }
+
+// Launch a sequence through fn() and count its kernels when it succeeds.
+template <typename Fn>
+hs_status launched(int n_kernels, Fn fn) {
+    const cudaError_t e = fn();
+    if (e == cudaSuccess) hs::count_launches(n_kernels);
+    return from_cuda(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+hs_status hs_full_attn_index(const hs_params* p, const void* q, const void* k, const void* v,
+                             void* o, float* lse, int32_t* idx, int32_t* idx_count,
+                             float* sel_scores, void* workspace, size_t ws_bytes, void* stream) {
+    (void)workspace;
+    (void)ws_bytes;
+    KParams kp;
+    hs_status s = resolve(p, false, &kp);
+    if (s != HS_OK) return s;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(o) || !ok_ptr(lse) || !ok_ptr(idx) ||
+        !ok_ptr(idx_count) || !ok_opt(sel_scores))
+        return HS_ERR_INVALID_ARG;
+    if (kp.t_q == 0) return HS_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return launched(1, [&] {
+        return hs::launch_full_simt(kp, p->dtype, q, k, v, o, lse, idx, idx_count, sel_scores,
+                                    st);
+    });
+}
+
+hs_status hs_sparse_attn_reuse(const hs_params* p, const void* q_sparse, const void* k_f,
+                               const void* v_f, const int32_t* idx, const int32_t* idx_count,
+                               const void* k_local, const void* v_local, void* o_global,
+                               float* lse_global, void* o_local, float* lse_local,
+                               void* workspace, size_t ws_bytes, void* stream) {
+    (void)workspace;
+    (void)ws_bytes;
+    KParams kp;
+    hs_status s = resolve(p, false, &kp);
+    if (s != HS_OK) return s;
+    if (!ok_ptr(q_sparse) || !ok_ptr(k_f) || !ok_ptr(v_f) || !ok_ptr(idx) || !ok_ptr(idx_count) ||
+        !ok_ptr(o_global) || !ok_ptr(lse_global))
+        return HS_ERR_INVALID_ARG;
+    const bool local = k_local != nullptr || v_local != nullptr;
+    if (local && (!ok_ptr(k_local) || !ok_ptr(v_local) || !ok_ptr(o_local) || !ok_ptr(lse_local)))
+        return HS_ERR_INVALID_ARG;
+    if (local && p->window < 1) return HS_ERR_INVALID_ARG;
+    if (kp.t_q == 0) return HS_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (p->dtype == HS_FP32)
+        return launched(1, [&] {
+            return hs::launch_sparse_simt(kp, p->dtype, q_sparse, k_f, v_f, idx, idx_count,
+                                          local ? k_local : nullptr, v_local, o_global,
+                                          lse_global, o_local, lse_local, st);
+        });
+    return launched(1, [&] {
+        return hs::launch_sparse_mma(kp, q_sparse, k_f, v_f, idx, idx_count,
+                                     local ? k_local : nullptr, v_local, o_global, lse_global,
+                                     o_local, lse_local, st);
+    });
+}
+
+size_t hs_workspace_size(const hs_params* p, int32_t which) {
+    KParams kp;
+    const bool decode = which == HS_WS_DECODE_FULL || which == HS_WS_DECODE_SPARSE;
+    if (which < HS_WS_FULL || which > HS_WS_DECODE_SPARSE) return (size_t)-1;
+    if (resolve(p, decode, &kp) != HS_OK) return (size_t)-1;
+    switch (which) {
+        case HS_WS_DECODE_FULL: return hs::decode_full_workspace(kp);
+        case HS_WS_DECODE_SPARSE: return hs::decode_sparse_workspace(kp);
+        default: return 0;
+    }
+}
+
+hs_status hs_decode_step(const hs_params* p, int32_t kind, const void* q, const void* k_cache,
+                         const void* v_cache, const int32_t* seq_len, int32_t* idx,
+                         int32_t* idx_count, void* o, float* lse, float* sel_scores,
+                         void* workspace, size_t ws_bytes, void* stream) {
+    KParams kp;
+    hs_status s = resolve(p, true, &kp);
+    if (s != HS_OK) return s;
+    if (kind != HS_DECODE_FULL_INDEX && kind != HS_DECODE_SPARSE) return HS_ERR_INVALID_ARG;
+    if (p->dtype != HS_BF16 || p->mode != HS_SEL_TOKEN) return HS_ERR_UNSUPPORTED;
+    if (!ok_ptr(q) || !ok_ptr(k_cache) || !ok_ptr(v_cache) || !ok_ptr(seq_len) || !ok_ptr(idx) ||
+        !ok_ptr(idx_count) || !ok_ptr(o) || !ok_opt(lse) || !ok_opt(sel_scores))
+        return HS_ERR_INVALID_ARG;
+    const size_t need = kind == HS_DECODE_FULL_INDEX ? hs::decode_full_workspace(kp)
+                                                     : hs::decode_sparse_workspace(kp);
+    if (need > 0 && (workspace == nullptr || ws_bytes < need || !aligned16(workspace)))
+        return HS_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (kind == HS_DECODE_FULL_INDEX) {
+        if (!lse) return HS_ERR_INVALID_ARG;
+        return launched(3, [&] {
+            return hs::launch_decode_full(kp, q, k_cache, v_cache, seq_len, idx, idx_count, o,
+                                          lse, sel_scores, workspace, st);
+        });
+    }
+    return launched(2, [&] {
+        return hs::launch_decode_sparse(kp, q, k_cache, v_cache, seq_len, idx, idx_count, o, lse,
+                                        workspace, st);
+    });
+}
+
+hs_status hs_device_status(void* stream, int32_t* out) {
+    if (!out) return HS_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return HS_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, hs::g_status, sizeof(int)) != cudaSuccess) return HS_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(hs::g_status, &zero, sizeof(int)) != cudaSuccess) return HS_ERR_CUDA;
+    *out = v;
+    return HS_OK;
+}
+
+uint64_t hs_launch_count(void) { return hs::g_launches.load(std::memory_order_relaxed); }
+
+const char* hs_status_string(int32_t status) {
+    switch (status) {
+        case HS_OK: return "HS_OK";
+        case HS_ERR_INVALID_ARG: return "HS_ERR_INVALID_ARG";
+        case HS_ERR_UNSUPPORTED: return "HS_ERR_UNSUPPORTED";
+        case HS_ERR_CUDA: return "HS_ERR_CUDA";
+        case HS_ERR_TIMEOUT: return "HS_ERR_TIMEOUT";
+        case HS_ERR_BOUNDS: return "HS_ERR_BOUNDS";
+        case HS_ERR_WORKSPACE: return "HS_ERR_WORKSPACE";
+        default: return "HS_UNKNOWN_STATUS";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,219 @@
+// hs_common.cuh -- device helpers shared by the sm_100a kernels of the
+// HySparse / HySparse2 hot path: element I/O, warp reductions, the sticky
+// device status word, mma.sync / ldmatrix / cp.async wrappers, and the exact
+// streaming top-k candidate buffer used by every selection step.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/hs.h"
+
+namespace hs {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// Sticky per-device status word (first error wins).  Set by kernels that find
+// an out-of-range index or length; read and cleared by hs_device_status.
+__device__ int g_status = 0;
+
+__device__ __forceinline__ void set_status(int code) { atomicCAS(&g_status, 0, code); }
+
+// ---------------------------------------------------------------- element I/O
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// ---------------------------------------------------------------- warp helpers
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Sortable image of a float: larger float <-> larger unsigned.
+__device__ __forceinline__ uint32_t float_order(float f) {
+    uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float order_float(uint32_t u) {
+    return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+// Composite selection key: larger = better.  High word: the score; low word:
+// the complement of the id, so that equal scores prefer the LOWER id.
+__device__ __forceinline__ uint64_t sel_key(float score, uint32_t id) {
+    return ((uint64_t)float_order(score) << 32) | (uint64_t)(0xffffffffu - id);
+}
+__device__ __forceinline__ uint32_t sel_key_id(uint64_t key) {
+    return 0xffffffffu - (uint32_t)(key & 0xffffffffu);
+}
+__device__ __forceinline__ float sel_key_score(uint64_t key) {
+    return order_float((uint32_t)(key >> 32));
+}
+
+// ---------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+    // valid == false zero-fills the 16 destination bytes without reading src.
+    const int n = valid ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(n));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n"); }
+template <int N> __device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+// D = A(16x16 bf16, row) * B(16x8 bf16, col) + D (fp32)
+__device__ __forceinline__ void mma_bf16(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Byte offset of 16-byte chunk `chunk` of row `row` in a tile whose rows are
+// `row_bytes` long, with the chunk index XOR-swizzled by the row so that
+// ldmatrix over 8 consecutive rows touches 8 distinct bank groups.
+__device__ __forceinline__ uint32_t swz(int row, int chunk, int row_bytes) {
+    return (uint32_t)(row * row_bytes + ((chunk ^ (row & 7)) << 4));
+}
+
+// ------------------------------------------------- exact streaming top-k buffer
+//
+// One selection = the K best (score, id) pairs under "higher score first,
+// lower id on ties".  Candidates are appended to a shared-memory buffer of
+// capacity `cap` (>= 2K) as 64-bit composite keys (sel_key).  When the buffer
+// runs full, the buffer is cut to its K best, and `thresh` becomes the K-th
+// best key: a later candidate can only enter the final K if its key is above
+// it, so nothing that could still be selected is ever dropped.
+
+// K-th largest of n unique keys (1 <= K <= n), computed by one warp with an
+// 8-bit-digit radix select.  hist: 256 words of shared scratch for this warp.
+__device__ __forceinline__ uint64_t warp_kth_largest(const uint64_t* buf, int n, int K,
+                                                     uint32_t* hist) {
+    const int lane = threadIdx.x & 31;
+    uint64_t prefix = 0, mask = 0;
+    int need = K;
+    for (int shift = 56; shift >= 0; shift -= 8) {
+#pragma unroll
+        for (int x = 0; x < 8; ++x) hist[lane * 8 + x] = 0;
+        __syncwarp();
+        for (int i = lane; i < n; i += 32) {
+            const uint64_t key = buf[i];
+            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1u);
+        }
+        __syncwarp();
+        // lane L owns bins 255-8L .. 248-8L (descending).  Count above each bin.
+        uint32_t own[8];
+        uint32_t s = 0;
+#pragma unroll
+        for (int x = 0; x < 8; ++x) { own[x] = hist[255 - (lane * 8 + x)]; s += own[x]; }
+        uint32_t incl = s;  // inclusive prefix over lanes (lane 0 = highest bins)
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        uint32_t above = incl - s;  // keys in bins higher than this lane's bins
+        int digit = -1;
+        uint32_t above_digit = 0;
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+            if (digit < 0 && above < (uint32_t)need && above + own[x] >= (uint32_t)need) {
+                digit = 255 - (lane * 8 + x);
+                above_digit = above;
+            }
+            above += own[x];
+        }
+        const uint32_t found = __ballot_sync(0xffffffffu, digit >= 0);
+        const int src = __ffs(found) - 1;
+        digit = __shfl_sync(0xffffffffu, digit, src);
+        above_digit = __shfl_sync(0xffffffffu, above_digit, src);
+        prefix |= (uint64_t)digit << shift;
+        mask |= (uint64_t)255 << shift;
+        need -= (int)above_digit;
+        __syncwarp();
+    }
+    return prefix;
+}
+
+// Keep only keys >= kth (in place, order not preserved); returns the new count.
+__device__ __forceinline__ int warp_keep_at_least(uint64_t* buf, int n, uint64_t kth) {
+    const int lane = threadIdx.x & 31;
+    int out = 0;
+    for (int base = 0; base < n; base += 32) {
+        const int i = base + lane;
+        uint64_t key = 0;
+        bool keep = false;
+        if (i < n) { key = buf[i]; keep = key >= kth; }
+        const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+        __syncwarp();
+        if (keep) buf[out + __popc(bal & ((1u << lane) - 1))] = key;
+        out += __popc(bal);
+        __syncwarp();
+    }
+    return out;
+}
+
+// Cut the buffer to its K best keys; returns the K-th best key (the new
+// admission threshold).  Requires n > K.
+__device__ __forceinline__ uint64_t warp_cut_to_k(uint64_t* buf, int n, int K, uint32_t* hist) {
+    const uint64_t kth = warp_kth_largest(buf, n, K, hist);
+    warp_keep_at_least(buf, n, kth);
+    return kth;
+}
+
+// In-place ascending bitonic sort of n_pow2 values by one warp.
+template <typename U>
+__device__ __forceinline__ void warp_bitonic_sort(U* a, int n_pow2) {
+    const int lane = threadIdx.x & 31;
+    for (int size = 2; size <= n_pow2; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int t = lane; t < (n_pow2 >> 1); t += 32) {
+                const int i = 2 * t - (t & (stride - 1));
+                const int j = i + stride;
+                const bool up = (i & size) == 0;
+                const U x = a[i], y = a[j];
+                if ((x > y) == up) { a[i] = y; a[j] = x; }
+            }
+            __syncwarp();
+        }
+    }
+}
+
+__host__ __device__ constexpr int next_pow2(int x) {
+    int p = 1;
+    while (p < x) p <<= 1;
+    return p;
+}
+
+}  // namespace hs

@@ -1,0 +1,49 @@
+// hs_kernels.cuh -- launch parameters and host-side launchers shared between
+// the C-ABI layer (hs_api.cu) and the kernel translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace hs {
+
+// Host-side count of kernel launches issued by this library (hs_launch_count).
+void count_launches(int n);
+
+// Resolved, validated parameters handed to every kernel (by value).
+struct KParams {
+    int batch, hq, hkv, group, head_dim;
+    int t_q, t_kv, q_offset;
+    int mode;        // 0 block, 1 token
+    int block_size;  // B (1 in token mode)
+    int k, window;
+    int ksel;        // entries per index row
+    float scale_log2;  // softmax scale * log2(e)
+};
+
+cudaError_t launch_full_simt(const KParams& p, int dtype, const void* q, const void* k,
+                             const void* v, void* o, float* lse, int32_t* idx, int32_t* cnt,
+                             float* sel, cudaStream_t st);
+
+cudaError_t launch_sparse_simt(const KParams& p, int dtype, const void* q, const void* kf,
+                               const void* vf, const int32_t* idx, const int32_t* cnt,
+                               const void* kl, const void* vl, void* og, float* lseg, void* ol,
+                               float* lsel, cudaStream_t st);
+
+// bf16 tensor-core paths (mma.sync fragments; d = 64 or 128).
+cudaError_t launch_sparse_mma(const KParams& p, const void* q, const void* kf, const void* vf,
+                              const int32_t* idx, const int32_t* cnt, const void* kl,
+                              const void* vl, void* og, float* lseg, void* ol, float* lsel,
+                              cudaStream_t st);
+
+// Decode (bf16, token mode).
+size_t decode_full_workspace(const KParams& p);
+size_t decode_sparse_workspace(const KParams& p);
+cudaError_t launch_decode_full(const KParams& p, const void* q, const void* kc, const void* vc,
+                               const int32_t* seq_len, int32_t* idx, int32_t* cnt, void* o,
+                               float* lse, float* sel, void* ws, cudaStream_t st);
+cudaError_t launch_decode_sparse(const KParams& p, const void* q, const void* kc, const void* vc,
+                                 const int32_t* seq_len, const int32_t* idx, const int32_t* cnt,
+                                 void* o, float* lse, void* ws, cudaStream_t st);
+
+}  // namespace hs

@@ -4,8 +4,11 @@ oracle on the same seeded inputs and compare them under the stated bars.
 Bars (written here once, used by every parity test):
   * index sets: identical, except candidates whose fp64 group score lies
     within 1e-3 relative of the k-th ranked score (near-ties);
-  * attention outputs: max-abs error <= 1e-4 for fp32 inputs, and
-    <= 1.5e-2 * RMS(oracle output) for bf16;
+  * attention outputs: max-abs error <= 1e-4 for fp32 inputs; for bf16,
+    every element of a head's output vector at a query row is within
+    1.5e-2 * RMS(that vector of the fp64 result) plus half a bf16 ulp of the
+    fp64 value -- the bar applies to the computed value, and storing it as
+    bf16 adds up to half an ulp that no bf16 output can avoid;
   * lse: |err| <= 1e-4 (fp32) / 2e-3 (bf16) -- the fp32 log-sum-exp of
     logits computed from the same (bf16-exact) inputs.
 The sparse layers are checked on the GPU's own index set (the oracle
@@ -40,16 +43,31 @@ def f64(t):
     return t.detach().to("cpu", torch.float64).numpy()
 
 
+def half_ulp_bf16(x):
+    """Half the spacing of bf16 numbers at |x| (8 significant bits)."""
+    _, e = np.frexp(np.abs(x))
+    return np.where(x == 0, 0.0, np.ldexp(1.0, e - 9))
+
+
 def check_o(got, want, dtype, what):
+    """got / want: [..., d] output vectors (one per query row and head)."""
     got = np.asarray(got, dtype=np.float64)
-    err = np.abs(got - want).max() if got.size else 0.0
+    if not got.size:
+        return 0.0
+    err = np.abs(got - want)
     if dtype == "fp32":
-        assert err <= O_TOL_FP32, f"{what}: max-abs {err:.3e} > {O_TOL_FP32}"
-    else:
-        rms = float(np.sqrt(np.mean(want ** 2)))
-        assert err <= O_TOL_BF16_REL_RMS * rms, (
-            f"{what}: max-abs {err:.3e} > {O_TOL_BF16_REL_RMS} * rms {rms:.3e}")
-    return err
+        e = err.max()
+        assert e <= O_TOL_FP32, f"{what}: max-abs {e:.3e} > {O_TOL_FP32}"
+        return e
+    rms = np.sqrt(np.mean(want ** 2, axis=-1, keepdims=True))
+    bound = O_TOL_BF16_REL_RMS * rms + half_ulp_bf16(want)
+    ratio = err / bound
+    worst = np.unravel_index(np.argmax(ratio), ratio.shape)
+    assert ratio.max() <= 1.0, (
+        f"{what}: element {worst} err {err[worst]:.3e} > bound {bound[worst]:.3e} "
+        f"(row rms {rms[worst[:-1]].item():.3e}, got {got[worst]:.5e}, want {want[worst]:.5e}); "
+        f"{int((ratio > 1).sum())} of {ratio.size} elements out")
+    return float((err / rms).max())
 
 
 def check_lse(got, want, dtype, what):

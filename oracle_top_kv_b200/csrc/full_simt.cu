@@ -38,7 +38,7 @@ __global__ void __launch_bounds__(512) full_simt_kernel(KParams p, const T* __re
                                                         float* __restrict__ lse,
                                                         int32_t* __restrict__ idx,
                                                         int32_t* __restrict__ cnt,
-                                                        float* __restrict__ sel) {
+                                                        float* __restrict__ sel, int do_attn) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     const int j = blockIdx.x, u = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -66,7 +66,11 @@ __global__ void __launch_bounds__(512) full_simt_kernel(KParams p, const T* __re
 
     // ---------------- phase A: exact attention, one warp per head
     constexpr int E = D / 32;
-    if (warp < g) {
+    if (!do_attn) {
+        // selection only: the attention (and lse) came from another kernel
+        if (threadIdx.x < g)
+            lse2[threadIdx.x] = lse[((size_t)b * p.hq + u * g + threadIdx.x) * p.t_q + j] * kLog2e;
+    } else if (warp < g) {
         const int h = u * g + warp;
         const float* qh = qs + warp * D;
         float m = -INFINITY, l = 0.f, acc[E];
@@ -161,7 +165,7 @@ __global__ void __launch_bounds__(512) full_simt_kernel(KParams p, const T* __re
 template <typename T, int D>
 static cudaError_t launch_full_simt_t(const KParams& p, const void* q, const void* k,
                                       const void* v, void* o, float* lse, int32_t* idx,
-                                      int32_t* cnt, float* sel, cudaStream_t st) {
+                                      int32_t* cnt, float* sel, int do_attn, cudaStream_t st) {
     const int nwarps = p.group < 4 ? 4 : p.group;
     const int Kc = p.mode == 0 ? p.ksel : p.k - p.window;
     const size_t smem = sizeof(float) * (p.group * D + 16) +
@@ -172,21 +176,21 @@ static cudaError_t launch_full_simt_t(const KParams& p, const void* q, const voi
     if (e != cudaSuccess) return e;
     dim3 grid(p.t_q, p.hkv, p.batch);
     kern<<<grid, nwarps * 32, smem, st>>>(p, (const T*)q, (const T*)k, (const T*)v, (T*)o, lse,
-                                           idx, cnt, sel);
+                                           idx, cnt, sel, do_attn);
     return cudaGetLastError();
 }
 
 cudaError_t launch_full_simt(const KParams& p, int dtype, const void* q, const void* k,
                              const void* v, void* o, float* lse, int32_t* idx, int32_t* cnt,
-                             float* sel, cudaStream_t st) {
+                             float* sel, int do_attn, cudaStream_t st) {
     if (dtype == HS_FP32) {
         if (p.head_dim == 64)
-            return launch_full_simt_t<float, 64>(p, q, k, v, o, lse, idx, cnt, sel, st);
-        return launch_full_simt_t<float, 128>(p, q, k, v, o, lse, idx, cnt, sel, st);
+            return launch_full_simt_t<float, 64>(p, q, k, v, o, lse, idx, cnt, sel, do_attn, st);
+        return launch_full_simt_t<float, 128>(p, q, k, v, o, lse, idx, cnt, sel, do_attn, st);
     }
     if (p.head_dim == 64)
-        return launch_full_simt_t<__nv_bfloat16, 64>(p, q, k, v, o, lse, idx, cnt, sel, st);
-    return launch_full_simt_t<__nv_bfloat16, 128>(p, q, k, v, o, lse, idx, cnt, sel, st);
+        return launch_full_simt_t<__nv_bfloat16, 64>(p, q, k, v, o, lse, idx, cnt, sel, do_attn, st);
+    return launch_full_simt_t<__nv_bfloat16, 128>(p, q, k, v, o, lse, idx, cnt, sel, do_attn, st);
 }
 
 }  // namespace hs

@@ -1,0 +1,501 @@
+// full_tc.cu -- full-attention layer + block-level oracle indexer on the
+// sm_100a tensor cores (tcgen05 MMA with TMEM accumulators, TMA-fed).
+//
+// What it computes ("HySparse 混合稀疏注意力（一）", "为什么不需要重新物化注意力
+// 矩阵"; "HySparse: ..." 3.2, Algorithm 1): flash attention over causal key
+// tiles of B_C = 64 keys, which in block mode are exactly the sparse blocks
+// (B = B_C).  The row max of each S tile, m~_ij, is the block's max logit;
+// S_ij = exp(m~_ij - lse_i) is its block score after the scan (the page's
+// corrected line 14).  Instead of writing the T x T/B score matrix, every row
+// keeps its 16 best (m~, block) pairs in registers; ranking within a head by
+// logit equals ranking by probability ("TopK 只需要排序，为什么还要归一化分数").
+// After the scan the heads of a GQA group are merged exactly: every member of
+// the group's top-K is in the list of the head that attains its max, so the
+// union of the lists, re-scored as m~ - lse_h, contains the answer
+// ("GQA 下为什么要组内共享索引": S_bar = max over the group's heads).
+//
+// Tile: 128 query rows = g heads x (128/g) positions of one KV group (rows are
+// head-major, exactly as one 4-D TMA box lands), so every K/V tile is loaded
+// once for the whole group.  Warp roles:
+//   warp 0      TMA producer (Q once; K and V tiles through a 3-stage ring)
+//   warp 1      TMEM owner and MMA issuer: S = Q K^T into one of two TMEM
+//               buffers, then O += P V (P from shared memory, V MN-major)
+//   warps 2..5  softmax, one thread per row (TMEM lane): online softmax with
+//               lazy rescaling of O (only when the max grows by > 2^8),
+//               P to shared memory, block-score capture, epilogue.
+// All waits are bounded (tc_ptx.cuh); a timeout aborts the CTA cleanly.
+#include "hs_common.cuh"
+#include "hs_kernels.cuh"
+#include "tc_ptx.cuh"
+
+namespace hs {
+namespace tc {
+
+constexpr int kBM = 128;
+constexpr int kBN = 64;
+constexpr int kD = 128;
+constexpr int kKV = 3;       // K/V ring stages
+constexpr int kList = 16;    // per-row candidate list (>= k/B)
+constexpr int kThreads = 192;
+
+constexpr uint32_t kQOff = 0;                       // 2 x 16 KB (d halves)
+constexpr uint32_t kKOff = 32768;                   // kKV x 16 KB
+constexpr uint32_t kVOff = kKOff + kKV * 16384;     // kKV x 16 KB
+constexpr uint32_t kPOff = kVOff + kKV * 16384;     // 2 x 16 KB
+constexpr uint32_t kBarOff = kPOff + 2 * 16384;
+enum {
+    BQ = 0,
+    BKVF = 1,
+    BKVE = BKVF + kKV,
+    BSF = BKVE + kKV,
+    BSE = BSF + 2,
+    BPF = BSE + 2,
+    BPVD = BPF + 2,
+    BOF = BPVD + 2,
+    BDRAIN = BOF + 1,
+    BCOUNT = BDRAIN + 1
+};
+constexpr uint32_t kMiscOff = kBarOff + BCOUNT * 8;
+constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;  // + room to align the base to 1 KB
+constexpr uint32_t kTmemCols = 256;                      // S0 | S1 | O
+constexpr uint32_t kColS = 0, kColO = 128;
+
+struct FullTcArgs {
+    KParams p;
+    __nv_bfloat16* o;
+    float* lse;
+    int32_t* idx;
+    int32_t* cnt;
+    float* sel;
+    int n_qtiles;
+    int P;        // positions per tile (128 / g)
+    int capture;  // 1: block-mode selection
+};
+
+// Bounded wait that ignores the abort flag (used to drain in-flight work).
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > kWaitCycles) { set_status(HS_ERR_TIMEOUT); return; }
+    }
+}
+
+// Warp-uniform bounded wait: every lane polls, the warp proceeds only if all saw it.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+    const bool ok = mbar_wait(bar, parity, abort);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Insert (v, id) into a list sorted by value descending; equal values keep the
+// earlier (lower) id first.  Static indices only, so the list stays in registers.
+__device__ __forceinline__ void list_insert(float (&lv)[kList], int (&li)[kList], float v, int id) {
+    if (!(v > lv[kList - 1])) return;
+#pragma unroll
+    for (int i = kList - 1; i >= 1; --i) {
+        if (lv[i - 1] < v) {
+            lv[i] = lv[i - 1];
+            li[i] = li[i - 1];
+        } else if (lv[i] < v) {
+            lv[i] = v;
+            li[i] = id;
+        }
+    }
+    if (lv[0] < v) { lv[0] = v; li[0] = id; }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    full_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                   const __grid_constant__ CUtensorMap tmap_k,
+                   const __grid_constant__ CUtensorMap tmap_v, FullTcArgs a) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    unsigned char* gbase = smem_raw + (base - raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const KParams& p = a.p;
+    const int g = p.group, P = a.P;
+
+    // tile -> (b, u, qt), heaviest query tiles first
+    const int bu_n = p.batch * p.hkv;
+    const int qt = a.n_qtiles - 1 - (int)(blockIdx.x / bu_n);
+    const int bu = (int)(blockIdx.x % bu_n);
+    const int b = bu / p.hkv, u = bu % p.hkv;
+    const int row0 = qt * P;                        // first query row of the tile
+    const int pos0 = p.q_offset + row0;             // its position
+    const int last_row = min(p.t_q, row0 + P) - 1;
+    const int pos_max = p.q_offset + last_row;
+    const int nt = min((p.t_kv + kBN - 1) / kBN, pos_max / kBN + 1);
+
+    auto bar = [&](int i) { return base + kBarOff + 8u * i; };
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + kMiscOff + 4);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kMiscOff);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(BQ), 1);
+        for (int i = 0; i < kKV; ++i) { mbar_init(bar(BKVF + i), 1); mbar_init(bar(BKVE + i), 1); }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(BSF + i), 1);
+            mbar_init(bar(BSE + i), 4);
+            mbar_init(bar(BPF + i), 4);
+            mbar_init(bar(BPVD + i), 1);
+        }
+        mbar_init(bar(BOF), 1);
+        mbar_init(bar(BDRAIN), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(base + kMiscOff, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tmap(&tmap_q);
+            prefetch_tmap(&tmap_k);
+            prefetch_tmap(&tmap_v);
+            mbar_arrive_expect_tx(bar(BQ), 2 * 16384);
+            tma_load_4d(base + kQOff, &tmap_q, bar(BQ), 0, row0, u * g, b);
+            tma_load_4d(base + kQOff + 16384, &tmap_q, bar(BQ), 64, row0, u * g, b);
+            int issued = 0;
+            for (int j = 0; j < nt; ++j) {
+                const int st = j % kKV;
+                if (j >= kKV && !mbar_wait(bar(BKVE + st), ((j / kKV) - 1) & 1, abort_flag)) break;
+                const uint32_t f = bar(BKVF + st);
+                mbar_arrive_expect_tx(f, 4 * 8192);
+                const uint32_t kd = base + kKOff + st * 16384, vd = base + kVOff + st * 16384;
+                const int key0 = j * kBN;
+                tma_load_3d(kd, &tmap_k, f, 0, key0, bu);
+                tma_load_3d(kd + 8192, &tmap_k, f, 64, key0, bu);
+                tma_load_3d(vd, &tmap_v, f, 0, key0, bu);
+                tma_load_3d(vd + 8192, &tmap_v, f, 64, key0, bu);
+                issued = j + 1;
+            }
+            // every issued load must have landed before the CTA may exit
+            mbar_drain(bar(BQ), 0);
+            for (int j = max(0, issued - kKV); j < issued; ++j)
+                mbar_drain(bar(BKVF + j % kKV), (j / kKV) & 1);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t id_s = idesc_bf16(kBM, kBN, false, false);
+            const uint32_t id_o = idesc_bf16(kBM, kD, false, true);
+            bool ok = mbar_wait(bar(BQ), 0, abort_flag);
+            tc_fence_after();
+            for (int j = 0; ok && j <= nt; ++j) {
+                if (j < nt) {
+                    const int st = j % kKV, s = j & 1;
+                    if (!mbar_wait(bar(BKVF + st), (j / kKV) & 1, abort_flag)) break;
+                    if (j >= 2 && !mbar_wait(bar(BSE + s), ((j >> 1) - 1) & 1, abort_flag)) break;
+                    tc_fence_after();
+                    const uint32_t kb = base + kKOff + st * 16384;
+#pragma unroll
+                    for (int kk = 0; kk < kD / 16; ++kk) {
+                        const uint64_t ad = sw128_desc(base + kQOff + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                        const uint64_t bd = sw128_desc(kb + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+                        umma_ss(tmem + kColS + 64 * s, ad, bd, id_s, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(bar(BSF + s));
+                }
+                if (j >= 1) {
+                    const int jj = j - 1, sp = jj & 1, stp = jj % kKV;
+                    if (!mbar_wait(bar(BPF + sp), (jj >> 1) & 1, abort_flag)) break;
+                    tc_fence_after();
+                    const uint32_t vb = base + kVOff + stp * 16384;
+                    const uint32_t pb = base + kPOff + sp * 16384;
+#pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk) {
+                        const uint64_t ad = sw128_desc(pb + kk * 32, 16, 1024);
+                        const uint64_t bd = sw128_desc(vb + kk * 2048, 8192, 1024);
+                        umma_ss(tmem + kColO, ad, bd, id_o, (jj > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(bar(BPVD + sp));
+                    umma_commit(bar(BKVE + stp));
+                }
+            }
+            umma_commit(bar(BOF));
+            umma_commit(bar(BDRAIN));
+            mbar_drain(bar(BDRAIN), 0);
+        }
+    } else {
+        // ------------------------------------------------------ softmax
+        const int quad = warp & 3;
+        const int row = quad * 32 + lane;
+        const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+        const int hh = row / P, pr = row % P;
+        const int pos = pos0 + pr;
+        const float sl2 = p.scale_log2;
+        float m_ref = -INFINITY, l = 0.f;
+        float lv[kList];
+        int li[kList];
+#pragma unroll
+        for (int i = 0; i < kList; ++i) { lv[i] = -INFINITY; li[i] = -1; }
+        bool ok = true;
+        for (int j = 0; j < nt; ++j) {
+            const int s = j & 1;
+            if (!warp_wait(bar(BSF + s), (j >> 1) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t r0[32], r1[32];
+            tmem_ld32(trow + kColS + 64 * s, r0);
+            tmem_ld32(trow + kColS + 64 * s + 32, r1);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(BSE + s));
+
+            const int key0 = j * kBN;
+            const int lim = pos - key0;  // keys c <= lim are visible
+            float x[64];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                x[c] = c <= lim ? __uint_as_float(r0[c]) * sl2 : -INFINITY;
+                x[32 + c] = 32 + c <= lim ? __uint_as_float(r1[c]) * sl2 : -INFINITY;
+            }
+            float mt = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) mt = fmaxf(mt, x[c]);
+            if (a.capture && mt > -INFINITY) list_insert(lv, li, mt, j);
+            // lazy rescale: keep the reference max unless the tile exceeds it by 2^8
+            bool resc = false;
+            float corr = 1.f;
+            if (mt > m_ref + 8.f) {
+                corr = exp2f(m_ref - mt);  // 0 on the first tile
+                resc = j > 0;
+                m_ref = mt;
+                l *= corr;
+            }
+            float sum = 0.f;
+            uint32_t pk[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                const float e0 = exp2f(x[2 * c] - m_ref);
+                const float e1 = exp2f(x[2 * c + 1] - m_ref);
+                sum += e0 + e1;
+                pk[c] = pack_bf16(e0, e1);
+            }
+            l += sum;
+            // P buffer s is free once the PV of tile j-2 is done
+            if (j >= 2 && !warp_wait(bar(BPVD + s), ((j >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+            unsigned char* prow = gbase + kPOff + s * 16384 + row * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint4 v4 = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) = v4;
+            }
+            fence_proxy_async_smem();
+            if (__any_sync(0xffffffffu, resc)) {
+                // O may only be touched once the PV of tile j-1 has finished
+                if (!warp_wait(bar(BPVD + (s ^ 1)), ((j - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const float cf = resc ? corr : 1.f;
+#pragma unroll
+                for (int c4 = 0; c4 < kD / 32; ++c4) {
+                    uint32_t ro[32];
+                    tmem_ld32(trow + kColO + 32 * c4, ro);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) ro[c] = __float_as_uint(__uint_as_float(ro[c]) * cf);
+                    tmem_st32(trow + kColO + 32 * c4, ro);
+                }
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(BPF + s));
+        }
+        if (ok) ok = warp_wait(bar(BOF), 0, abort_flag);
+        const bool row_ok = row0 + pr < p.t_q;
+        const int h = u * g + hh;
+        const size_t orow = ((size_t)b * p.hq + h) * p.t_q + row0 + pr;
+        const float lse2 = m_ref + log2f(l);
+        if (ok) {
+            tc_fence_after();
+            const float inv = 1.f / l;
+            __nv_bfloat16* og = a.o + orow * kD;
+#pragma unroll
+            for (int c4 = 0; c4 < kD / 32; ++c4) {
+                uint32_t ro[32];
+                tmem_ld32(trow + kColO + 32 * c4, ro);
+                tmem_wait_ld();
+                if (row_ok) {
+#pragma unroll
+                    for (int c = 0; c < 32; c += 8) {
+                        uint4 v4;
+                        v4.x = pack_bf16(__uint_as_float(ro[c]) * inv, __uint_as_float(ro[c + 1]) * inv);
+                        v4.y = pack_bf16(__uint_as_float(ro[c + 2]) * inv, __uint_as_float(ro[c + 3]) * inv);
+                        v4.z = pack_bf16(__uint_as_float(ro[c + 4]) * inv, __uint_as_float(ro[c + 5]) * inv);
+                        v4.w = pack_bf16(__uint_as_float(ro[c + 6]) * inv, __uint_as_float(ro[c + 7]) * inv);
+                        *reinterpret_cast<uint4*>(og + c4 * 32 + c) = v4;
+                    }
+                }
+            }
+            if (row_ok) a.lse[orow] = lse2 * kLn2;
+        }
+        if (a.capture) {
+            // ---- group merge: rows hh*P + pr of the g heads share position pr
+            float* cs = reinterpret_cast<float*>(gbase + kPOff);            // [128][kList]
+            int* ci = reinterpret_cast<int*>(gbase + kPOff + 128 * kList * 4);
+            unsigned char* flags = gbase + kPOff + 2 * 128 * kList * 4;     // [g*kList]
+            // every PV has completed (BOF), so the P buffers are free to reuse
+#pragma unroll
+            for (int i = 0; i < kList; ++i) {
+                cs[row * kList + i] = li[i] >= 0 ? lv[i] - lse2 : -INFINITY;
+                ci[row * kList + i] = ok ? li[i] : -1;
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            const int wq = warp - 2;
+            const int n = g * kList;
+            unsigned char* fl = flags + wq * 256;
+            for (int pp = wq; pp < P && ok; pp += 4) {
+                const int rj = row0 + pp;
+                if (rj >= p.t_q) break;
+                // candidate i -> entry (head i / kList, slot i % kList) of position pp
+                auto eidx = [&](int i) { return ((i / kList) * P + pp) * kList + (i % kList); };
+                // 1) primary: best occurrence of its id (ties: first occurrence)
+                for (int i = lane; i < n; i += 32) {
+                    const int e = eidx(i);
+                    const int id = ci[e];
+                    bool prim = id >= 0;
+                    for (int i2 = 0; i2 < n && prim; ++i2) {
+                        const int e2 = eidx(i2);
+                        if (ci[e2] == id && (cs[e2] > cs[e] || (cs[e2] == cs[e] && i2 < i))) prim = false;
+                    }
+                    fl[i] = prim ? 1 : 0;
+                }
+                __syncwarp();
+                // 2) rank among primaries: (score desc, id asc)
+                for (int i = lane; i < n; i += 32) {
+                    if (!fl[i]) continue;
+                    const int e = eidx(i);
+                    int rank = 0;
+                    for (int i2 = 0; i2 < n; ++i2) {
+                        if (!fl[i2]) continue;
+                        const int e2 = eidx(i2);
+                        if (cs[e2] > cs[e] || (cs[e2] == cs[e] && ci[e2] < ci[e])) ++rank;
+                    }
+                    if (rank < p.ksel) fl[i] = 2;
+                }
+                __syncwarp();
+                // 3) output in ascending id order
+                const size_t orow_i = ((size_t)b * p.hkv + u) * p.t_q + rj;
+                int32_t* irow = a.idx + orow_i * p.ksel;
+                float* srow = a.sel ? a.sel + orow_i * p.ksel : nullptr;
+                int nsel = 0;
+                for (int i0 = 0; i0 < n; i0 += 32) {
+                    const int i = i0 + lane;
+                    nsel += __popc(__ballot_sync(0xffffffffu, i < n && fl[i] == 2));
+                }
+                for (int i = lane; i < n; i += 32) {
+                    if (fl[i] != 2) continue;
+                    const int e = eidx(i);
+                    int op = 0;
+                    for (int i2 = 0; i2 < n; ++i2)
+                        if (fl[i2] == 2 && ci[eidx(i2)] < ci[e]) ++op;
+                    if (op < p.ksel) {
+                        irow[op] = ci[e];
+                        if (srow) srow[op] = exp2f(cs[e]);
+                    }
+                }
+                for (int x = min(nsel, p.ksel) + lane; x < p.ksel; x += 32) {
+                    irow[x] = -1;
+                    if (srow) srow[x] = 0.f;
+                }
+                nsel = min(nsel, p.ksel);
+                if (lane == 0) a.cnt[orow_i] = nsel;
+                __syncwarp();
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------- host
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encoder() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+static bool encode(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims,
+                   const cuuint64_t* strides, const cuuint32_t* box) {
+    EncodeTiledFn fn = get_encoder();
+    if (!fn) return false;
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims, strides,
+              box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+}  // namespace tc
+
+bool full_tc_supported(const KParams& p, int dtype) {
+    if (dtype != HS_BF16 || p.head_dim != 128) return false;
+    if (128 % p.group != 0) return false;
+    if (p.mode == 0) return p.block_size == tc::kBN && p.ksel <= tc::kList;
+    return true;
+}
+
+// capture = 1: block-mode index into idx/cnt/sel.  capture = 0: o and lse only.
+cudaError_t launch_full_tc(const KParams& p, const void* q, const void* k, const void* v,
+                           void* o, float* lse, int32_t* idx, int32_t* cnt, float* sel,
+                           int capture, cudaStream_t st) {
+    using namespace tc;
+    const int g = p.group, P = kBM / g;
+    CUtensorMap mq, mk, mv;
+    const cuuint64_t qd[4] = {(cuuint64_t)kD, (cuuint64_t)p.t_q, (cuuint64_t)p.hq,
+                              (cuuint64_t)p.batch};
+    const cuuint64_t qs[3] = {(cuuint64_t)kD * 2, (cuuint64_t)p.t_q * kD * 2,
+                              (cuuint64_t)p.hq * p.t_q * kD * 2};
+    const cuuint32_t qb[4] = {64, (cuuint32_t)P, (cuuint32_t)g, 1};
+    const cuuint64_t kdims[3] = {(cuuint64_t)kD, (cuuint64_t)p.t_kv,
+                                 (cuuint64_t)p.hkv * p.batch};
+    const cuuint64_t ks[2] = {(cuuint64_t)kD * 2, (cuuint64_t)p.t_kv * kD * 2};
+    const cuuint32_t kb[3] = {64, (cuuint32_t)kBN, 1};
+    if (!encode(&mq, q, 4, qd, qs, qb) || !encode(&mk, k, 3, kdims, ks, kb) ||
+        !encode(&mv, v, 3, kdims, ks, kb))
+        return cudaErrorInvalidValue;
+    FullTcArgs a;
+    a.p = p;
+    a.o = (__nv_bfloat16*)o;
+    a.lse = lse;
+    a.idx = idx;
+    a.cnt = cnt;
+    a.sel = sel;
+    a.P = P;
+    a.n_qtiles = (p.t_q + P - 1) / P;
+    a.capture = capture;
+    cudaError_t e = cudaFuncSetAttribute(full_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const long long grid = (long long)a.n_qtiles * p.batch * p.hkv;
+    full_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, a);
+    return cudaGetLastError();
+}
+
+}  // namespace hs

@@ -15,6 +15,7 @@
 
 #include "decode_full.cu"
 #include "full_simt.cu"
+#include "full_tc.cu"
 #include "sparse.cu"
 
 namespace hs {
@@ -113,9 +114,23 @@ hs_status hs_full_attn_index(const hs_params* p, const void* q, const void* k, c
         return HS_ERR_INVALID_ARG;
     if (kp.t_q == 0) return HS_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (hs::full_tc_supported(kp, p->dtype)) {
+        if (kp.mode == HS_SEL_BLOCK)
+            return launched(1, [&] {
+                return hs::launch_full_tc(kp, q, k, v, o, lse, idx, idx_count, sel_scores, 1, st);
+            });
+        // token mode: tensor-core attention pass, then the selection pass
+        return launched(2, [&] {
+            cudaError_t e =
+                hs::launch_full_tc(kp, q, k, v, o, lse, idx, idx_count, sel_scores, 0, st);
+            if (e != cudaSuccess) return e;
+            return hs::launch_full_simt(kp, p->dtype, q, k, v, o, lse, idx, idx_count,
+                                        sel_scores, 0, st);
+        });
+    }
     return launched(1, [&] {
         return hs::launch_full_simt(kp, p->dtype, q, k, v, o, lse, idx, idx_count, sel_scores,
-                                    st);
+                                    1, st);
     });
 }
 

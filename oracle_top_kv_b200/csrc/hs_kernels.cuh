@@ -21,9 +21,16 @@ struct KParams {
     float scale_log2;  // softmax scale * log2(e)
 };
 
+// do_attn = 0: selection only, reading lse from a previous attention pass.
 cudaError_t launch_full_simt(const KParams& p, int dtype, const void* q, const void* k,
                              const void* v, void* o, float* lse, int32_t* idx, int32_t* cnt,
-                             float* sel, cudaStream_t st);
+                             float* sel, int do_attn, cudaStream_t st);
+
+// tcgen05 flash attention (bf16, d = 128).  capture = 1: block-mode index.
+bool full_tc_supported(const KParams& p, int dtype);
+cudaError_t launch_full_tc(const KParams& p, const void* q, const void* k, const void* v,
+                           void* o, float* lse, int32_t* idx, int32_t* cnt, float* sel,
+                           int capture, cudaStream_t st);
 
 cudaError_t launch_sparse_simt(const KParams& p, int dtype, const void* q, const void* kf,
                                const void* vf, const int32_t* idx, const int32_t* cnt,

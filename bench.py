@@ -186,10 +186,22 @@ def traffic_for(kernel, workload):
     return d["bytes_per_launch"] if h.hexdigest() == d.get("sha256") else None
 
 
+def workload_of(args):
+    w = wl.WORKLOADS[args.workload]
+    kw = {}
+    if args.batch:
+        kw["batch"] = args.batch
+    if args.seq:
+        kw["t"] = args.seq
+    if kw:
+        w = wl.scaled(w, name=w.name + "".join(f"_{k}{v}" for k, v in kw.items()), **kw)
+    return w
+
+
 def run_ours(args, rank, world, device):
     from oracle_top_kv_b200 import hs
     hs.load()
-    w = wl.WORKLOADS[args.workload]
+    w = workload_of(args)
     peaks, peak_kind = load_peaks()
     blk = HybridBlock(w, device)
     stream = torch.cuda.current_stream(device)
@@ -415,6 +427,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="hysparse_7b_block", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--batch", type=int, default=0, help="override the batch (reduced replica)")
+    ap.add_argument("--seq", type=int, default=0, help="override the sequence length")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -422,7 +436,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    w = wl.WORKLOADS[args.workload]
+    w = workload_of(args)
 
     if args.impl == "reference":
         if rank == 0:

@@ -14,15 +14,19 @@
 // union of the lists, re-scored as m~ - lse_h, contains the answer
 // ("GQA 下为什么要组内共享索引": S_bar = max over the group's heads).
 //
-// Tile: 128 query rows = g heads x (128/g) positions of one KV group (rows are
-// head-major, exactly as one 4-D TMA box lands), so every K/V tile is loaded
-// once for the whole group.  Warp roles:
-//   warp 0      TMA producer (Q once; K and V tiles through a 3-stage ring)
-//   warp 1      TMEM owner and MMA issuer: S = Q K^T into one of two TMEM
-//               buffers, then O += P V (P from shared memory, V MN-major)
-//   warps 2..5  softmax, one thread per row (TMEM lane): online softmax with
-//               lazy rescaling of O (only when the max grows by > 2^8),
-//               P to shared memory, block-score capture, epilogue.
+// Q tile: 128 query rows = g heads x (128/g) positions of one KV group (rows
+// are head-major, exactly as one 4-D TMA box lands), so every K/V tile is
+// loaded once for the whole group.  A CTA runs two consecutive Q tiles that
+// share every K/V tile; their softmax warpgroups alternate on the tensor core.
+// Warp roles:
+//   warp 0       TMA producer (both Q tiles once; K and V tiles, 3-stage ring)
+//   warp 1       TMEM owner and MMA issuer: per Q tile S = Q K^T into one of
+//                two TMEM buffers, then O += P V (P from shared memory, V
+//                MN-major)
+//   warps 2..9   two softmax warpgroups, one thread per row (TMEM lane):
+//                online softmax with lazy rescaling of O (only when the max
+//                grows by > 2^8), P to shared memory, block-score capture,
+//                epilogue.
 // All waits are bounded (tc_ptx.cuh); a timeout aborts the CTA cleanly.
 #include "hs_common.cuh"
 #include "hs_kernels.cuh"
@@ -31,34 +35,34 @@
 namespace hs {
 namespace tc {
 
-constexpr int kBM = 128;
-constexpr int kBN = 64;
+constexpr int kBM = 128;      // rows per Q tile (one softmax warpgroup)
+constexpr int kNQ = 2;        // Q tiles per CTA, sharing every K/V tile
+constexpr int kBN = 64;       // keys per K/V tile (= block size B)
 constexpr int kD = 128;
-constexpr int kKV = 3;       // K/V ring stages
-constexpr int kList = 16;    // per-row candidate list (>= k/B)
-constexpr int kThreads = 192;
+constexpr int kKV = 3;        // K/V ring stages
+constexpr int kList = 16;     // per-row candidate list (>= k/B)
+constexpr int kThreads = 64 + 128 * kNQ;
 
-constexpr uint32_t kQOff = 0;                       // 2 x 16 KB (d halves)
-constexpr uint32_t kKOff = 32768;                   // kKV x 16 KB
-constexpr uint32_t kVOff = kKOff + kKV * 16384;     // kKV x 16 KB
-constexpr uint32_t kPOff = kVOff + kKV * 16384;     // 2 x 16 KB
-constexpr uint32_t kBarOff = kPOff + 2 * 16384;
+constexpr uint32_t kQOff = 0;                         // kNQ x 32 KB (two d halves each)
+constexpr uint32_t kKOff = kNQ * 32768;               // kKV x 16 KB
+constexpr uint32_t kVOff = kKOff + kKV * 16384;       // kKV x 16 KB
+constexpr uint32_t kPOff = kVOff + kKV * 16384;       // kNQ x 2 x 16 KB
+constexpr uint32_t kBarOff = kPOff + kNQ * 2 * 16384;
 enum {
     BQ = 0,
     BKVF = 1,
     BKVE = BKVF + kKV,
-    BSF = BKVE + kKV,
-    BSE = BSF + 2,
-    BPF = BSE + 2,
-    BPVD = BPF + 2,
-    BOF = BPVD + 2,
+    BSF = BKVE + kKV,      // [q][s]
+    BSE = BSF + 2 * kNQ,
+    BPF = BSE + 2 * kNQ,
+    BPVD = BPF + 2 * kNQ,
+    BOF = BPVD + 2 * kNQ,
     BDRAIN = BOF + 1,
     BCOUNT = BDRAIN + 1
 };
 constexpr uint32_t kMiscOff = kBarOff + BCOUNT * 8;
 constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;  // + room to align the base to 1 KB
-constexpr uint32_t kTmemCols = 256;                      // S0 | S1 | O
-constexpr uint32_t kColS = 0, kColO = 128;
+constexpr uint32_t kTmemCols = 256 * kNQ;              // per Q tile: S0 | S1 | O
 
 struct FullTcArgs {
     KParams p;
@@ -67,15 +71,15 @@ struct FullTcArgs {
     int32_t* idx;
     int32_t* cnt;
     float* sel;
-    int n_qtiles;
-    int P;        // positions per tile (128 / g)
-    int capture;  // 1: block-mode selection
+    int n_ctas_q;  // CTAs along the query axis
+    int P;         // positions per Q tile (128 / g)
+    int capture;   // 1: block-mode selection
 };
 
 // Bounded wait that ignores the abort flag (used to drain in-flight work).
 __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_sleep(bar, parity)) {
         if (clock64() - t0 > kWaitCycles) { set_status(HS_ERR_TIMEOUT); return; }
     }
 }
@@ -103,6 +107,13 @@ __device__ __forceinline__ void list_insert(float (&lv)[kList], int (&li)[kList]
     if (lv[0] < v) { lv[0] = v; li[0] = id; }
 }
 
+// Number of K/V tiles a Q tile needs: keys up to its last valid row's position.
+__device__ __forceinline__ int tiles_for(const KParams& p, int first_row, int P) {
+    if (first_row >= p.t_q) return 0;
+    const int last_row = min(p.t_q, first_row + P) - 1;
+    return min((p.t_kv + kBN - 1) / kBN, (p.q_offset + last_row) / kBN + 1);
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     full_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                    const __grid_constant__ CUtensorMap tmap_k,
@@ -115,16 +126,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const KParams& p = a.p;
     const int g = p.group, P = a.P;
 
-    // tile -> (b, u, qt), heaviest query tiles first
+    // CTA -> (b, u, query tile pair), heaviest (latest) query tiles first
     const int bu_n = p.batch * p.hkv;
-    const int qt = a.n_qtiles - 1 - (int)(blockIdx.x / bu_n);
+    const int qc = a.n_ctas_q - 1 - (int)(blockIdx.x / bu_n);
     const int bu = (int)(blockIdx.x % bu_n);
     const int b = bu / p.hkv, u = bu % p.hkv;
-    const int row0 = qt * P;                        // first query row of the tile
-    const int pos0 = p.q_offset + row0;             // its position
-    const int last_row = min(p.t_q, row0 + P) - 1;
-    const int pos_max = p.q_offset + last_row;
-    const int nt = min((p.t_kv + kBN - 1) / kBN, pos_max / kBN + 1);
+    const int row0 = qc * kNQ * P;  // first query row of the CTA
+    int ntq[kNQ];
+#pragma unroll
+    for (int q = 0; q < kNQ; ++q) ntq[q] = tiles_for(p, row0 + q * P, P);
+    int nt = 0;
+#pragma unroll
+    for (int q = 0; q < kNQ; ++q) nt = max(nt, ntq[q]);
 
     auto bar = [&](int i) { return base + kBarOff + 8u * i; };
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + kMiscOff + 4);
@@ -133,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         mbar_init(bar(BQ), 1);
         for (int i = 0; i < kKV; ++i) { mbar_init(bar(BKVF + i), 1); mbar_init(bar(BKVE + i), 1); }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < 2 * kNQ; ++i) {
             mbar_init(bar(BSF + i), 1);
             mbar_init(bar(BSE + i), 4);
             mbar_init(bar(BPF + i), 4);
@@ -159,9 +172,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tmap(&tmap_q);
             prefetch_tmap(&tmap_k);
             prefetch_tmap(&tmap_v);
-            mbar_arrive_expect_tx(bar(BQ), 2 * 16384);
-            tma_load_4d(base + kQOff, &tmap_q, bar(BQ), 0, row0, u * g, b);
-            tma_load_4d(base + kQOff + 16384, &tmap_q, bar(BQ), 64, row0, u * g, b);
+            mbar_arrive_expect_tx(bar(BQ), kNQ * 32768);
+#pragma unroll
+            for (int q = 0; q < kNQ; ++q) {
+                tma_load_4d(base + kQOff + q * 32768, &tmap_q, bar(BQ), 0, row0 + q * P, u * g, b);
+                tma_load_4d(base + kQOff + q * 32768 + 16384, &tmap_q, bar(BQ), 64, row0 + q * P,
+                            u * g, b);
+            }
             int issued = 0;
             for (int j = 0; j < nt; ++j) {
                 const int st = j % kKV;
@@ -192,30 +209,47 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (j < nt) {
                     const int st = j % kKV, s = j & 1;
                     if (!mbar_wait(bar(BKVF + st), (j / kKV) & 1, abort_flag)) break;
-                    if (j >= 2 && !mbar_wait(bar(BSE + s), ((j >> 1) - 1) & 1, abort_flag)) break;
-                    tc_fence_after();
                     const uint32_t kb = base + kKOff + st * 16384;
 #pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk) {
-                        const uint64_t ad = sw128_desc(base + kQOff + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                        const uint64_t bd = sw128_desc(kb + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-                        umma_ss(tmem + kColS + 64 * s, ad, bd, id_s, kk > 0 ? 1u : 0u);
+                    for (int q = 0; q < kNQ; ++q) {
+                        if (j >= ntq[q]) continue;
+                        if (j >= 2 && !mbar_wait(bar(BSE + 2 * q + s), ((j >> 1) - 1) & 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t qb = base + kQOff + q * 32768;
+#pragma unroll
+                        for (int kk = 0; kk < kD / 16; ++kk) {
+                            const uint64_t ad = sw128_desc(qb + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                            const uint64_t bd = sw128_desc(kb + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+                            umma_ss(tmem + q * 256 + 64 * s, ad, bd, id_s, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(bar(BSF + 2 * q + s));
                     }
-                    umma_commit(bar(BSF + s));
+                    if (!ok) break;
                 }
                 if (j >= 1) {
                     const int jj = j - 1, sp = jj & 1, stp = jj % kKV;
-                    if (!mbar_wait(bar(BPF + sp), (jj >> 1) & 1, abort_flag)) break;
-                    tc_fence_after();
                     const uint32_t vb = base + kVOff + stp * 16384;
-                    const uint32_t pb = base + kPOff + sp * 16384;
 #pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk) {
-                        const uint64_t ad = sw128_desc(pb + kk * 32, 16, 1024);
-                        const uint64_t bd = sw128_desc(vb + kk * 2048, 8192, 1024);
-                        umma_ss(tmem + kColO, ad, bd, id_o, (jj > 0 || kk > 0) ? 1u : 0u);
+                    for (int q = 0; q < kNQ; ++q) {
+                        if (jj >= ntq[q]) continue;
+                        if (!mbar_wait(bar(BPF + 2 * q + sp), (jj >> 1) & 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t pb = base + kPOff + (2 * q + sp) * 16384;
+#pragma unroll
+                        for (int kk = 0; kk < kBN / 16; ++kk) {
+                            const uint64_t ad = sw128_desc(pb + kk * 32, 16, 1024);
+                            const uint64_t bd = sw128_desc(vb + kk * 2048, 8192, 1024);
+                            umma_ss(tmem + q * 256 + 128, ad, bd, id_o, (jj > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit(bar(BPVD + 2 * q + sp));
                     }
-                    umma_commit(bar(BPVD + sp));
+                    if (!ok) break;
                     umma_commit(bar(BKVE + stp));
                 }
             }
@@ -225,11 +259,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------ softmax
-        const int quad = warp & 3;
+        const int q = (warp - 2) >> 2;   // warpgroup = Q tile
+        const int quad = warp & 3;       // TMEM lane quadrant of this warp
         const int row = quad * 32 + lane;
-        const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+        const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16) + q * 256;
         const int hh = row / P, pr = row % P;
-        const int pos = pos0 + pr;
+        const int qrow0 = row0 + q * P;              // first query row of this Q tile
+        const int pos_first = p.q_offset + qrow0;    // its position
+        const int pos = pos_first + pr;
+        const int nt_me = ntq[q];
         const float sl2 = p.scale_log2;
         float m_ref = -INFINITY, l = 0.f;
         float lv[kList];
@@ -237,52 +275,65 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < kList; ++i) { lv[i] = -INFINITY; li[i] = -1; }
         bool ok = true;
-        for (int j = 0; j < nt; ++j) {
+        for (int j = 0; j < nt_me; ++j) {
             const int s = j & 1;
-            if (!warp_wait(bar(BSF + s), (j >> 1) & 1, abort_flag)) { ok = false; break; }
+            if (!warp_wait(bar(BSF + 2 * q + s), (j >> 1) & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
-            uint32_t r0[32], r1[32];
-            tmem_ld32(trow + kColS + 64 * s, r0);
-            tmem_ld32(trow + kColS + 64 * s + 32, r1);
+            uint32_t r[64];
+            tmem_ld32(trow + 64 * s, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+            tmem_ld32(trow + 64 * s + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(BSE + s));
+            if (lane == 0) mbar_arrive(bar(BSE + 2 * q + s));
 
             const int key0 = j * kBN;
-            const int lim = pos - key0;  // keys c <= lim are visible
             float x[64];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                x[c] = c <= lim ? __uint_as_float(r0[c]) * sl2 : -INFINITY;
-                x[32 + c] = 32 + c <= lim ? __uint_as_float(r1[c]) * sl2 : -INFINITY;
-            }
-            float mt = -INFINITY;
+            for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(r[c]);
+            if (key0 + kBN - 1 > pos_first) {  // diagonal tile: causal mask per row
+                const int lim = pos - key0;
 #pragma unroll
-            for (int c = 0; c < 64; ++c) mt = fmaxf(mt, x[c]);
+                for (int c = 0; c < 64; ++c) x[c] = c <= lim ? x[c] : -INFINITY;
+            }
+            // tile max of the raw logits (tree), then to the log2 domain
+            float mx[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+                mx[c] = fmaxf(fmaxf(x[c], x[c + 16]), fmaxf(x[c + 32], x[c + 48]));
+#pragma unroll
+            for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+                for (int c = 0; c < w; ++c) mx[c] = fmaxf(mx[c], mx[c + w]);
+            const float mt = mx[0] * sl2;  // -inf stays -inf (sl2 > 0)
             if (a.capture && mt > -INFINITY) list_insert(lv, li, mt, j);
             // lazy rescale: keep the reference max unless the tile exceeds it by 2^8
             bool resc = false;
             float corr = 1.f;
             if (mt > m_ref + 8.f) {
-                corr = exp2f(m_ref - mt);  // 0 on the first tile
+                corr = ex2(m_ref - mt);  // 0 on the first tile
                 resc = j > 0;
                 m_ref = mt;
                 l *= corr;
             }
-            float sum = 0.f;
+            const float nm = -m_ref;
+            float e[64];
+#pragma unroll
+            for (int c = 0; c < 64; ++c) e[c] = ex2(fmaf(x[c], sl2, nm));
+            float sm[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) sm[c] = (e[c] + e[c + 16]) + (e[c + 32] + e[c + 48]);
+#pragma unroll
+            for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+                for (int c = 0; c < w; ++c) sm[c] += sm[c + w];
+            l += sm[0];
             uint32_t pk[32];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const float e0 = exp2f(x[2 * c] - m_ref);
-                const float e1 = exp2f(x[2 * c + 1] - m_ref);
-                sum += e0 + e1;
-                pk[c] = pack_bf16(e0, e1);
-            }
-            l += sum;
-            // P buffer s is free once the PV of tile j-2 is done
-            if (j >= 2 && !warp_wait(bar(BPVD + s), ((j >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
-            unsigned char* prow = gbase + kPOff + s * 16384 + row * 128;
+            for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(e[2 * c], e[2 * c + 1]);
+            // P buffer s of this tile is free once the PV of tile j-2 is done
+            if (j >= 2 && !warp_wait(bar(BPVD + 2 * q + s), ((j >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+            unsigned char* prow = gbase + kPOff + (2 * q + s) * 16384 + row * 128;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 uint4 v4 = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
@@ -291,37 +342,37 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
             if (__any_sync(0xffffffffu, resc)) {
                 // O may only be touched once the PV of tile j-1 has finished
-                if (!warp_wait(bar(BPVD + (s ^ 1)), ((j - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+                if (!warp_wait(bar(BPVD + 2 * q + (s ^ 1)), ((j - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const float cf = resc ? corr : 1.f;
 #pragma unroll
                 for (int c4 = 0; c4 < kD / 32; ++c4) {
                     uint32_t ro[32];
-                    tmem_ld32(trow + kColO + 32 * c4, ro);
+                    tmem_ld32(trow + 128 + 32 * c4, ro);
                     tmem_wait_ld();
 #pragma unroll
                     for (int c = 0; c < 32; ++c) ro[c] = __float_as_uint(__uint_as_float(ro[c]) * cf);
-                    tmem_st32(trow + kColO + 32 * c4, ro);
+                    tmem_st32(trow + 128 + 32 * c4, ro);
                 }
                 tmem_wait_st();
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(BPF + s));
+            if (lane == 0) mbar_arrive(bar(BPF + 2 * q + s));
         }
-        if (ok) ok = warp_wait(bar(BOF), 0, abort_flag);
-        const bool row_ok = row0 + pr < p.t_q;
+        if (ok && nt_me > 0) ok = warp_wait(bar(BOF), 0, abort_flag);
+        const bool row_ok = nt_me > 0 && qrow0 + pr < p.t_q;
         const int h = u * g + hh;
-        const size_t orow = ((size_t)b * p.hq + h) * p.t_q + row0 + pr;
+        const size_t orow = ((size_t)b * p.hq + h) * p.t_q + qrow0 + pr;
         const float lse2 = m_ref + log2f(l);
-        if (ok) {
+        if (ok && nt_me > 0) {
             tc_fence_after();
             const float inv = 1.f / l;
             __nv_bfloat16* og = a.o + orow * kD;
 #pragma unroll
             for (int c4 = 0; c4 < kD / 32; ++c4) {
                 uint32_t ro[32];
-                tmem_ld32(trow + kColO + 32 * c4, ro);
+                tmem_ld32(trow + 128 + 32 * c4, ro);
                 tmem_wait_ld();
                 if (row_ok) {
 #pragma unroll
@@ -339,21 +390,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (a.capture) {
             // ---- group merge: rows hh*P + pr of the g heads share position pr
-            float* cs = reinterpret_cast<float*>(gbase + kPOff);            // [128][kList]
-            int* ci = reinterpret_cast<int*>(gbase + kPOff + 128 * kList * 4);
-            unsigned char* flags = gbase + kPOff + 2 * 128 * kList * 4;     // [g*kList]
+            unsigned char* reg = gbase + kPOff + q * 32768;    // this tile's P buffers
+            float* cs = reinterpret_cast<float*>(reg);         // [128][kList]
+            int* ci = reinterpret_cast<int*>(reg + 128 * kList * 4);
+            unsigned char* flags = reg + 2 * 128 * kList * 4;  // 4 warps x 256
             // every PV has completed (BOF), so the P buffers are free to reuse
 #pragma unroll
             for (int i = 0; i < kList; ++i) {
                 cs[row * kList + i] = li[i] >= 0 ? lv[i] - lse2 : -INFINITY;
                 ci[row * kList + i] = ok ? li[i] : -1;
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            const int wq = warp - 2;
+            asm volatile("bar.sync %0, 128;" ::"r"(1 + q) : "memory");
             const int n = g * kList;
-            unsigned char* fl = flags + wq * 256;
-            for (int pp = wq; pp < P && ok; pp += 4) {
-                const int rj = row0 + pp;
+            unsigned char* fl = flags + quad * 256;
+            for (int pp = quad; pp < P && ok; pp += 4) {
+                const int rj = qrow0 + pp;
                 if (rj >= p.t_q) break;
                 // candidate i -> entry (head i / kList, slot i % kList) of position pp
                 auto eidx = [&](int i) { return ((i / kList) * P + pp) * kList + (i % kList); };
@@ -391,6 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int i = i0 + lane;
                     nsel += __popc(__ballot_sync(0xffffffffu, i < n && fl[i] == 2));
                 }
+                nsel = min(nsel, p.ksel);
                 for (int i = lane; i < n; i += 32) {
                     if (fl[i] != 2) continue;
                     const int e = eidx(i);
@@ -402,11 +454,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (srow) srow[op] = exp2f(cs[e]);
                     }
                 }
-                for (int x = min(nsel, p.ksel) + lane; x < p.ksel; x += 32) {
+                for (int x = nsel + lane; x < p.ksel; x += 32) {
                     irow[x] = -1;
                     if (srow) srow[x] = 0.f;
                 }
-                nsel = min(nsel, p.ksel);
                 if (lane == 0) a.cnt[orow_i] = nsel;
                 __syncwarp();
             }
@@ -488,12 +539,12 @@ cudaError_t launch_full_tc(const KParams& p, const void* q, const void* k, const
     a.cnt = cnt;
     a.sel = sel;
     a.P = P;
-    a.n_qtiles = (p.t_q + P - 1) / P;
+    a.n_ctas_q = (p.t_q + kNQ * P - 1) / (kNQ * P);
     a.capture = capture;
     cudaError_t e = cudaFuncSetAttribute(full_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
-    const long long grid = (long long)a.n_qtiles * p.batch * p.hkv;
+    const long long grid = (long long)a.n_ctas_q * p.batch * p.hkv;
     full_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, a);
     return cudaGetLastError();
 }

@@ -79,11 +79,30 @@ __device__ __forceinline__ void load_chunk(uint32_t stage_base, const __nv_bfloa
     }
 }
 
-// S = Q K^T for one chunk (16 x 32), scaled to log2 domain and masked.
+// Issue the cp.async loads of a chunk of 32 consecutive keys key0..key0+31;
+// rows whose bit is clear in `valid` are zero-filled without being read.
+template <int D>
+__device__ __forceinline__ void load_chunk_contig(uint32_t stage_base, const __nv_bfloat16* kbase,
+                                                  const __nv_bfloat16* vbase, int key0,
+                                                  uint32_t valid) {
+    const int lane = threadIdx.x & 31;
+    constexpr int CPR = D / 8;  // 16-byte chunks per row
+#pragma unroll
+    for (int it = 0; it < CPR; ++it) {
+        const int x = it * 32 + lane;
+        const int r = x / CPR, c = x % CPR;
+        const bool ok = (valid >> r) & 1u;
+        const size_t off = (size_t)(ok ? key0 + r : 0) * D + c * 8;
+        const uint32_t so = swz(r, c, WarpSmem<D>::kRowBytes);
+        cp_async16(stage_base + so, kbase + off, ok);
+        cp_async16(stage_base + WarpSmem<D>::kTileBytes + so, vbase + off, ok);
+    }
+}
+
+// S = Q K^T for one chunk (16 x 32), raw logits, masked rows at -inf.
 template <int D>
 __device__ __forceinline__ void chunk_scores(float (&s)[4][4], const uint32_t (&qf)[D / 16][4],
-                                             uint32_t kst, uint32_t valid_mask,
-                                             float scale_log2) {
+                                             uint32_t kst, uint32_t valid_mask) {
     const int lane = threadIdx.x & 31, tig = lane & 3;
 #pragma unroll
     for (int n = 0; n < 4; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
@@ -104,40 +123,52 @@ __device__ __forceinline__ void chunk_scores(float (&s)[4][4], const uint32_t (&
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int col = n * 8 + tig * 2 + (e & 1);
-            s[n][e] = ((valid_mask >> col) & 1u) ? s[n][e] * scale_log2 : -INFINITY;
+            s[n][e] = ((valid_mask >> col) & 1u) ? s[n][e] : -INFINITY;
         }
     }
 }
 
-// Online-softmax update with one chunk of scores, then O += P V.
+__device__ __forceinline__ float ex2f_fast(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Online-softmax update with one chunk of raw logits, then O += P V.  The
+// reference max m (log2 domain) only moves when a chunk exceeds it by more
+// than 2^8, so O is rescaled rarely; p = 2^(s * scale_log2 - m) <= 2^8.
 template <int D>
-__device__ __forceinline__ void chunk_update(AttnState<D>& st, float (&s)[4][4], uint32_t vst) {
+__device__ __forceinline__ void chunk_update(AttnState<D>& st, float (&s)[4][4], uint32_t vst,
+                                             float scale_log2) {
     const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {  // row gid (hr=0) and gid+8 (hr=1)
-        float mx = -INFINITY;
-#pragma unroll
-        for (int n = 0; n < 4; ++n) mx = fmaxf(mx, fmaxf(s[n][2 * hr], s[n][2 * hr + 1]));
+        float mx = fmaxf(fmaxf(fmaxf(s[0][2 * hr], s[0][2 * hr + 1]),
+                               fmaxf(s[1][2 * hr], s[1][2 * hr + 1])),
+                         fmaxf(fmaxf(s[2][2 * hr], s[2][2 * hr + 1]),
+                               fmaxf(s[3][2 * hr], s[3][2 * hr + 1])));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const float m_new = fmaxf(st.m[hr], mx);
-        // all -inf so far: keep exp2 arguments finite
-        const float m_use = m_new == -INFINITY ? 0.f : m_new;
-        const float corr = exp2f(st.m[hr] - m_use);
+        mx *= scale_log2;  // -inf stays -inf
+        if (mx > st.m[hr] + 8.f) {
+            const float corr = ex2f_fast(st.m[hr] - mx);  // 0 while nothing was seen
+            st.l[hr] *= corr;
+#pragma unroll
+            for (int n = 0; n < D / 8; ++n) {
+                st.o[n][2 * hr] *= corr;
+                st.o[n][2 * hr + 1] *= corr;
+            }
+            st.m[hr] = mx;
+        }
+        const float nm = st.m[hr] == -INFINITY ? 0.f : -st.m[hr];
         float sum = 0.f;
 #pragma unroll
         for (int n = 0; n < 4; ++n) {
-            s[n][2 * hr] = exp2f(s[n][2 * hr] - m_use);
-            s[n][2 * hr + 1] = exp2f(s[n][2 * hr + 1] - m_use);
+            s[n][2 * hr] = ex2f_fast(fmaf(s[n][2 * hr], scale_log2, nm));
+            s[n][2 * hr + 1] = ex2f_fast(fmaf(s[n][2 * hr + 1], scale_log2, nm));
             sum += s[n][2 * hr] + s[n][2 * hr + 1];
         }
-        st.l[hr] = st.l[hr] * corr + sum;
-        st.m[hr] = m_new;
-#pragma unroll
-        for (int n = 0; n < D / 8; ++n) {
-            st.o[n][2 * hr] *= corr;
-            st.o[n][2 * hr + 1] *= corr;
-        }
+        st.l[hr] += sum;
     }
     // P (16 x 32) as two k-steps of A fragments.
 #pragma unroll
@@ -169,60 +200,67 @@ __device__ __forceinline__ void finish_rows(AttnState<D>& st) {
     }
 }
 
-// Run the pipeline over n_rows rows; key_of(r) gives the key of list row r
-// (< 0: masked).  Optional per-chunk hook sees the scaled logits before the
-// softmax (used by the decode indexer to export logits).
-template <int D, typename KeyOf, typename Hook>
+// Run the pipeline over n_chunks chunks of 32 rows.  Src describes where
+// chunk c's rows are:
+//   Src::kContig == true:  Src::chunk(c, &key0) -> valid-row mask; rows are the
+//                          consecutive keys key0 .. key0+31;
+//   Src::kContig == false: Src::key(r) -> key of list row r (< 0: masked).
+// The optional per-chunk hook sees the masked raw logits and the chunk's first
+// key (contiguous sources) before the softmax.
+template <int D, typename Src, typename Hook>
 __device__ __forceinline__ void attend_rows(AttnState<D>& st, const uint32_t (&qf)[D / 16][4],
                                             const __nv_bfloat16* kbase,
-                                            const __nv_bfloat16* vbase, int n_rows,
-                                            KeyOf key_of, uint32_t smem_base, float scale_log2,
+                                            const __nv_bfloat16* vbase, int n_chunks,
+                                            const Src& src, uint32_t smem_base, float scale_log2,
                                             Hook hook) {
     const int lane = threadIdx.x & 31;
-    const int n_chunks = (n_rows + kChunk - 1) / kChunk;
-    int keys[kStages];
-    uint32_t masks[kStages];
-    // prologue
-#pragma unroll
-    for (int sgi = 0; sgi < kStages - 1; ++sgi) {
-        if (sgi < n_chunks) {
-            const int r = sgi * kChunk + lane;
-            const int key = r < n_rows ? key_of(r) : -1;
-            keys[sgi] = key;
-            masks[sgi] = __ballot_sync(0xffffffffu, key >= 0);
-            load_chunk<D>(smem_base + sgi * WarpSmem<D>::kStageBytes, kbase, vbase, key);
+    uint32_t mask_a = 0, mask_b = 0;  // valid-row masks of the two stages
+    int key0_a = 0, key0_b = 0;
+    auto issue = [&](int c, uint32_t& mask, int& key0) {
+        const uint32_t sb = smem_base + (c & 1) * WarpSmem<D>::kStageBytes;
+        if constexpr (Src::kContig) {
+            mask = src.chunk(c, &key0);
+            load_chunk_contig<D>(sb, kbase, vbase, key0, mask);
+        } else {
+            const int key = src.key(c * kChunk + lane);
+            mask = __ballot_sync(0xffffffffu, key >= 0);
+            key0 = 0;
+            load_chunk<D>(sb, kbase, vbase, key);
         }
-        cp_async_commit();
-    }
+    };
+    static_assert(kStages == 2, "two-stage ring");
+    if (n_chunks > 0) issue(0, mask_a, key0_a);
+    cp_async_commit();
     for (int c = 0; c < n_chunks; ++c) {
-        const int nxt = c + kStages - 1;
-        if (nxt < n_chunks) {
-            const int r = nxt * kChunk + lane;
-            const int key = r < n_rows ? key_of(r) : -1;
-            keys[nxt % kStages] = key;
-            masks[nxt % kStages] = __ballot_sync(0xffffffffu, key >= 0);
-            load_chunk<D>(smem_base + (nxt % kStages) * WarpSmem<D>::kStageBytes, kbase, vbase,
-                          key);
+        if (c + 1 < n_chunks) {
+            if ((c + 1) & 1) issue(c + 1, mask_b, key0_b);
+            else issue(c + 1, mask_a, key0_a);
         }
         cp_async_commit();
-        cp_async_wait<kStages - 1>();
+        cp_async_wait<1>();
         __syncwarp();
-        const uint32_t sb = smem_base + (c % kStages) * WarpSmem<D>::kStageBytes;
+        const uint32_t sb = smem_base + (c & 1) * WarpSmem<D>::kStageBytes;
+        const uint32_t mask = (c & 1) ? mask_b : mask_a;
+        const int key0 = (c & 1) ? key0_b : key0_a;
         float s[4][4];
-        chunk_scores<D>(s, qf, sb, masks[c % kStages], scale_log2);
-        hook(c, s, keys[c % kStages]);
-        chunk_update<D>(st, s, sb + WarpSmem<D>::kTileBytes);
+        chunk_scores<D>(s, qf, sb, mask);
+        hook(c, s, key0);
+        chunk_update<D>(st, s, sb + WarpSmem<D>::kTileBytes, scale_log2);
         __syncwarp();  // the stage is refilled by the next iteration
     }
     cp_async_wait<0>();
     finish_rows<D>(st);
 }
 
+// Keys first..last (inclusive) as contiguous chunks.
 struct ContiguousKeys {
-    int first, last;  // inclusive range
-    __device__ __forceinline__ int operator()(int r) const {
-        const int key = first + r;
-        return key <= last ? key : -1;
+    static constexpr bool kContig = true;
+    int first, last;
+    __device__ __forceinline__ int n_chunks() const { return (last - first + kChunk) / kChunk; }
+    __device__ __forceinline__ uint32_t chunk(int c, int* key0) const {
+        *key0 = first + c * kChunk;
+        const int n = last - *key0 + 1;  // valid rows in this chunk
+        return n >= 32 ? 0xffffffffu : (n <= 0 ? 0u : ((1u << n) - 1u));
     }
 };
 
@@ -230,7 +268,6 @@ struct ContiguousKeys {
 // Layout [16][D + 2]: m2, l, o[0..D).
 template <int D>
 __device__ __forceinline__ void store_partial(const AttnState<D>& st, float* part, int g) {
-    // part layout: [16][D + 2]: m2, l, o[0..D)
     const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {

@@ -61,19 +61,21 @@ size_t decode_full_workspace(const KParams& p) {
            align256((size_t)p.batch * p.hq * sizeof(float));
 }
 
+// Writes every head's scaled logit a2 = scale_log2 * q.k of the chunk's keys.
 template <int D>
 struct LogitExport {
     float* logits;  // this unit's [t_kv][16]
-    int first, last, g;
-    __device__ __forceinline__ void operator()(int c, float (&s)[4][4], int) const {
+    int last, g;
+    float scale_log2;
+    __device__ __forceinline__ void operator()(int, float (&s)[4][4], int key0) const {
         const int lane = threadIdx.x & 31, gid = lane >> 2, tig = lane & 3;
 #pragma unroll
         for (int n = 0; n < 4; ++n) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int h = gid + 8 * (e >> 1);
-                const int key = first + c * kChunk + n * 8 + tig * 2 + (e & 1);
-                if (h < g && key <= last) logits[(size_t)key * 16 + h] = s[n][e];
+                const int key = key0 + n * 8 + tig * 2 + (e & 1);
+                if (h < g && key <= last) logits[(size_t)key * 16 + h] = s[n][e] * scale_log2;
             }
         }
     }
@@ -103,9 +105,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
         uint32_t qf[D / 16][4];
         load_q_frags<D>(qf, q + ((size_t)b * p.hq + u * g) * D, D, g);
         const size_t kvoff = (size_t)unit * p.t_kv * D;
-        LogitExport<D> hook{ws.logits + (size_t)unit * p.t_kv * 16, first, last, g};
-        attend_rows<D>(st, qf, kc + kvoff, vc + kvoff, last - first + 1,
-                       ContiguousKeys{first, last}, sbase, p.scale_log2, hook);
+        LogitExport<D> hook{ws.logits + (size_t)unit * p.t_kv * 16, last, g, p.scale_log2};
+        const ContiguousKeys src{first, last};
+        attend_rows<D>(st, qf, kc + kvoff, vc + kvoff, src.n_chunks(), src, sbase, p.scale_log2,
+                       hook);
     }
     store_partial<D>(st, ws.part + (size_t)task * 16 * (D + 2), g);
 }

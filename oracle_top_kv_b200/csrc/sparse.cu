@@ -23,10 +23,14 @@
 namespace hs {
 
 // Key of row r of the gathered list, -1 if masked; flags out-of-range ids.
+// Token mode: the selected keys themselves.  Block mode: block r / B, offset
+// r % B, clipped to keys <= t (a selected block may cross the query).
 struct GatherKeys {
+    static constexpr bool kContig = false;
     const int32_t* ids;
-    int n_ids, B, t, mode;
-    __device__ __forceinline__ int operator()(int r) const {
+    int n_rows, B, t, mode;
+    __device__ __forceinline__ int key(int r) const {
+        if (r >= n_rows) return -1;
         if (mode == 0) {
             const int jb = r / B;
             const int id = ids[jb];
@@ -38,8 +42,29 @@ struct GatherKeys {
         if (key < 0 || key > t) { set_status(HS_ERR_BOUNDS); return -1; }
         return key;
     }
+    __device__ __forceinline__ int operator()(int r) const { return key(r); }
 };
 
+// Block mode with B a multiple of 32: every 32-row chunk is 32 consecutive
+// keys of one selected block, so it is loaded as one contiguous range.
+struct BlockChunks {
+    static constexpr bool kContig = true;
+    const int32_t* ids;
+    int B, t;
+    __device__ __forceinline__ uint32_t chunk(int c, int* key0) const {
+        const int per = B / kChunk;
+        const int jb = c / per;
+        const int id = ids[jb];
+        if (id < 0 || id > t / B) {
+            set_status(HS_ERR_BOUNDS);
+            *key0 = 0;
+            return 0u;
+        }
+        *key0 = id * B + (c - jb * per) * kChunk;
+        const int n = t - *key0 + 1;
+        return n >= 32 ? 0xffffffffu : (n <= 0 ? 0u : ((1u << n) - 1u));
+    }
+};
 
 __device__ __forceinline__ int clamp_count(int c, int ksel) {
     if (c < 0 || c > ksel) { set_status(HS_ERR_BOUNDS); return c < 0 ? 0 : ksel; }
@@ -115,14 +140,15 @@ __global__ void sparse_simt_kernel(KParams p, const T* __restrict__ q, const T* 
     const size_t orow = ((size_t)b * p.hq + h) * p.t_q + j;
     const size_t kvoff = ((size_t)b * p.hkv + u) * p.t_kv * D;
     const int c = clamp_count(cnt[row], p.ksel);
-    GatherKeys keys{idx + row * p.ksel, c, p.block_size, t, p.mode};
     const int n_rows = p.mode == 0 ? c * p.block_size : c;
+    GatherKeys keys{idx + row * p.ksel, n_rows, p.block_size, t, p.mode};
     simt_attend<T, D>(qs + warp * D, kf + kvoff, vf + kvoff, n_rows, keys, og + orow * D,
                       lseg + orow);
     if (kl) {
         const int first = max(0, t - p.window + 1);
         simt_attend<T, D>(qs + warp * D, kl + kvoff, vl + kvoff, t - first + 1,
-                          ContiguousKeys{first, t}, ol + orow * D, lsel + orow);
+                          [=](int r) { return first + r <= t ? first + r : -1; }, ol + orow * D,
+                          lsel + orow);
     }
 }
 
@@ -157,7 +183,7 @@ cudaError_t launch_sparse_simt(const KParams& p, int dtype, const void* q, const
 }
 
 // ------------------------------------------------------------ tensor-core path
-constexpr int kSparseWarps = 4;
+constexpr int kSparseWarps = 6;
 
 // Normalise and store rows < g of a finished warp state.
 template <int D>
@@ -210,19 +236,27 @@ __global__ void __launch_bounds__(kSparseWarps * 32)
     const size_t row = ((size_t)b * p.hkv + u) * p.t_q + j;
     const size_t kvoff = ((size_t)b * p.hkv + u) * p.t_kv * D;
     const int c = clamp_count(cnt[row], p.ksel);
-    GatherKeys keys{idx + row * p.ksel, c, p.block_size, t, p.mode};
     const int n_rows = p.mode == 0 ? c * p.block_size : c;
+    GatherKeys keys{idx + row * p.ksel, n_rows, p.block_size, t, p.mode};
 
     AttnState<D> st;
     st.init();
-    attend_rows<D>(st, qf, kf + kvoff, vf + kvoff, n_rows, keys, sbase, p.scale_log2, NoHook{});
+    if (p.mode == 0 && p.block_size % kChunk == 0) {
+        BlockChunks src{idx + row * p.ksel, p.block_size, t};
+        attend_rows<D>(st, qf, kf + kvoff, vf + kvoff, c * (p.block_size / kChunk), src, sbase,
+                       p.scale_log2, NoHook{});
+    } else {
+        attend_rows<D>(st, qf, kf + kvoff, vf + kvoff, (n_rows + kChunk - 1) / kChunk, keys,
+                       sbase, p.scale_log2, NoHook{});
+    }
     store_rows<D>(st, og + q0 * D, head_stride, lseg + q0, p.t_q, g);
     if (kl) {
         const int first = max(0, t - p.window + 1);
         AttnState<D> sl;
         sl.init();
-        attend_rows<D>(sl, qf, kl + kvoff, vl + kvoff, t - first + 1, ContiguousKeys{first, t},
-                       sbase, p.scale_log2, NoHook{});
+        const ContiguousKeys win{first, t};
+        attend_rows<D>(sl, qf, kl + kvoff, vl + kvoff, win.n_chunks(), win, sbase, p.scale_log2,
+                       NoHook{});
         store_rows<D>(sl, ol + q0 * D, head_stride, lsel + q0, p.t_q, g);
     }
 }
@@ -290,8 +324,8 @@ __global__ void __launch_bounds__(kSparseWarps * 32)
         load_q_frags<D>(qf, q + ((size_t)b * p.hq + u * g) * D, D, g);
         GatherKeys keys{idx + (size_t)unit * p.ksel + r0, n_rows, 1, t, 1};
         const size_t kvoff = (size_t)unit * p.t_kv * D;
-        attend_rows<D>(st, qf, kc + kvoff, vc + kvoff, n_rows, keys, sbase, p.scale_log2,
-                       NoHook{});
+        attend_rows<D>(st, qf, kc + kvoff, vc + kvoff, (n_rows + kChunk - 1) / kChunk, keys,
+                       sbase, p.scale_log2, NoHook{});
     } else if (sp == 0 && (threadIdx.x & 31) == 0) {
         set_status(HS_ERR_BOUNDS);
     }

@@ -153,6 +153,32 @@ hs_status hs_decode_step(const hs_params* p, int32_t kind, const void* q,
                          int32_t* idx, int32_t* idx_count, void* o, float* lse,
                          float* sel_scores, void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * The sparse decode step of hs_decode_step(HS_DECODE_SPARSE), for callers that
+ * cannot allocate device memory -- e.g. a plugin that only receives its input
+ * and output buffers from an engine whose memory planner owns all device
+ * memory, or a decode loop that must not call cudaMalloc (it can synchronise
+ * the device).  It takes no workspace and allocates nothing: its scratch is a
+ * fixed 32 MiB array inside the library, present on every GPU that loads the
+ * library until the process exits.  (The pages have no counterpart of this
+ * entry point; it only changes where the scratch lives.)
+ *
+ * Arguments, layouts and results are those of hs_decode_step with
+ * kind = HS_DECODE_SPARSE.  Limits: batch * hkv * ceil(k / 64) split units of
+ * 16 * (head_dim + 2) floats must fit in the 32 MiB (4032 units at
+ * head_dim 128, e.g. 32 sequences x 4 kv groups x k = 1024); larger calls
+ * return HS_ERR_WORKSPACE without launching anything.
+ * The first call on a device looks up the array's device address (with that
+ * device current); make that first call before any stream capture.  All calls
+ * on a device share the one array: calls whose kernels could overlap on the
+ * GPU (e.g. on unordered streams) race and must not be issued.  Nothing
+ * persists from one call to the next.
+ */
+hs_status hs_decode_sparse_noalloc(const hs_params* p, const void* q, const void* k_cache,
+                                   const void* v_cache, const int32_t* seq_len,
+                                   const int32_t* idx, const int32_t* idx_count, void* o,
+                                   float* lse, void* stream);
+
 enum { HS_WS_FULL = 0, HS_WS_SPARSE = 1, HS_WS_DECODE_FULL = 2, HS_WS_DECODE_SPARSE = 3 };
 
 /* Bytes of workspace the matching entry point needs for these parameters

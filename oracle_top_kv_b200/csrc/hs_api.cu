@@ -16,6 +16,7 @@
 #include "decode_full.cu"
 #include "full_simt.cu"
 #include "full_tc.cu"
+#include "noalloc.cu"
 #include "sparse.cu"
 
 namespace hs {
@@ -205,6 +206,25 @@ hs_status hs_decode_step(const hs_params* p, int32_t kind, const void* q, const 
     return launched(2, [&] {
         return hs::launch_decode_sparse(kp, q, k_cache, v_cache, seq_len, idx, idx_count, o, lse,
                                         workspace, st);
+    });
+}
+
+hs_status hs_decode_sparse_noalloc(const hs_params* p, const void* q, const void* k_cache,
+                                   const void* v_cache, const int32_t* seq_len,
+                                   const int32_t* idx, const int32_t* idx_count, void* o,
+                                   float* lse, void* stream) {
+    KParams kp;
+    hs_status s = resolve(p, true, &kp);
+    if (s != HS_OK) return s;
+    if (p->dtype != HS_BF16 || p->mode != HS_SEL_TOKEN) return HS_ERR_UNSUPPORTED;
+    if (!ok_ptr(q) || !ok_ptr(k_cache) || !ok_ptr(v_cache) || !ok_ptr(seq_len) || !ok_ptr(idx) ||
+        !ok_ptr(idx_count) || !ok_ptr(o) || !ok_opt(lse))
+        return HS_ERR_INVALID_ARG;
+    if (hs::decode_sparse_workspace(kp) > hs::noalloc_scratch_bytes()) return HS_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return launched(2, [&] {
+        return hs::launch_decode_sparse_noalloc(kp, q, k_cache, v_cache, seq_len, idx, idx_count,
+                                                o, lse, st);
     });
 }
 

@@ -53,4 +53,11 @@ cudaError_t launch_decode_sparse(const KParams& p, const void* q, const void* kc
                                  const int32_t* seq_len, const int32_t* idx, const int32_t* cnt,
                                  void* o, float* lse, void* ws, cudaStream_t st);
 
+// Sparse decode step with its scratch in a file-scope device array.
+size_t noalloc_scratch_bytes();
+cudaError_t launch_decode_sparse_noalloc(const KParams& p, const void* q, const void* kc,
+                                         const void* vc, const int32_t* seq_len,
+                                         const int32_t* idx, const int32_t* cnt, void* o,
+                                         float* lse, cudaStream_t st);
+
 }  // namespace hs

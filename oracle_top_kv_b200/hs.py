@@ -25,7 +25,7 @@ HS_DECODE_FULL_INDEX, HS_DECODE_SPARSE = 0, 1
 HS_WS_FULL, HS_WS_SPARSE, HS_WS_DECODE_FULL, HS_WS_DECODE_SPARSE = 0, 1, 2, 3
 
 EXPORTS = ("hs_full_attn_index", "hs_sparse_attn_reuse", "hs_decode_step", "hs_workspace_size",
-           "hs_device_status", "hs_status_string", "hs_launch_count")
+           "hs_device_status", "hs_status_string", "hs_launch_count", "hs_decode_sparse_noalloc")
 
 
 class HsError(RuntimeError):
@@ -71,6 +71,7 @@ def load(path: str = LIB_PATH):
     lib.hs_full_attn_index.argtypes = [PP, P, P, P, P, P, P, P, P, P, S, P]
     lib.hs_sparse_attn_reuse.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, P, P, S, P]
     lib.hs_decode_step.argtypes = [PP, I32, P, P, P, P, P, P, P, P, P, P, S, P]
+    lib.hs_decode_sparse_noalloc.argtypes = [PP, P, P, P, P, P, P, P, P, P]
     lib.hs_workspace_size.argtypes = [PP, I32]
     lib.hs_workspace_size.restype = S
     lib.hs_device_status.argtypes = [P, ctypes.POINTER(I32)]
@@ -79,7 +80,7 @@ def load(path: str = LIB_PATH):
     lib.hs_launch_count.argtypes = []
     lib.hs_launch_count.restype = ctypes.c_uint64
     for name in ("hs_full_attn_index", "hs_sparse_attn_reuse", "hs_decode_step",
-                 "hs_device_status"):
+                 "hs_device_status", "hs_decode_sparse_noalloc"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -145,6 +146,15 @@ def hs_decode_step(p, kind, q, k_cache, v_cache, seq_len, idx, idx_count, o, lse
     _check(lib.hs_decode_step(ctypes.byref(p), int(kind), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                               _ptr(seq_len), _ptr(idx), _ptr(idx_count), _ptr(o), _ptr(lse),
                               _ptr(sel_scores), wp, wb, _stream(stream)), "hs_decode_step")
+
+
+def hs_decode_sparse_noalloc(p, q, k_cache, v_cache, seq_len, idx, idx_count, o, lse=None,
+                             stream=None):
+    """hs_decode_step(HS_DECODE_SPARSE) without a workspace (library-owned scratch)."""
+    _check(load().hs_decode_sparse_noalloc(ctypes.byref(p), _ptr(q), _ptr(k_cache),
+                                           _ptr(v_cache), _ptr(seq_len), _ptr(idx),
+                                           _ptr(idx_count), _ptr(o), _ptr(lse), _stream(stream)),
+           "hs_decode_sparse_noalloc")
 
 
 def hs_workspace_size(p, which) -> int:

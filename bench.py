@@ -38,6 +38,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from oracle_top_kv_b200 import accounting as A  # noqa: E402
+from oracle_top_kv_b200 import dist as hdist  # noqa: E402
 from oracle_top_kv_b200 import workloads as wl  # noqa: E402
 
 METRIC = "full+index prefill TFLOP/s and sparse-reuse KV GB/s (fraction of B200 peak)"
@@ -224,8 +225,7 @@ def run_ours(args, rank, world, device):
     clocks = ClockSampler(device)
     clocks.start()
     time.sleep(0.5)
-    if world > 1:
-        torch.distributed.barrier()
+    hdist.barrier(device)
     torch.cuda.synchronize(device)
     launches0 = hs.hs_launch_count()
     t0 = torch.cuda.Event(enable_timing=True)
@@ -241,14 +241,9 @@ def run_ours(args, rank, world, device):
     t1.record(stream)
     torch.cuda.synchronize(device)
     launches = hs.hs_launch_count() - launches0
-    if world > 1:
-        torch.distributed.barrier()
+    hdist.barrier(device)
     clocks.stop()
-    total_ms = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([total_ms], device=device)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = hdist.max_over_ranks(t0.elapsed_time(t1), device)
     assert hs.hs_device_status(sh) == 0
     full_ms = [evs[s][0].elapsed_time(evs[s][1]) for s in range(args.steps)]
     sparse_ms = [evs[s][1 + l].elapsed_time(evs[s][2 + l]) for s in range(args.steps)
@@ -325,8 +320,7 @@ def run_e2e(args, blk, w, stream, ideal, world, device):
     n = max(1, min(args.steps, 3))
     step()
     torch.cuda.synchronize(device)
-    if world > 1:
-        torch.distributed.barrier()
+    hdist.barrier(device)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -334,11 +328,7 @@ def run_e2e(args, blk, w, stream, ideal, world, device):
         step()
     e1.record(stream)
     torch.cuda.synchronize(device)
-    ms = e0.elapsed_time(e1) / n
-    if world > 1:
-        tt = torch.tensor([ms], device=device)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = hdist.max_over_ranks(e0.elapsed_time(e1) / n, device)
     return {"value": world * ideal / (ms / 1e3), "unit": UNIT, "ms_per_step": ms,
             "steps": n, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
@@ -433,9 +423,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = hdist.world()
     w = workload_of(args)
 
     if args.impl == "reference":
@@ -446,9 +434,7 @@ def main():
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     if world > 1:
-        import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=device)
+        hdist.init("nccl", device)
     line = run_ours(args, rank, world, device)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         t, sample, cores = oracle_sample_time(w, oracle_inputs(w))

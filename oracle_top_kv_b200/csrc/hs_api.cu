@@ -16,6 +16,7 @@
 #include "decode_full.cu"
 #include "full_simt.cu"
 #include "full_tc.cu"
+#include "token_select_tc.cu"
 #include "noalloc.cu"
 #include "sparse.cu"
 
@@ -125,6 +126,8 @@ hs_status hs_full_attn_index(const hs_params* p, const void* q, const void* k, c
             cudaError_t e =
                 hs::launch_full_tc(kp, q, k, v, o, lse, idx, idx_count, sel_scores, 0, st);
             if (e != cudaSuccess) return e;
+            if (hs::token_select_tc_supported(kp, p->dtype))
+                return hs::launch_token_select_tc(kp, q, k, lse, idx, idx_count, sel_scores, st);
             return hs::launch_full_simt(kp, p->dtype, q, k, v, o, lse, idx, idx_count,
                                         sel_scores, 0, st);
         });

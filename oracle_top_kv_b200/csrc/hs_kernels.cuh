@@ -53,6 +53,13 @@ cudaError_t launch_decode_sparse(const KParams& p, const void* q, const void* kc
                                  const int32_t* seq_len, const int32_t* idx, const int32_t* cnt,
                                  void* o, float* lse, void* ws, cudaStream_t st);
 
+// Token-mode selection on the tensor cores (bf16, d = 128, 16 heads per group,
+// k - w <= 1024); reads lse from the attention pass.
+bool token_select_tc_supported(const KParams& p, int dtype);
+cudaError_t launch_token_select_tc(const KParams& p, const void* q, const void* k,
+                                   const float* lse, int32_t* idx, int32_t* cnt, float* sel,
+                                   cudaStream_t st);
+
 // Sparse decode step with its scratch in a file-scope device array.
 size_t noalloc_scratch_bytes();
 cudaError_t launch_decode_sparse_noalloc(const KParams& p, const void* q, const void* kc,

@@ -162,14 +162,68 @@ class HybridBlock:
         return t
 
 
+class DecodeBlock:
+    """One decode step of a HySparse2 block: the full layer's step over the
+    whole cache (index selection for the new token), then the block's sparse
+    layers gathering the selected rows of the same cache."""
+
+    def __init__(self, w, device):
+        from oracle_top_kv_b200 import hs
+        self.hs = hs
+        self.w = w
+        q, kc, vc, _ = wl.full_layer_inputs(w, device=device)
+        self.q, self.k, self.v = q, kc, vc
+        self.seq = wl.decode_seq_lens(w, ragged=False, device=device)
+        self.p = hs.make_params(w.batch, w.hq, w.hkv, w.head_dim, 1, w.t, 0, w.dtype, w.mode,
+                                w.block_size, w.k, w.window)
+        ks = self.p.ksel
+        self.idx = torch.empty(w.batch, w.hkv, ks, dtype=torch.int32, device=device)
+        self.cnt = torch.empty(w.batch, w.hkv, dtype=torch.int32, device=device)
+        self.o = torch.empty_like(q)
+        self.lse = torch.empty(w.batch, w.hq, 1, dtype=torch.float32, device=device)
+        self.ws_full = hs.workspace(self.p, hs.HS_WS_DECODE_FULL, device)
+        self.ws_sp = hs.workspace(self.p, hs.HS_WS_DECODE_SPARSE, device)
+        self.qs = [wl.sparse_layer_query(w, l, device=device) for l in range(w.n_sparse)]
+        self.os = [torch.empty_like(x) for x in self.qs]
+        self.ls = [torch.empty(w.batch, w.hq, 1, dtype=torch.float32, device=device)
+                   for _ in self.qs]
+
+    def full(self, stream):
+        self.hs.hs_decode_step(self.p, self.hs.HS_DECODE_FULL_INDEX, self.q, self.k, self.v,
+                               self.seq, self.idx, self.cnt, self.o, self.lse, None, self.ws_full,
+                               stream)
+
+    def sparse(self, layer, stream):
+        self.hs.hs_decode_step(self.p, self.hs.HS_DECODE_SPARSE, self.qs[layer], self.k, self.v,
+                               self.seq, self.idx, self.cnt, self.os[layer], self.ls[layer], None,
+                               self.ws_sp, stream)
+
+    def inputs(self):
+        # per-step inputs: the new token's queries; the K/V cache is resident state
+        return [self.q, self.seq] + self.qs
+
+    def outputs(self):
+        return [self.o, self.lse, self.idx, self.cnt] + self.os + self.ls
+
+
 def work(w, blk):
-    """Algorithmic FLOPs of the full layer and bytes of each sparse layer."""
+    """Algorithmic FLOPs of the full layer and bytes of each sparse layer.
+    Decode: the full layer is counted in bytes (the whole cache), returned as
+    (full_bytes, sparse_bytes) with flops = None."""
+    if w.decode:
+        elt = 2
+        full_b = A.decode_full_bytes(w.batch, w.hkv, w.head_dim, blk.seq.tolist(), elt)
+        full_b += w.batch * w.hq * w.head_dim * elt * 2  # q in, o out
+        rows = int(blk.cnt.sum().item())
+        sp = rows * 2 * w.head_dim * elt + w.batch * w.hq * (w.head_dim * elt * 2 + 4)
+        sp += w.batch * w.hkv * (w.ksel + 1) * 4
+        return None, full_b, sp
     flops = A.full_layer_flops(w.batch, w.hq, w.head_dim, w.tq, w.q_offset)
     rows = A.sparse_rows_from_index(blk.idx, blk.cnt, w.mode, w.block_size, w.q_offset)
     local = A.window_rows(w.batch, w.hkv, w.tq, w.window, w.q_offset) if w.swa_branch else 0
     elt = 2 if w.dtype == "bf16" else 4
     sbytes = A.sparse_layer_bytes(rows, w.batch, w.hq, w.tq, w.head_dim, elt, w.ksel, w.hkv, local)
-    return flops, sbytes
+    return flops, None, sbytes
 
 
 def traffic_for(kernel, workload):
@@ -204,7 +258,7 @@ def run_ours(args, rank, world, device):
     hs.load()
     w = workload_of(args)
     peaks, peak_kind = load_peaks()
-    blk = HybridBlock(w, device)
+    blk = DecodeBlock(w, device) if w.decode else HybridBlock(w, device)
     stream = torch.cuda.current_stream(device)
     sh = stream.cuda_stream
 
@@ -217,7 +271,7 @@ def run_ours(args, rank, world, device):
         step()
     torch.cuda.synchronize(device)
     assert hs.hs_device_status(sh) == 0
-    flops, sbytes = work(w, blk)
+    flops, full_bytes, sbytes = work(w, blk)
 
     n_ev = 1 + w.n_sparse
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev + 1)]
@@ -254,25 +308,36 @@ def run_ours(args, rank, world, device):
     p_hbm = peaks["hbm_gbs"] * 1e9
     full_s = statistics.mean(full_ms) / 1e3
     sparse_s = statistics.mean(sparse_ms) / 1e3
-    ideal = flops / p_tensor + w.n_sparse * sbytes / p_hbm
-    value = world * ideal / (ms_step / 1e3)
-    full_tflops = flops / full_s / 1e12
     sparse_gbs = sbytes / sparse_s / 1e9
     tokens = w.batch * w.tq
+    if flops is not None:
+        ideal = flops / p_tensor + w.n_sparse * sbytes / p_hbm
+        full_rate, full_unit, full_peak = flops / full_s / 1e12, "TFLOP/s", peaks["bf16_tflops_sustained"]
+        full_bound, full_peak_src = "tensor", f"{peak_kind} bf16_tflops_sustained"
+    else:
+        ideal = (full_bytes + w.n_sparse * sbytes) / p_hbm
+        full_rate, full_unit, full_peak = full_bytes / full_s / 1e9, "GB/s", peaks["hbm_gbs"]
+        full_bound, full_peak_src = "hbm", f"{peak_kind} hbm_gbs"
+    value = world * ideal / (ms_step / 1e3)
     # dominant kernel: the one with the larger share of the step
     if sum(full_ms) >= sum(sparse_ms):
-        roof = {"kernel": "full_attn_index", "bound": "tensor", "achieved": full_tflops,
-                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                "frac": full_tflops / peaks["bf16_tflops_sustained"],
-                "traffic": traffic_for("full_attn_index", w.name),
-                "peak_source": f"{peak_kind} bf16_tflops_sustained",
-                "work_per_launch": flops, "avg_launch_ms": full_s * 1e3}
+        roof = {"kernel": "decode_full_index" if w.decode else "full_attn_index",
+                "bound": full_bound, "achieved": full_rate, "peak": full_peak,
+                "unit": full_unit, "frac": full_rate / full_peak,
+                "traffic": traffic_for("decode_full_index" if w.decode else "full_attn_index",
+                                       w.name),
+                "peak_source": full_peak_src,
+                "work_per_launch": flops if flops is not None else full_bytes,
+                "avg_launch_ms": full_s * 1e3}
     else:
-        roof = {"kernel": "sparse_attn_reuse", "bound": "hbm", "achieved": sparse_gbs,
-                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": sparse_gbs / peaks["hbm_gbs"],
-                "traffic": traffic_for("sparse_attn_reuse", w.name),
+        roof = {"kernel": "decode_sparse" if w.decode else "sparse_attn_reuse", "bound": "hbm",
+                "achieved": sparse_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": sparse_gbs / peaks["hbm_gbs"],
+                "traffic": traffic_for("decode_sparse" if w.decode else "sparse_attn_reuse",
+                                       w.name),
                 "peak_source": f"{peak_kind} hbm_gbs",
                 "work_per_launch": sbytes, "avg_launch_ms": sparse_s * 1e3}
+    full_key = "full_index_gbs" if flops is None else "full_index_tflops"
 
     e2e = run_e2e(args, blk, w, stream, ideal, world, device) if not args.no_e2e else None
     line = {
@@ -282,10 +347,11 @@ def run_ours(args, rank, world, device):
         "config": {"workload": w.name, "batch": w.batch, "seq_len": w.t, "hq": w.hq,
                    "hkv": w.hkv, "head_dim": w.head_dim, "mode": w.mode,
                    "block_size": w.block_size, "k": w.k, "window": w.window,
+                   "decode": w.decode, "t_q": w.tq, "q_offset": w.q_offset,
                    "sparse_layers": w.n_sparse, "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2 (step reads > 1 GB; K^F+V^F alone 134 MB)"},
-        "full_index_tflops": full_tflops * world,
-        "full_index_frac_of_peak": full_tflops / peaks["bf16_tflops_sustained"],
+        full_key: full_rate * world,
+        "full_index_frac_of_peak": full_rate / full_peak,
         "sparse_kv_gbs": sparse_gbs * world,
         "sparse_frac_of_hbm_peak": sparse_gbs / peaks["hbm_gbs"],
         "full_ms": full_s * 1e3, "sparse_ms_per_layer": sparse_s * 1e3,
@@ -355,10 +421,20 @@ def oracle_sample_time(w, inputs, budget_rows=48, seed=0):
     import oracle
     q, k, v, layers = inputs
     rng = np.random.default_rng(seed)
-    js = np.unique(np.linspace(0, w.tq - 1, budget_rows).astype(int))
-    rows = np.array([(int(rng.integers(0, w.batch)), int(rng.integers(0, w.hkv)), int(j))
-                     for j in js], np.int32)
-    pos = w.q_offset + rows[:, 2]
+    if w.decode:
+        # rows = (sequence, kv group) units at the newest position
+        n_units = w.batch * w.hkv
+        pick = rng.choice(n_units, size=min(n_units, max(1, budget_rows // 8)), replace=False)
+        rows = np.array([(int(x) // w.hkv, int(x) % w.hkv, 0) for x in pick], np.int32)
+        pos = np.full(len(rows), w.t - 1)
+        n_all, full_scale = n_units, n_units / len(rows)
+    else:
+        js = np.unique(np.linspace(0, w.tq - 1, budget_rows).astype(int))
+        rows = np.array([(int(rng.integers(0, w.batch)), int(rng.integers(0, w.hkv)), int(j))
+                         for j in js], np.int32)
+        pos = w.q_offset + rows[:, 2]
+        n_all = w.batch * w.hkv * w.tq
+        full_scale = w.batch * w.hkv * A.causal_pairs(w.tq, w.q_offset) / float((pos + 1).sum())
     t0 = time.perf_counter()
     orc = oracle.full_attn_rows(q, k, v, rows, pos, w.mode, w.block_size, w.k, w.window)
     t_full = time.perf_counter() - t0
@@ -368,9 +444,7 @@ def oracle_sample_time(w, inputs, budget_rows=48, seed=0):
         oracle.sparse_attn_rows(qs, k, v, orc["idx"], orc["cnt"], rows, pos, w.mode,
                                 w.block_size, w.k, w.window, kl, vl)
         t_sp += time.perf_counter() - t0
-    n_all = w.batch * w.hkv * w.tq
-    all_pairs = w.batch * w.hkv * A.causal_pairs(w.tq, w.q_offset)
-    est_full = t_full * all_pairs / float((pos + 1).sum())
+    est_full = t_full * full_scale
     est_sparse = t_sp * n_all / len(rows)
     sample = (f"{len(rows)} query rows (all heads of their group) through the full layer and "
               f"{w.n_sparse} sparse layers, timed {t_full + t_sp:.2f} s, extrapolated to the "
@@ -380,12 +454,16 @@ def oracle_sample_time(w, inputs, budget_rows=48, seed=0):
 
 def cpu_value(w, t_step):
     peaks, _ = load_peaks()
+    p_hbm = peaks["hbm_gbs"] * 1e9
+    if w.decode:
+        full_b = A.decode_full_bytes(w.batch, w.hkv, w.head_dim, [w.t] * w.batch, 2)
+        sp = w.batch * w.hkv * min(w.k, w.t) * 2 * w.head_dim * 2
+        return (full_b + w.n_sparse * sp) / p_hbm / t_step
     flops = A.full_layer_flops(w.batch, w.hq, w.head_dim, w.tq, w.q_offset)
     rows = w.batch * w.hkv * sum(min(w.k, w.q_offset + j + 1) for j in range(w.tq))
     local = A.window_rows(w.batch, w.hkv, w.tq, w.window, w.q_offset) if w.swa_branch else 0
     sbytes = A.sparse_layer_bytes(rows, w.batch, w.hq, w.tq, w.head_dim, 2, w.ksel, w.hkv, local)
-    ideal = (flops / (peaks["bf16_tflops_sustained"] * 1e12) +
-             w.n_sparse * sbytes / (peaks["hbm_gbs"] * 1e9))
+    ideal = (flops / (peaks["bf16_tflops_sustained"] * 1e12) + w.n_sparse * sbytes / p_hbm)
     return ideal / t_step
 
 

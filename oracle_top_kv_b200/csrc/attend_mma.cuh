@@ -5,12 +5,15 @@
 // The 16 MMA rows are the heads of the group, so every gathered K/V row is
 // loaded once and used by all of them ("HySparse 混合稀疏注意力（一）", GQA:
 // the group shares one index set so each selected row is read once).  Rows are
-// fetched 32 at a time with 16-byte cp.async into a 2-stage, XOR-swizzled
-// shared-memory ring owned by the warp; masked rows are zero-filled and get a
-// -inf logit.
+// fetched 32 at a time into a 2-stage shared-memory ring owned by the warp:
+// runs of consecutive keys (selected blocks, windows, cache splits) by TMA
+// (one lane, 2-D boxes, 128-byte swizzle), gathered keys (token selection) by
+// 16-byte cp.async into the same swizzled layout.  Masked rows get a -inf
+// logit.
 #pragma once
 
 #include "hs_common.cuh"
+#include "tc_ptx.cuh"
 
 namespace hs {
 
@@ -24,6 +27,14 @@ struct WarpSmem {
     static constexpr int kStageBytes = 2 * kTileBytes;  // K tile + V tile
     static constexpr int kBytes = kStages * kStageBytes;
 };
+
+// Byte offset of 16-byte chunk c (elements 8c..8c+7) of row `row` in a tile of
+// kChunk rows: the tile is stored as d-halves of [kChunk][64] elements with
+// 128-byte rows, each XOR-swizzled by the row -- exactly the layout a TMA box
+// {64, kChunk} with 128-byte swizzle writes at a 1 KB-aligned address.
+__device__ __forceinline__ uint32_t tile_off(int row, int c) {
+    return (uint32_t)(((c >> 3) * (kChunk * 128)) + row * 128 + (((c & 7) ^ (row & 7)) << 4));
+}
 
 // Online-softmax state of one warp: rows gid and gid+8 of the 16-row tile.
 template <int D>
@@ -73,7 +84,7 @@ __device__ __forceinline__ void load_chunk(uint32_t stage_base, const __nv_bfloa
         const int key = __shfl_sync(0xffffffffu, my_key, r);
         const bool ok = key >= 0;
         const size_t off = (size_t)(ok ? key : 0) * D + c * 8;
-        const uint32_t so = swz(r, c, WarpSmem<D>::kRowBytes);
+        const uint32_t so = tile_off(r, c);
         cp_async16(stage_base + so, kbase + off, ok);
         cp_async16(stage_base + WarpSmem<D>::kTileBytes + so, vbase + off, ok);
     }
@@ -93,7 +104,7 @@ __device__ __forceinline__ void load_chunk_contig(uint32_t stage_base, const __n
         const int r = x / CPR, c = x % CPR;
         const bool ok = (valid >> r) & 1u;
         const size_t off = (size_t)(ok ? key0 + r : 0) * D + c * 8;
-        const uint32_t so = swz(r, c, WarpSmem<D>::kRowBytes);
+        const uint32_t so = tile_off(r, c);
         cp_async16(stage_base + so, kbase + off, ok);
         cp_async16(stage_base + WarpSmem<D>::kTileBytes + so, vbase + off, ok);
     }
@@ -113,7 +124,7 @@ __device__ __forceinline__ void chunk_scores(float (&s)[4][4], const uint32_t (&
             const int key = np * 16 + (lane & 7) + ((lane >> 4) << 3);
             const int chunk = kk * 2 + ((lane >> 3) & 1);
             uint32_t b0, b1, b2, b3;
-            ldsm_x4(kst + swz(key, chunk, WarpSmem<D>::kRowBytes), b0, b1, b2, b3);
+            ldsm_x4(kst + tile_off(key, chunk), b0, b1, b2, b3);
             mma_bf16(s[np * 2], qf[kk], b0, b1);
             mma_bf16(s[np * 2 + 1], qf[kk], b2, b3);
         }
@@ -183,7 +194,7 @@ __device__ __forceinline__ void chunk_update(AttnState<D>& st, float (&s)[4][4],
             const int key = ks * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
             const int chunk = dp * 2 + (lane >> 4);
             uint32_t b0, b1, b2, b3;
-            ldsm_x4_t(vst + swz(key, chunk, WarpSmem<D>::kRowBytes), b0, b1, b2, b3);
+            ldsm_x4_t(vst + tile_off(key, chunk), b0, b1, b2, b3);
             mma_bf16(st.o[dp * 2], a, b0, b1);
             mma_bf16(st.o[dp * 2 + 1], a, b2, b3);
         }
@@ -200,56 +211,122 @@ __device__ __forceinline__ void finish_rows(AttnState<D>& st) {
     }
 }
 
-// Run the pipeline over n_chunks chunks of 32 rows.  Src describes where
-// chunk c's rows are:
-//   Src::kContig == true:  Src::chunk(c, &key0) -> valid-row mask; rows are the
-//                          consecutive keys key0 .. key0+31;
-//   Src::kContig == false: Src::key(r) -> key of list row r (< 0: masked).
-// The optional per-chunk hook sees the masked raw logits and the chunk's first
-// key (contiguous sources) before the softmax.
+// Run the pipeline over n_chunks chunks of 32 gathered rows; src.key(r) gives
+// the key of list row r (< 0: masked).  cp.async, 2 stages.
 template <int D, typename Src, typename Hook>
 __device__ __forceinline__ void attend_rows(AttnState<D>& st, const uint32_t (&qf)[D / 16][4],
                                             const __nv_bfloat16* kbase,
                                             const __nv_bfloat16* vbase, int n_chunks,
                                             const Src& src, uint32_t smem_base, float scale_log2,
                                             Hook hook) {
+    static_assert(!Src::kContig, "gathered rows");
     const int lane = threadIdx.x & 31;
     uint32_t mask_a = 0, mask_b = 0;  // valid-row masks of the two stages
-    int key0_a = 0, key0_b = 0;
-    auto issue = [&](int c, uint32_t& mask, int& key0) {
+    auto issue = [&](int c, uint32_t& mask) {
         const uint32_t sb = smem_base + (c & 1) * WarpSmem<D>::kStageBytes;
-        if constexpr (Src::kContig) {
-            mask = src.chunk(c, &key0);
-            load_chunk_contig<D>(sb, kbase, vbase, key0, mask);
-        } else {
-            const int key = src.key(c * kChunk + lane);
-            mask = __ballot_sync(0xffffffffu, key >= 0);
-            key0 = 0;
-            load_chunk<D>(sb, kbase, vbase, key);
-        }
+        const int key = src.key(c * kChunk + lane);
+        mask = __ballot_sync(0xffffffffu, key >= 0);
+        load_chunk<D>(sb, kbase, vbase, key);
     };
     static_assert(kStages == 2, "two-stage ring");
-    if (n_chunks > 0) issue(0, mask_a, key0_a);
+    if (n_chunks > 0) issue(0, mask_a);
     cp_async_commit();
     for (int c = 0; c < n_chunks; ++c) {
         if (c + 1 < n_chunks) {
-            if ((c + 1) & 1) issue(c + 1, mask_b, key0_b);
-            else issue(c + 1, mask_a, key0_a);
+            if ((c + 1) & 1) issue(c + 1, mask_b);
+            else issue(c + 1, mask_a);
         }
         cp_async_commit();
         cp_async_wait<1>();
         __syncwarp();
         const uint32_t sb = smem_base + (c & 1) * WarpSmem<D>::kStageBytes;
         const uint32_t mask = (c & 1) ? mask_b : mask_a;
-        const int key0 = (c & 1) ? key0_b : key0_a;
+        float s[4][4];
+        chunk_scores<D>(s, qf, sb, mask);
+        hook(c, s, 0);
+        chunk_update<D>(st, s, sb + WarpSmem<D>::kTileBytes, scale_log2);
+        __syncwarp();  // the stage is refilled by the next iteration
+    }
+    cp_async_wait<0>();
+    finish_rows<D>(st);
+}
+
+// Per-warp TMA pipeline state: two mbarriers (one per stage) and how many
+// times each has been used, so that the phases stay right across calls.
+struct TmaRing {
+    uint32_t bar;      // shared address of 2 consecutive mbarriers
+    uint32_t uses[2];
+};
+
+// Run the pipeline over n_chunks chunks of 32 consecutive keys each;
+// src.chunk(c, &key0) gives chunk c's first key and its valid-row mask.  One
+// lane issues the TMA boxes {64, 32} of K and V (coordinates d, key, unit);
+// rows past the cache end are zero-filled by the TMA.  The optional per-chunk
+// hook sees the masked raw logits and the chunk's first key.  Returns false if
+// a wait timed out (HS_ERR_TIMEOUT is then set).
+template <int D, typename Src, typename Hook>
+__device__ __forceinline__ bool attend_rows_tma(AttnState<D>& st, const uint32_t (&qf)[D / 16][4],
+                                                const CUtensorMap* tk, const CUtensorMap* tv,
+                                                int unit, int n_chunks, const Src& src,
+                                                uint32_t smem_base, TmaRing& ring,
+                                                float scale_log2, Hook hook) {
+    static_assert(Src::kContig, "consecutive keys");
+    constexpr uint32_t kHalf = kChunk * 128;          // one d-half box
+    constexpr uint32_t kTx = 2 * (D / 64) * kHalf;    // K and V, all halves
+    const int lane = threadIdx.x & 31;
+    uint32_t mask_a = 0, mask_b = 0;
+    int key0_a = 0, key0_b = 0;
+    int dummy = 0;
+    volatile int* no_abort = &dummy;
+    auto issue = [&](int c, uint32_t& mask, int& key0) {
+        const uint32_t sb = smem_base + (c & 1) * WarpSmem<D>::kStageBytes;
+        mask = src.chunk(c, &key0);
+        if (lane == 0) {
+            const uint32_t b = ring.bar + 8u * (c & 1);
+            tc::mbar_arrive_expect_tx(b, kTx);
+#pragma unroll
+            for (int h = 0; h < D / 64; ++h) {
+                tc::tma_load_3d(sb + h * kHalf, tk, b, 64 * h, key0, unit);
+                tc::tma_load_3d(sb + WarpSmem<D>::kTileBytes + h * kHalf, tv, b, 64 * h, key0,
+                                unit);
+            }
+        }
+    };
+    int issued = 0, failed = -1;
+    if (n_chunks > 0) { issue(0, mask_a, key0_a); issued = 1; }
+    for (int c = 0; c < n_chunks; ++c) {
+        if (c + 1 < n_chunks) {
+            if ((c + 1) & 1) issue(c + 1, mask_b, key0_b);
+            else issue(c + 1, mask_a, key0_a);
+            issued = c + 2;
+        }
+        const int sidx = c & 1;
+        const bool got = tc::mbar_wait(ring.bar + 8u * sidx, ring.uses[sidx] & 1, no_abort);
+        if (!__all_sync(0xffffffffu, got)) { failed = c; break; }
+        ring.uses[sidx]++;
+        const uint32_t sb = smem_base + sidx * WarpSmem<D>::kStageBytes;
+        const uint32_t mask = sidx ? mask_b : mask_a;
+        const int key0 = sidx ? key0_b : key0_a;
         float s[4][4];
         chunk_scores<D>(s, qf, sb, mask);
         hook(c, s, key0);
         chunk_update<D>(st, s, sb + WarpSmem<D>::kTileBytes, scale_log2);
         __syncwarp();  // the stage is refilled by the next iteration
     }
-    cp_async_wait<0>();
+    if (failed >= 0) {
+        // wait (bounded) for every load issued but not consumed before the
+        // buffers can be reused, keeping the phase counts consistent
+        for (int c = failed; c < issued; ++c) {
+            const int sidx = c & 1;
+            const long long t0 = clock64();
+            while (!tc::mbar_try_wait(ring.bar + 8u * sidx, ring.uses[sidx] & 1))
+                if (clock64() - t0 > tc::kWaitCycles) break;
+            ring.uses[sidx]++;
+        }
+        return false;
+    }
     finish_rows<D>(st);
+    return true;
 }
 
 // Keys first..last (inclusive) as contiguous chunks.

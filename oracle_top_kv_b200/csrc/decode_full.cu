@@ -83,12 +83,13 @@ struct LogitExport {
 
 template <int D>
 __global__ void __launch_bounds__(kDecodeWarps * 32)
-    decode_full_split_kernel(KParams p, const __nv_bfloat16* __restrict__ q,
-                             const __nv_bfloat16* __restrict__ kc,
-                             const __nv_bfloat16* __restrict__ vc,
+    decode_full_split_kernel(const __grid_constant__ CUtensorMap tm_k,
+                             const __grid_constant__ CUtensorMap tm_v, KParams p,
+                             const __nv_bfloat16* __restrict__ q,
                              const int32_t* __restrict__ seq_len, DecodeWs ws) {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    const int warp = threadIdx.x >> 5;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int task = blockIdx.x * kDecodeWarps + warp;
     if (task >= p.batch * p.hkv * ws.n_split) return;
     const int sp = task % ws.n_split;
@@ -101,14 +102,20 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
     const int first = sp * kDecodeKeys;
     if (L >= 1 && L <= p.t_kv && first < L) {
         const int last = min(L - 1, first + kDecodeKeys - 1);
-        const uint32_t sbase = smem_u32(smem_raw) + warp * WarpSmem<D>::kBytes;
+        const uint32_t sbase = base + warp * WarpSmem<D>::kBytes;
+        TmaRing ring{base + kDecodeWarps * WarpSmem<D>::kBytes + 16u * warp, {0u, 0u}};
+        if (lane == 0) {
+            tc::mbar_init(ring.bar, 1);
+            tc::mbar_init(ring.bar + 8, 1);
+            tc::fence_mbar_init();
+        }
+        __syncwarp();
         uint32_t qf[D / 16][4];
         load_q_frags<D>(qf, q + ((size_t)b * p.hq + u * g) * D, D, g);
-        const size_t kvoff = (size_t)unit * p.t_kv * D;
         LogitExport<D> hook{ws.logits + (size_t)unit * p.t_kv * 16, last, g, p.scale_log2};
         const ContiguousKeys src{first, last};
-        attend_rows<D>(st, qf, kc + kvoff, vc + kvoff, src.n_chunks(), src, sbase, p.scale_log2,
-                       hook);
+        attend_rows_tma<D>(st, qf, &tm_k, &tm_v, unit, src.n_chunks(), src, sbase, ring,
+                           p.scale_log2, hook);
     }
     store_partial<D>(st, ws.part + (size_t)task * 16 * (D + 2), g);
 }
@@ -117,7 +124,7 @@ __global__ void __launch_bounds__(kSelectThreads)
     decode_select_kernel(KParams p, const int32_t* __restrict__ seq_len, DecodeWs ws,
                          int32_t* __restrict__ idx, int32_t* __restrict__ cnt,
                          float* __restrict__ sel) {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
     __shared__ int s_count;
     __shared__ unsigned long long s_thresh;
     __shared__ float s_lse2[16];
@@ -192,15 +199,19 @@ static cudaError_t launch_decode_full_t(const KParams& p, const void* q, const v
                                         int32_t* cnt, void* o, float* lse, float* sel, void* ws,
                                         cudaStream_t st) {
     DecodeWs w = decode_ws_layout(p, ws);
-    const size_t smem = (size_t)kDecodeWarps * WarpSmem<D>::kBytes;
+    const size_t smem = (size_t)kDecodeWarps * (WarpSmem<D>::kBytes + 16) + 1024;
+    CUtensorMap mk, mv;
+    const long long units = (long long)p.batch * p.hkv;
+    if (!tc::encode_rows(&mk, kc, D, p.t_kv, units, kChunk) ||
+        !tc::encode_rows(&mv, vc, D, p.t_kv, units, kChunk))
+        return cudaErrorInvalidValue;
     auto kern = decode_full_split_kernel<D>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int n_tasks = p.batch * p.hkv * w.n_split;
     kern<<<(n_tasks + kDecodeWarps - 1) / kDecodeWarps, kDecodeWarps * 32, smem, st>>>(
-        p, (const __nv_bfloat16*)q, (const __nv_bfloat16*)kc, (const __nv_bfloat16*)vc, seq_len,
-        w);
+        mk, mv, p, (const __nv_bfloat16*)q, seq_len, w);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = launch_decode_combine(p, w.part, w.n_split, seq_len, o, lse, w.lse2, st)) !=
         cudaSuccess)

@@ -39,7 +39,7 @@ __global__ void __launch_bounds__(512) full_simt_kernel(KParams p, const T* __re
                                                         int32_t* __restrict__ idx,
                                                         int32_t* __restrict__ cnt,
                                                         float* __restrict__ sel, int do_attn) {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
     const int j = blockIdx.x, u = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = p.group;

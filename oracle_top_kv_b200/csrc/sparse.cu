@@ -208,16 +208,27 @@ __device__ __forceinline__ void store_rows(const AttnState<D>& st, __nv_bfloat16
     }
 }
 
+// Dynamic shared memory: per warp a 2-stage K/V ring, then per warp 2 mbarriers.
+template <int D>
+constexpr size_t sparse_smem_bytes() {
+    return (size_t)kSparseWarps * WarpSmem<D>::kBytes + kSparseWarps * 16 + 1024;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kSparseWarps * 32)
-    sparse_mma_kernel(KParams p, const __nv_bfloat16* __restrict__ q,
-                      const __nv_bfloat16* __restrict__ kf, const __nv_bfloat16* __restrict__ vf,
-                      const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt,
-                      const __nv_bfloat16* __restrict__ kl, const __nv_bfloat16* __restrict__ vl,
+    sparse_mma_kernel(const __grid_constant__ CUtensorMap tm_kf,
+                      const __grid_constant__ CUtensorMap tm_vf,
+                      const __grid_constant__ CUtensorMap tm_kl,
+                      const __grid_constant__ CUtensorMap tm_vl, KParams p,
+                      const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kf,
+                      const __nv_bfloat16* __restrict__ vf, const int32_t* __restrict__ idx,
+                      const int32_t* __restrict__ cnt, int has_local,
                       __nv_bfloat16* __restrict__ og, float* __restrict__ lseg,
                       __nv_bfloat16* __restrict__ ol, float* __restrict__ lsel) {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    const int warp = threadIdx.x >> 5;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long task = (long long)blockIdx.x * kSparseWarps + warp;
     const long long n_tasks = (long long)p.batch * p.hkv * p.t_q;
     if (task >= n_tasks) return;
@@ -226,37 +237,45 @@ __global__ void __launch_bounds__(kSparseWarps * 32)
     const int b = (int)(task / ((long long)p.t_q * p.hkv));
     const int g = p.group;
     const int t = p.q_offset + j;
-    const uint32_t sbase = smem_u32(smem_raw) + warp * WarpSmem<D>::kBytes;
+    const uint32_t sbase = base + warp * WarpSmem<D>::kBytes;
+    TmaRing ring{base + kSparseWarps * WarpSmem<D>::kBytes + 16u * warp, {0u, 0u}};
+    if (lane == 0) {
+        tc::mbar_init(ring.bar, 1);
+        tc::mbar_init(ring.bar + 8, 1);
+        tc::fence_mbar_init();
+    }
+    __syncwarp();
 
     const size_t head_stride = (size_t)p.t_q * D;
     const size_t q0 = (((size_t)b * p.hq + u * g) * p.t_q + j);  // row of head u*g
     uint32_t qf[D / 16][4];
     load_q_frags<D>(qf, q + q0 * D, head_stride, g);
 
-    const size_t row = ((size_t)b * p.hkv + u) * p.t_q + j;
-    const size_t kvoff = ((size_t)b * p.hkv + u) * p.t_kv * D;
+    const int unit = b * p.hkv + u;
+    const size_t row = (size_t)unit * p.t_q + j;
+    const size_t kvoff = (size_t)unit * p.t_kv * D;
     const int c = clamp_count(cnt[row], p.ksel);
     const int n_rows = p.mode == 0 ? c * p.block_size : c;
-    GatherKeys keys{idx + row * p.ksel, n_rows, p.block_size, t, p.mode};
 
     AttnState<D> st;
     st.init();
     if (p.mode == 0 && p.block_size % kChunk == 0) {
         BlockChunks src{idx + row * p.ksel, p.block_size, t};
-        attend_rows<D>(st, qf, kf + kvoff, vf + kvoff, c * (p.block_size / kChunk), src, sbase,
-                       p.scale_log2, NoHook{});
+        attend_rows_tma<D>(st, qf, &tm_kf, &tm_vf, unit, c * (p.block_size / kChunk), src, sbase,
+                           ring, p.scale_log2, NoHook{});
     } else {
+        GatherKeys keys{idx + row * p.ksel, n_rows, p.block_size, t, p.mode};
         attend_rows<D>(st, qf, kf + kvoff, vf + kvoff, (n_rows + kChunk - 1) / kChunk, keys,
                        sbase, p.scale_log2, NoHook{});
     }
     store_rows<D>(st, og + q0 * D, head_stride, lseg + q0, p.t_q, g);
-    if (kl) {
+    if (has_local) {
         const int first = max(0, t - p.window + 1);
         AttnState<D> sl;
         sl.init();
         const ContiguousKeys win{first, t};
-        attend_rows<D>(sl, qf, kl + kvoff, vl + kvoff, win.n_chunks(), win, sbase, p.scale_log2,
-                       NoHook{});
+        attend_rows_tma<D>(sl, qf, &tm_kl, &tm_vl, unit, win.n_chunks(), win, sbase, ring,
+                           p.scale_log2, NoHook{});
         store_rows<D>(sl, ol + q0 * D, head_stride, lsel + q0, p.t_q, g);
     }
 }
@@ -266,7 +285,20 @@ static cudaError_t launch_sparse_mma_t(const KParams& p, const void* q, const vo
                                        const void* vf, const int32_t* idx, const int32_t* cnt,
                                        const void* kl, const void* vl, void* og, float* lseg,
                                        void* ol, float* lsel, cudaStream_t st) {
-    const size_t smem = (size_t)kSparseWarps * WarpSmem<D>::kBytes;
+    const size_t smem = sparse_smem_bytes<D>();
+    CUtensorMap mk, mv, mkl, mvl;
+    const long long units = (long long)p.batch * p.hkv;
+    if (!tc::encode_rows(&mk, kf, D, p.t_kv, units, kChunk) ||
+        !tc::encode_rows(&mv, vf, D, p.t_kv, units, kChunk))
+        return cudaErrorInvalidValue;
+    if (kl) {
+        if (!tc::encode_rows(&mkl, kl, D, p.t_kv, units, kChunk) ||
+            !tc::encode_rows(&mvl, vl, D, p.t_kv, units, kChunk))
+            return cudaErrorInvalidValue;
+    } else {
+        mkl = mk;
+        mvl = mv;
+    }
     auto kern = sparse_mma_kernel<D>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -274,8 +306,8 @@ static cudaError_t launch_sparse_mma_t(const KParams& p, const void* q, const vo
     const long long n_tasks = (long long)p.batch * p.hkv * p.t_q;
     const unsigned grid = (unsigned)((n_tasks + kSparseWarps - 1) / kSparseWarps);
     kern<<<grid, kSparseWarps * 32, smem, st>>>(
-        p, (const __nv_bfloat16*)q, (const __nv_bfloat16*)kf, (const __nv_bfloat16*)vf, idx, cnt,
-        (const __nv_bfloat16*)kl, (const __nv_bfloat16*)vl, (__nv_bfloat16*)og, lseg,
+        mk, mv, mkl, mvl, p, (const __nv_bfloat16*)q, (const __nv_bfloat16*)kf,
+        (const __nv_bfloat16*)vf, idx, cnt, kl ? 1 : 0, (__nv_bfloat16*)og, lseg,
         (__nv_bfloat16*)ol, lsel);
     return cudaGetLastError();
 }
@@ -302,7 +334,8 @@ __global__ void __launch_bounds__(kSparseWarps * 32)
                                const int32_t* __restrict__ seq_len,
                                const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt,
                                float* __restrict__ part, int n_split) {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
     const int warp = threadIdx.x >> 5;
     const int task = blockIdx.x * kSparseWarps + warp;
     if (task >= p.batch * p.hkv * n_split) return;
@@ -319,7 +352,7 @@ __global__ void __launch_bounds__(kSparseWarps * 32)
         const int c = clamp_count(cnt[unit], p.ksel);
         const int r0 = sp * kDecodeSparseRows;
         const int n_rows = max(0, min(kDecodeSparseRows, c - r0));
-        const uint32_t sbase = smem_u32(smem_raw) + warp * WarpSmem<D>::kBytes;
+        const uint32_t sbase = base + warp * WarpSmem<D>::kBytes;
         uint32_t qf[D / 16][4];
         load_q_frags<D>(qf, q + ((size_t)b * p.hq + u * g) * D, D, g);
         GatherKeys keys{idx + (size_t)unit * p.ksel + r0, n_rows, 1, t, 1};
@@ -383,7 +416,7 @@ static cudaError_t launch_decode_sparse_t(const KParams& p, const void* q, const
                                           const int32_t* idx, const int32_t* cnt, void* o,
                                           float* lse, void* ws, cudaStream_t st) {
     const int n_split = (p.ksel + kDecodeSparseRows - 1) / kDecodeSparseRows;
-    const size_t smem = (size_t)kSparseWarps * WarpSmem<D>::kBytes;
+    const size_t smem = (size_t)kSparseWarps * WarpSmem<D>::kBytes + 1024;
     auto kern = decode_sparse_split_kernel<D>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -296,12 +296,6 @@ bool token_select_tc_supported(const KParams& p, int dtype) {
            p.k - p.window <= tsel::kMaxRanked;
 }
 
-// Host helpers of full_tc.cu (same translation unit).
-namespace tc {
-static bool encode(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims,
-                   const cuuint64_t* strides, const cuuint32_t* box);
-}
-
 cudaError_t launch_token_select_tc(const KParams& p, const void* q, const void* k,
                                    const float* lse, int32_t* idx, int32_t* cnt, float* sel,
                                    cudaStream_t st) {

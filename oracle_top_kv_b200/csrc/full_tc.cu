@@ -389,11 +389,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (row_ok) a.lse[orow] = lse2 * kLn2;
         }
         if (a.capture) {
-            // ---- group merge: rows hh*P + pr of the g heads share position pr
+            // ---- group merge.  Rows hh*P + pr of the g heads share position
+            // pr; each row's list is sorted by (score desc, id asc).  One
+            // thread per position k-way merges the g lists in that order and
+            // skips ids already taken: an id's first occurrence carries its
+            // largest listed score, so this is the union rule's top-k.
             unsigned char* reg = gbase + kPOff + q * 32768;    // this tile's P buffers
             float* cs = reinterpret_cast<float*>(reg);         // [128][kList]
             int* ci = reinterpret_cast<int*>(reg + 128 * kList * 4);
-            unsigned char* flags = reg + 2 * 128 * kList * 4;  // 4 warps x 256
             // every PV has completed (BOF), so the P buffers are free to reuse
 #pragma unroll
             for (int i = 0; i < kList; ++i) {
@@ -401,65 +404,63 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ci[row * kList + i] = ok ? li[i] : -1;
             }
             asm volatile("bar.sync %0, 128;" ::"r"(1 + q) : "memory");
-            const int n = g * kList;
-            unsigned char* fl = flags + quad * 256;
-            for (int pp = quad; pp < P && ok; pp += 4) {
-                const int rj = qrow0 + pp;
-                if (rj >= p.t_q) break;
-                // candidate i -> entry (head i / kList, slot i % kList) of position pp
-                auto eidx = [&](int i) { return ((i / kList) * P + pp) * kList + (i % kList); };
-                // 1) primary: best occurrence of its id (ties: first occurrence)
-                for (int i = lane; i < n; i += 32) {
-                    const int e = eidx(i);
-                    const int id = ci[e];
-                    bool prim = id >= 0;
-                    for (int i2 = 0; i2 < n && prim; ++i2) {
-                        const int e2 = eidx(i2);
-                        if (ci[e2] == id && (cs[e2] > cs[e] || (cs[e2] == cs[e] && i2 < i))) prim = false;
+            const int pp = row;  // position handled by this thread
+            if (ok && pp < P && qrow0 + pp < p.t_q) {
+                int ptr[16];
+#pragma unroll
+                for (int h2 = 0; h2 < 16; ++h2) ptr[h2] = 0;
+                int sid[kList];
+                float ssc[kList];
+                int nsel = 0;
+                for (int guard = 0; guard < 16 * kList && nsel < p.ksel; ++guard) {
+                    float best = -INFINITY;
+                    int best_id = 0x7fffffff, bh = -1;
+#pragma unroll
+                    for (int h2 = 0; h2 < 16; ++h2) {
+                        if (h2 < g && ptr[h2] < kList) {
+                            const int e = (h2 * P + pp) * kList + ptr[h2];
+                            const float v = cs[e];
+                            const int id = ci[e];
+                            if (id >= 0 && (v > best || (v == best && id < best_id))) {
+                                best = v;
+                                best_id = id;
+                                bh = h2;
+                            }
+                        }
                     }
-                    fl[i] = prim ? 1 : 0;
+                    if (bh < 0) break;  // every list exhausted
+#pragma unroll
+                    for (int h2 = 0; h2 < 16; ++h2)
+                        if (h2 == bh) ++ptr[h2];
+                    bool dup = false;
+#pragma unroll
+                    for (int x = 0; x < kList; ++x)
+                        if (x < nsel && sid[x] == best_id) dup = true;
+                    if (dup) continue;
+#pragma unroll
+                    for (int x = 0; x < kList; ++x)
+                        if (x == nsel) { sid[x] = best_id; ssc[x] = best; }
+                    ++nsel;
                 }
-                __syncwarp();
-                // 2) rank among primaries: (score desc, id asc)
-                for (int i = lane; i < n; i += 32) {
-                    if (!fl[i]) continue;
-                    const int e = eidx(i);
-                    int rank = 0;
-                    for (int i2 = 0; i2 < n; ++i2) {
-                        if (!fl[i2]) continue;
-                        const int e2 = eidx(i2);
-                        if (cs[e2] > cs[e] || (cs[e2] == cs[e] && ci[e2] < ci[e])) ++rank;
-                    }
-                    if (rank < p.ksel) fl[i] = 2;
-                }
-                __syncwarp();
-                // 3) output in ascending id order
-                const size_t orow_i = ((size_t)b * p.hkv + u) * p.t_q + rj;
+                // write in ascending id order
+                const size_t orow_i = ((size_t)b * p.hkv + u) * p.t_q + qrow0 + pp;
                 int32_t* irow = a.idx + orow_i * p.ksel;
                 float* srow = a.sel ? a.sel + orow_i * p.ksel : nullptr;
-                int nsel = 0;
-                for (int i0 = 0; i0 < n; i0 += 32) {
-                    const int i = i0 + lane;
-                    nsel += __popc(__ballot_sync(0xffffffffu, i < n && fl[i] == 2));
-                }
-                nsel = min(nsel, p.ksel);
-                for (int i = lane; i < n; i += 32) {
-                    if (fl[i] != 2) continue;
-                    const int e = eidx(i);
+#pragma unroll
+                for (int x = 0; x < kList; ++x) {
+                    if (x >= nsel) continue;
                     int op = 0;
-                    for (int i2 = 0; i2 < n; ++i2)
-                        if (fl[i2] == 2 && ci[eidx(i2)] < ci[e]) ++op;
-                    if (op < p.ksel) {
-                        irow[op] = ci[e];
-                        if (srow) srow[op] = exp2f(cs[e]);
-                    }
+#pragma unroll
+                    for (int y = 0; y < kList; ++y)
+                        if (y < nsel && sid[y] < sid[x]) ++op;
+                    irow[op] = sid[x];
+                    if (srow) srow[op] = exp2f(ssc[x]);
                 }
-                for (int x = nsel + lane; x < p.ksel; x += 32) {
+                for (int x = nsel; x < p.ksel; ++x) {
                     irow[x] = -1;
                     if (srow) srow[x] = 0.f;
                 }
-                if (lane == 0) a.cnt[orow_i] = nsel;
-                __syncwarp();
+                a.cnt[orow_i] = nsel;
             }
         }
     }

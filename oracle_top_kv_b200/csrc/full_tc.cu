@@ -42,6 +42,9 @@ constexpr int kD = 128;
 constexpr int kKV = 3;        // K/V ring stages
 constexpr int kList = 16;     // per-row candidate list (>= k/B)
 constexpr int kThreads = 64 + 128 * kNQ;
+// The TMA producer and the MMA issuer are single threads on the critical
+// path: they poll their barriers instead of sleeping.
+constexpr bool kRoleSleep = false;
 
 constexpr uint32_t kQOff = 0;                         // kNQ x 32 KB (two d halves each)
 constexpr uint32_t kKOff = kNQ * 32768;               // kKV x 16 KB
@@ -182,7 +185,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             int issued = 0;
             for (int j = 0; j < nt; ++j) {
                 const int st = j % kKV;
-                if (j >= kKV && !mbar_wait(bar(BKVE + st), ((j / kKV) - 1) & 1, abort_flag)) break;
+                if (j >= kKV &&
+                    !mbar_wait(bar(BKVE + st), ((j / kKV) - 1) & 1, abort_flag, kRoleSleep))
+                    break;
                 const uint32_t f = bar(BKVF + st);
                 mbar_arrive_expect_tx(f, 4 * 8192);
                 const uint32_t kd = base + kKOff + st * 16384, vd = base + kVOff + st * 16384;
@@ -203,17 +208,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             const uint32_t id_s = idesc_bf16(kBM, kBN, false, false);
             const uint32_t id_o = idesc_bf16(kBM, kD, false, true);
-            bool ok = mbar_wait(bar(BQ), 0, abort_flag);
+            bool ok = mbar_wait(bar(BQ), 0, abort_flag, kRoleSleep);
             tc_fence_after();
             for (int j = 0; ok && j <= nt; ++j) {
                 if (j < nt) {
                     const int st = j % kKV, s = j & 1;
-                    if (!mbar_wait(bar(BKVF + st), (j / kKV) & 1, abort_flag)) break;
+                    if (!mbar_wait(bar(BKVF + st), (j / kKV) & 1, abort_flag, kRoleSleep)) break;
                     const uint32_t kb = base + kKOff + st * 16384;
 #pragma unroll
                     for (int q = 0; q < kNQ; ++q) {
                         if (j >= ntq[q]) continue;
-                        if (j >= 2 && !mbar_wait(bar(BSE + 2 * q + s), ((j >> 1) - 1) & 1, abort_flag)) {
+                        if (j >= 2 && !mbar_wait(bar(BSE + 2 * q + s), ((j >> 1) - 1) & 1,
+                                                 abort_flag, kRoleSleep)) {
                             ok = false;
                             break;
                         }
@@ -235,7 +241,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int q = 0; q < kNQ; ++q) {
                         if (jj >= ntq[q]) continue;
-                        if (!mbar_wait(bar(BPF + 2 * q + sp), (jj >> 1) & 1, abort_flag)) {
+                        if (!mbar_wait(bar(BPF + 2 * q + sp), (jj >> 1) & 1, abort_flag,
+                                       kRoleSleep)) {
                             ok = false;
                             break;
                         }
@@ -316,18 +323,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m_ref = mt;
                 l *= corr;
             }
-            const float nm = -m_ref;
+            // p = 2^(x * scale_log2 - m): packed FFMA for the arguments and
+            // packed adds for the row sum
+            const float2 s2 = make_float2(sl2, sl2), n2 = make_float2(-m_ref, -m_ref);
             float e[64];
+            float2 acc[8];
 #pragma unroll
-            for (int c = 0; c < 64; ++c) e[c] = ex2(fmaf(x[c], sl2, nm));
-            float sm[16];
+            for (int c2 = 0; c2 < 32; ++c2) {
+                const float2 y = ffma2(make_float2(x[2 * c2], x[2 * c2 + 1]), s2, n2);
+                e[2 * c2] = ex2(y.x);
+                e[2 * c2 + 1] = ex2(y.y);
+                const float2 ev = make_float2(e[2 * c2], e[2 * c2 + 1]);
+                acc[c2 & 7] = c2 < 8 ? ev : fadd2(acc[c2 & 7], ev);
+            }
 #pragma unroll
-            for (int c = 0; c < 16; ++c) sm[c] = (e[c] + e[c + 16]) + (e[c + 32] + e[c + 48]);
+            for (int w = 4; w >= 1; w >>= 1)
 #pragma unroll
-            for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-                for (int c = 0; c < w; ++c) sm[c] += sm[c + w];
-            l += sm[0];
+                for (int c = 0; c < w; ++c) acc[c] = fadd2(acc[c], acc[c + w]);
+            l += acc[0].x + acc[0].y;
             uint32_t pk[32];
 #pragma unroll
             for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(e[2 * c], e[2 * c + 1]);

@@ -25,7 +25,7 @@ def lib():
 def declared_functions():
     text = open(os.path.join(ROOT, "include", "hs.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(hs_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(hs_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_every_declared_symbol_is_exported(lib):

@@ -12,10 +12,12 @@
 //     final lse, known only after all splits;
 //  2. the exact log-sum-exp merge of the splits (shared with the sparse
 //     decode) -> o, lse, and lse2 for the selector;
-//  3. decode_select_kernel: one CTA per (sequence, group) ranks keys
-//     0..t-w by max_h (a2_{h,i} - lse2_h) (= log2 of max_h p_{h,t,i}) with the
-//     exact streaming top-k and appends the forced window t-w+1..t
-//     ("HySparse2 ..." 4.2).
+//  3. the selector ranks keys 0..t-w by max_h (a2_{h,i} - lse2_h) (= log2 of
+//     max_h p_{h,t,i}) with the exact streaming top-k and appends the forced
+//     window t-w+1..t ("HySparse2 ..." 4.2): 8 CTAs per (sequence, group)
+//     each keep the top-(k-w) of a slice of the keys, and a merge kernel
+//     takes the top-(k-w) of their union (decode_select_kernel, one CTA per
+//     unit, serves budgets above 1024).
 #include "attend_mma.cuh"
 #include "block_topk.cuh"
 #include "hs_common.cuh"
@@ -31,10 +33,15 @@ constexpr int kDecodeKeys = 2048;  // cache keys per split
 constexpr int kDecodeWarps = 4;
 constexpr int kSelectThreads = 512;
 
+constexpr int kSelSplits = 8;          // CTAs per (sequence, group) in the selector
+constexpr int kSelMaxRanked = 1024;    // k - w handled by the split selector
+
 struct DecodeWs {
-    float* logits;  // [batch*hkv][t_kv][16]
-    float* part;    // [batch*hkv][n_split][16][D+2]
-    float* lse2;    // [batch*hq]
+    float* logits;    // [batch*hkv][t_kv][16]
+    float* part;      // [batch*hkv][n_split][16][D+2]
+    float* lse2;      // [batch*hq]
+    uint64_t* cand;   // [batch*hkv][kSelSplits][kSelMaxRanked] selection keys
+    int* cand_n;      // [batch*hkv][kSelSplits]
     int n_split;
 };
 
@@ -46,10 +53,14 @@ static DecodeWs decode_ws_layout(const KParams& p, void* base) {
     const size_t units = (size_t)p.batch * p.hkv;
     const size_t logits_b = align256(units * p.t_kv * 16 * sizeof(float));
     const size_t part_b = align256(units * w.n_split * 16 * (p.head_dim + 2) * sizeof(float));
+    const size_t lse_b = align256((size_t)p.batch * p.hq * sizeof(float));
+    const size_t cand_b = align256(units * kSelSplits * kSelMaxRanked * sizeof(uint64_t));
     char* c = static_cast<char*>(base);
     w.logits = reinterpret_cast<float*>(c);
     w.part = reinterpret_cast<float*>(c + logits_b);
     w.lse2 = reinterpret_cast<float*>(c + logits_b + part_b);
+    w.cand = reinterpret_cast<uint64_t*>(c + logits_b + part_b + lse_b);
+    w.cand_n = reinterpret_cast<int*>(c + logits_b + part_b + lse_b + cand_b);
     return w;
 }
 
@@ -58,7 +69,9 @@ size_t decode_full_workspace(const KParams& p) {
     const size_t units = (size_t)p.batch * p.hkv;
     return align256(units * p.t_kv * 16 * sizeof(float)) +
            align256(units * n_split * 16 * (p.head_dim + 2) * sizeof(float)) +
-           align256((size_t)p.batch * p.hq * sizeof(float));
+           align256((size_t)p.batch * p.hq * sizeof(float)) +
+           align256(units * kSelSplits * kSelMaxRanked * sizeof(uint64_t)) +
+           align256(units * kSelSplits * sizeof(int));
 }
 
 // Writes every head's scaled logit a2 = scale_log2 * q.k of the chunk's keys.
@@ -193,6 +206,147 @@ __global__ void __launch_bounds__(kSelectThreads)
     if (threadIdx.x == 0) cnt[unit] = n_out;
 }
 
+// Group log-score of key i: max over the group's heads of a2 - lse2 (log2 of
+// max_h p_{h,t,i}).
+__device__ __forceinline__ float group_score(const float* lg_row, const float* lse2, int g) {
+    const float4* r4 = reinterpret_cast<const float4*>(lg_row);
+    float s = -INFINITY;
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+        if (q4 * 4 >= g) break;
+        const float4 a = r4[q4];
+        const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            if (q4 * 4 + e < g) s = fmaxf(s, av[e] - lse2[q4 * 4 + e]);
+    }
+    return s;
+}
+
+// Stage 1 of the split selector: CTA (unit, split) keeps the exact top-(k-w)
+// of its slice of the ranked keys 0..t-w and writes them out unsorted.  The
+// group's top-(k-w) is contained in the union of the slices' top-(k-w).
+__global__ void __launch_bounds__(kSelectThreads)
+    decode_select_split_kernel(KParams p, const int32_t* __restrict__ seq_len, DecodeWs ws) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    __shared__ int s_count;
+    __shared__ unsigned long long s_thresh;
+    __shared__ float s_lse2[16];
+    const int unit = blockIdx.x / kSelSplits, sp = blockIdx.x % kSelSplits;
+    const int u = unit % p.hkv, b = unit / p.hkv;
+    const int g = p.group;
+    const int L = seq_len[b];
+    const int Kc = p.k - p.window;
+    int* out_n = ws.cand_n + (size_t)unit * kSelSplits + sp;
+    if (L < 1 || L > p.t_kv || L <= p.k || Kc <= 0) {  // nothing ranked here
+        if (threadIdx.x == 0) *out_n = 0;
+        return;
+    }
+    const int lo = L - p.window;  // ranked keys 0..lo-1
+    const int per = (lo + kSelSplits - 1) / kSelSplits;
+    const int i0 = sp * per, i1 = min(lo, i0 + per);
+    BlockTopK topk;
+    topk.setup(smem_raw, Kc, blockDim.x, &s_count, &s_thresh);
+    if (threadIdx.x < 16) s_lse2[threadIdx.x] = threadIdx.x < g ? ws.lse2[b * p.hq + u * g + threadIdx.x] : 0.f;
+    __syncthreads();
+    const float* lg = ws.logits + (size_t)unit * p.t_kv * 16;
+    for (int c0 = i0; c0 < i1; c0 += blockDim.x) {
+        const int i = c0 + threadIdx.x;
+        if (i < i1) topk.offer(group_score(lg + (size_t)i * 16, s_lse2, g), (uint32_t)i);
+        topk.end_round();
+    }
+    __syncthreads();
+    if (threadIdx.x >= 32) return;
+    int n = *topk.count;
+    if (n > Kc) { warp_cut_to_k(topk.buf, n, Kc, topk.hist); n = Kc; }
+    __syncwarp();
+    uint64_t* dst = ws.cand + ((size_t)unit * kSelSplits + sp) * kSelMaxRanked;
+    for (int x = threadIdx.x; x < n; x += 32) dst[x] = topk.buf[x];
+    if (threadIdx.x == 0) *out_n = n;
+}
+
+// Stage 2: per unit, the final top-(k-w) of the slices' candidates, sorted by
+// id, then the forced window; or every key when the budget covers them all.
+__global__ void __launch_bounds__(kSelectThreads)
+    decode_select_merge_kernel(KParams p, const int32_t* __restrict__ seq_len, DecodeWs ws,
+                               int32_t* __restrict__ idx, int32_t* __restrict__ cnt,
+                               float* __restrict__ sel) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    __shared__ float s_lse2[16];
+    __shared__ int s_base[kSelSplits + 1];
+    const int unit = blockIdx.x;
+    const int u = unit % p.hkv, b = unit / p.hkv;
+    const int g = p.group;
+    const int L = seq_len[b];
+    int32_t* irow = idx + (size_t)unit * p.ksel;
+    float* srow = sel ? sel + (size_t)unit * p.ksel : nullptr;
+    if (L < 1 || L > p.t_kv) {
+        for (int x = threadIdx.x; x < p.ksel; x += blockDim.x) {
+            irow[x] = -1;
+            if (srow) srow[x] = 0.f;
+        }
+        if (threadIdx.x == 0) { cnt[unit] = 0; set_status(HS_ERR_BOUNDS); }
+        return;
+    }
+    const int t = L - 1;
+    const int Kc = p.k - p.window;
+    if (threadIdx.x < 16) s_lse2[threadIdx.x] = threadIdx.x < g ? ws.lse2[b * p.hq + u * g + threadIdx.x] : 0.f;
+    if (threadIdx.x == 0) {
+        int acc = 0;
+        for (int sp = 0; sp < kSelSplits; ++sp) {
+            s_base[sp] = acc;
+            acc += ws.cand_n[(size_t)unit * kSelSplits + sp];
+        }
+        s_base[kSelSplits] = acc;
+    }
+    __syncthreads();
+    const float* lg = ws.logits + (size_t)unit * p.t_kv * 16;
+    if (t + 1 <= p.k) {  // the budget covers every key
+        for (int x = threadIdx.x; x < p.ksel; x += blockDim.x) {
+            irow[x] = x <= t ? x : -1;
+            if (srow) srow[x] = x <= t ? exp2f(group_score(lg + (size_t)x * 16, s_lse2, g)) : 0.f;
+        }
+        if (threadIdx.x == 0) cnt[unit] = t + 1;
+        return;
+    }
+    const int lo = t - p.window + 1;
+    // window scores (only wanted with sel)
+    if (srow)
+        for (int x = threadIdx.x; x <= t - lo; x += blockDim.x)
+            srow[Kc + x] = exp2f(group_score(lg + (size_t)(lo + x) * 16, s_lse2, g));
+    uint64_t* buf = reinterpret_cast<uint64_t*>(smem_raw);          // [kSplits * Kc]
+    uint64_t* sortb = buf + kSelSplits * kSelMaxRanked;              // [next_pow2(Kc)]
+    uint32_t* hist = reinterpret_cast<uint32_t*>(sortb + kSelMaxRanked);
+    const int total = s_base[kSelSplits];
+    for (int sp = 0; sp < kSelSplits; ++sp) {
+        const uint64_t* src = ws.cand + ((size_t)unit * kSelSplits + sp) * kSelMaxRanked;
+        const int n = s_base[sp + 1] - s_base[sp];
+        for (int x = threadIdx.x; x < n; x += blockDim.x) buf[s_base[sp] + x] = src[x];
+    }
+    __syncthreads();
+    if (threadIdx.x >= 32) return;
+    int n = total;
+    if (Kc > 0 && n > Kc) { warp_cut_to_k(buf, n, Kc, hist); n = Kc; }
+    if (Kc <= 0) n = 0;
+    __syncwarp();
+    const int sort_n = next_pow2(Kc > 0 ? Kc : 1);
+    for (int x = threadIdx.x; x < sort_n; x += 32)
+        sortb[x] = x < n ? (((uint64_t)sel_key_id(buf[x]) << 32) | (buf[x] >> 32)) : ~0ull;
+    __syncwarp();
+    warp_bitonic_sort(sortb, sort_n);
+    for (int x = threadIdx.x; x < n; x += 32) {
+        irow[x] = (int32_t)(sortb[x] >> 32);
+        if (srow) srow[x] = exp2f(order_float((uint32_t)(sortb[x] & 0xffffffffu)));
+    }
+    for (int x = threadIdx.x; x <= t - lo; x += 32) irow[n + x] = lo + x;
+    const int n_out = n + (t - lo + 1);
+    for (int x = n_out + threadIdx.x; x < p.ksel; x += 32) {
+        irow[x] = -1;
+        if (srow) srow[x] = 0.f;
+    }
+    if (threadIdx.x == 0) cnt[unit] = n_out;
+}
+
 template <int D>
 static cudaError_t launch_decode_full_t(const KParams& p, const void* q, const void* kc,
                                         const void* vc, const int32_t* seq_len, int32_t* idx,
@@ -216,7 +370,25 @@ static cudaError_t launch_decode_full_t(const KParams& p, const void* q, const v
     if ((e = launch_decode_combine(p, w.part, w.n_split, seq_len, o, lse, w.lse2, st)) !=
         cudaSuccess)
         return e;
-    const size_t sel_smem = BlockTopK::smem_bytes(p.k - p.window, kSelectThreads);
+    const int Kc = p.k - p.window;
+    if (Kc <= kSelMaxRanked) {
+        const size_t s1 = BlockTopK::smem_bytes(Kc, kSelectThreads);
+        e = cudaFuncSetAttribute(decode_select_split_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1);
+        if (e != cudaSuccess) return e;
+        decode_select_split_kernel<<<p.batch * p.hkv * kSelSplits, kSelectThreads, s1, st>>>(
+            p, seq_len, w);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        const size_t s2 = sizeof(uint64_t) * (kSelSplits * kSelMaxRanked + kSelMaxRanked) +
+                          sizeof(uint32_t) * 256;
+        e = cudaFuncSetAttribute(decode_select_merge_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2);
+        if (e != cudaSuccess) return e;
+        decode_select_merge_kernel<<<p.batch * p.hkv, kSelectThreads, s2, st>>>(p, seq_len, w, idx,
+                                                                               cnt, sel);
+        return cudaGetLastError();
+    }
+    const size_t sel_smem = BlockTopK::smem_bytes(Kc, kSelectThreads);
     e = cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sel_smem);
     if (e != cudaSuccess) return e;

@@ -116,54 +116,97 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk, int row_bytes) {
 // best key: a later candidate can only enter the final K if its key is above
 // it, so nothing that could still be selected is ever dropped.
 
-// K-th largest of n unique keys (1 <= K <= n), computed by one warp with an
-// 8-bit-digit radix select.  hist: 256 words of shared scratch for this warp.
+__device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int o) {
+    const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, o);
+    const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), o);
+    return ((uint64_t)hi << 32) | lo;
+}
+
+// K-th largest of n unique keys (1 <= K <= n), computed by one warp with a
+// range bucket select: each pass spreads the keys of the live range [lo, hi]
+// over 256 equal-width buckets (bucket = (key - lo) >> shift, with shift set
+// by the width of the range, so nearby scores still land in different
+// buckets), keeps the bucket holding the K-th key, and stops as soon as that
+// bucket holds a single key.  hist: 256 words of shared scratch for this warp.
 __device__ __forceinline__ uint64_t warp_kth_largest(const uint64_t* buf, int n, int K,
                                                      uint32_t* hist) {
     const int lane = threadIdx.x & 31;
-    uint64_t prefix = 0, mask = 0;
-    int need = K;
-    for (int shift = 56; shift >= 0; shift -= 8) {
+    uint64_t lo = ~0ull, hi = 0ull;
+    for (int i = lane; i < n; i += 32) {
+        const uint64_t key = buf[i];
+        lo = key < lo ? key : lo;
+        hi = key > hi ? key : hi;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t a = shfl_xor_u64(lo, o), b = shfl_xor_u64(hi, o);
+        lo = a < lo ? a : lo;
+        hi = b > hi ? b : hi;
+    }
+    int need = K;  // rank of the wanted key, counted from the top of [lo, hi]
+    for (int pass = 0; pass < 16; ++pass) {
+        if (lo == hi) return lo;
+        const uint64_t range = hi - lo;
+        const int top = 63 - __clzll((long long)range);
+        const int shift = top > 7 ? top - 7 : 0;  // (range >> shift) <= 255
 #pragma unroll
         for (int x = 0; x < 8; ++x) hist[lane * 8 + x] = 0;
         __syncwarp();
         for (int i = lane; i < n; i += 32) {
             const uint64_t key = buf[i];
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1u);
+            if (key >= lo && key <= hi) atomicAdd(&hist[(uint32_t)((key - lo) >> shift)], 1u);
         }
         __syncwarp();
-        // lane L owns bins 255-8L .. 248-8L (descending).  Count above each bin.
+        // lane L owns buckets 255-8L .. 248-8L (descending).  Count above each.
         uint32_t own[8];
         uint32_t s = 0;
 #pragma unroll
         for (int x = 0; x < 8; ++x) { own[x] = hist[255 - (lane * 8 + x)]; s += own[x]; }
-        uint32_t incl = s;  // inclusive prefix over lanes (lane 0 = highest bins)
+        uint32_t incl = s;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += y;
         }
-        uint32_t above = incl - s;  // keys in bins higher than this lane's bins
-        int digit = -1;
-        uint32_t above_digit = 0;
+        uint32_t above = incl - s;
+        int bucket = -1;
+        uint32_t above_b = 0, in_b = 0;
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
-            if (digit < 0 && above < (uint32_t)need && above + own[x] >= (uint32_t)need) {
-                digit = 255 - (lane * 8 + x);
-                above_digit = above;
+            if (bucket < 0 && above < (uint32_t)need && above + own[x] >= (uint32_t)need) {
+                bucket = 255 - (lane * 8 + x);
+                above_b = above;
+                in_b = own[x];
             }
             above += own[x];
         }
-        const uint32_t found = __ballot_sync(0xffffffffu, digit >= 0);
+        const uint32_t found = __ballot_sync(0xffffffffu, bucket >= 0);
         const int src = __ffs(found) - 1;
-        digit = __shfl_sync(0xffffffffu, digit, src);
-        above_digit = __shfl_sync(0xffffffffu, above_digit, src);
-        prefix |= (uint64_t)digit << shift;
-        mask |= (uint64_t)255 << shift;
-        need -= (int)above_digit;
+        bucket = __shfl_sync(0xffffffffu, bucket, src);
+        above_b = __shfl_sync(0xffffffffu, above_b, src);
+        in_b = __shfl_sync(0xffffffffu, in_b, src);
+        need -= (int)above_b;
+        const uint64_t nlo = lo + ((uint64_t)bucket << shift);
+        const uint64_t nhi = nlo + (((uint64_t)1 << shift) - 1);
+        lo = nlo;
+        hi = nhi < hi ? nhi : hi;
         __syncwarp();
+        if (in_b == 1) {
+            // the K-th key is the only one left in [lo, hi]: fetch it
+            uint64_t hit = 0;
+            for (int i = lane; i < n; i += 32) {
+                const uint64_t key = buf[i];
+                if (key >= lo && key <= hi) hit = key;
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const uint64_t y = shfl_xor_u64(hit, o);
+                hit = y > hit ? y : hit;
+            }
+            return hit;
+        }
     }
-    return prefix;
+    return lo;  // not reached for unique keys: each pass shrinks the range 256-fold
 }
 
 // Keep only keys >= kth (in place, order not preserved); returns the new count.

@@ -195,6 +195,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(BSE + s));
             const int key = j * kKeys + quad * 32 + lane;
+            uint64_t k64[4];
+            uint32_t bal[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const uint32_t* rr = i < 2 ? r0 : r1;
@@ -210,22 +212,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float* srow = a.sel ? a.sel + orow * p.ksel : nullptr;
                 // Every lane reaches the ballot below: no per-lane early exit.
                 const int lo = t - p.window + 1;
-                const uint64_t k64 = sel_key(sc, (uint32_t)key);
+                k64[i] = sel_key(sc, (uint32_t)key);
                 bool cand = false;
                 if (all_sel[i]) {
                     if (visible && srow) srow[key] = exp2f(sc);
                 } else if (visible && key >= lo) {
                     if (srow) srow[Kc + (key - lo)] = exp2f(sc);
                 } else {
-                    cand = visible && Kc > 0 && key < lo && k64 > s_th[pos];
+                    cand = visible && Kc > 0 && key < lo && k64[i] > s_th[pos];
                 }
-                const uint32_t bal = __ballot_sync(0xffffffffu, cand);
-                if (bal) {
-                    int basei = 0;
-                    if (lane == 0) basei = atomicAdd(&s_cnt[pos], __popc(bal));
-                    basei = __shfl_sync(0xffffffffu, basei, 0);
-                    if (cand) bufs[(size_t)pos * kCap + basei + __popc(bal & ((1u << lane) - 1))] = k64;
-                }
+                bal[i] = __ballot_sync(0xffffffffu, cand);
+            }
+            // one lane reserves the slots of all four positions (independent atomics)
+            int basei[4] = {0, 0, 0, 0};
+            if (lane == 0) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    if (bal[i]) basei[i] = atomicAdd(&s_cnt[set * 4 + i], __popc(bal[i]));
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if (!bal[i]) continue;  // warp-uniform
+                const int bi = __shfl_sync(0xffffffffu, basei[i], 0);
+                if ((bal[i] >> lane) & 1u)
+                    bufs[(size_t)(set * 4 + i) * kCap + bi + __popc(bal[i] & ((1u << lane) - 1))] =
+                        k64[i];
             }
             }  // got
             // cut a buffer that could overflow on the next tile

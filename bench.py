@@ -15,6 +15,10 @@ full+index TFLOP/s and sparse-reuse K/V GB/s, each with its fraction of peak.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
+Each step replays two CUDA graphs captured from the C-ABI calls (the full
+layer's launches, then the sparse layers'), so the GPU runs the kernels back
+to back; --no-graph times the per-call launches instead.
+
 --impl reference times the fp64 CPU oracle on the host cores on a bounded
 sample of the same workload (the only place besides the cpu_baseline field
 where this script runs the oracle).
@@ -272,8 +276,13 @@ def run_ours(args, rank, world, device):
     torch.cuda.synchronize(device)
     assert hs.hs_device_status(sh) == 0
     flops, full_bytes, sbytes = work(w, blk)
+    graphs = None if args.no_graph else capture_step(blk, w, device)
+    if graphs:  # one more untimed step, through the graphs
+        graphs[0].replay()
+        graphs[1].replay()
+        torch.cuda.synchronize(device)
 
-    n_ev = 1 + w.n_sparse
+    n_ev = 1 + (1 if graphs else w.n_sparse)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev + 1)]
            for _ in range(args.steps)]
     clocks = ClockSampler(device)
@@ -287,6 +296,12 @@ def run_ours(args, rank, world, device):
     t0.record(stream)
     for s in range(args.steps):
         evs[s][0].record(stream)
+        if graphs:
+            graphs[0].replay()
+            evs[s][1].record(stream)
+            graphs[1].replay()
+            evs[s][2].record(stream)
+            continue
         blk.full(sh)
         evs[s][1].record(stream)
         for layer in range(w.n_sparse):
@@ -295,13 +310,19 @@ def run_ours(args, rank, world, device):
     t1.record(stream)
     torch.cuda.synchronize(device)
     launches = hs.hs_launch_count() - launches0
+    if graphs:  # replays do not pass through the library: count the captured launches
+        launches = args.steps * (graphs[2] + graphs[3])
     hdist.barrier(device)
     clocks.stop()
     total_ms = hdist.max_over_ranks(t0.elapsed_time(t1), device)
     assert hs.hs_device_status(sh) == 0
     full_ms = [evs[s][0].elapsed_time(evs[s][1]) for s in range(args.steps)]
-    sparse_ms = [evs[s][1 + l].elapsed_time(evs[s][2 + l]) for s in range(args.steps)
-                 for l in range(w.n_sparse)]
+    if graphs:  # the sparse layers of a step run as one graph: per layer = step share / n
+        sparse_ms = [evs[s][1].elapsed_time(evs[s][2]) / w.n_sparse for s in range(args.steps)
+                     for _ in range(w.n_sparse)]
+    else:
+        sparse_ms = [evs[s][1 + l].elapsed_time(evs[s][2 + l]) for s in range(args.steps)
+                     for l in range(w.n_sparse)]
     ms_step = total_ms / args.steps
 
     p_tensor = peaks["bf16_tflops_sustained"] * 1e12
@@ -349,7 +370,9 @@ def run_ours(args, rank, world, device):
                    "block_size": w.block_size, "k": w.k, "window": w.window,
                    "decode": w.decode, "t_q": w.tq, "q_offset": w.q_offset,
                    "sparse_layers": w.n_sparse, "parallelism": f"replicas{world}",
-                   "l2": "inputs larger than L2 (step reads > 1 GB; K^F+V^F alone 134 MB)"},
+                   "l2": "inputs larger than L2 (step reads > 1 GB; K^F+V^F alone 134 MB)",
+                   "launch": "cuda graph replays (full-layer graph, sparse-layers graph)"
+                   if graphs else "per-call launches"},
         full_key: full_rate * world,
         "full_index_frac_of_peak": full_rate / full_peak,
         "sparse_kv_gbs": sparse_gbs * world,
@@ -362,6 +385,27 @@ def run_ours(args, rank, world, device):
         "e2e": e2e,
     }
     return line
+
+
+def capture_step(blk, w, device):
+    """CUDA graphs of one step: (full-layer graph, sparse-layers graph, kernels
+    captured in each).  The library's launches are recorded as they are
+    issued on the capture stream; replaying a graph launches the same kernels
+    on the same buffers without the per-call host work."""
+    from oracle_top_kv_b200 import hs
+    cap = torch.cuda.Stream(device)
+    cap.wait_stream(torch.cuda.current_stream(device))
+    g_full, g_sparse = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    c0 = hs.hs_launch_count()
+    with torch.cuda.graph(g_full, stream=cap):
+        blk.full(cap.cuda_stream)
+    c1 = hs.hs_launch_count()
+    with torch.cuda.graph(g_sparse, stream=cap):
+        for layer in range(w.n_sparse):
+            blk.sparse(layer, cap.cuda_stream)
+    c2 = hs.hs_launch_count()
+    torch.cuda.current_stream(device).wait_stream(cap)
+    return g_full, g_sparse, c1 - c0, c2 - c1
 
 
 def run_e2e(args, blk, w, stream, ideal, world, device):
@@ -498,6 +542,8 @@ def main():
     ap.add_argument("--batch", type=int, default=0, help="override the batch (reduced replica)")
     ap.add_argument("--seq", type=int, default=0, help="override the sequence length")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time per-call launches instead of CUDA graph replays")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
 

@@ -144,7 +144,10 @@ typedef enum { HS_DECODE_FULL_INDEX = 0, HS_DECODE_SPARSE = 1 } hs_decode_kind;
  * HS_DECODE_SPARSE: reads idx/idx_count and writes o (and lse) of the sparse
  *           layer with query q over K^F = k_cache, V^F = v_cache.
  * sel_scores: optional (FULL_INDEX only), as in hs_full_attn_index.
- * workspace: hs_workspace_size(p, HS_WS_DECODE_FULL / HS_WS_DECODE_SPARSE).
+ * workspace: hs_workspace_size(p, HS_WS_DECODE_FULL) bytes for FULL_INDEX;
+ *           HS_DECODE_SPARSE needs none (its size is 0; NULL allowed): one
+ *           kernel per step, each (sequence, group) on a cluster of CTAs that
+ *           merge their partial results in distributed shared memory.
  * The caller keeps k_cache, v_cache and idx alive until the last sparse layer
  * of the block has run.
  */
@@ -161,7 +164,9 @@ hs_status hs_decode_step(const hs_params* p, int32_t kind, const void* q,
  * the device).  It takes no workspace and allocates nothing: its scratch is a
  * fixed 32 MiB array inside the library, present on every GPU that loads the
  * library until the process exits.  (The pages have no counterpart of this
- * entry point; it only changes where the scratch lives.)
+ * entry point.)  It runs the split-k form of the step -- a split kernel that
+ * writes per-split partial results, then a combine kernel -- with those
+ * partials in the library's array.
  *
  * Arguments, layouts and results are those of hs_decode_step with
  * kind = HS_DECODE_SPARSE.  Limits: batch * hkv * ceil(k / 64) split units of

@@ -20,6 +20,7 @@
 //     unit, serves budgets above 1024).
 #include "attend_mma.cuh"
 #include "block_topk.cuh"
+#include "cta_select.cuh"
 #include "hs_common.cuh"
 #include "hs_kernels.cuh"
 
@@ -33,16 +34,27 @@ constexpr int kDecodeKeys = 2048;  // cache keys per split
 constexpr int kDecodeWarps = 4;
 constexpr int kSelectThreads = 512;
 
-constexpr int kSelSplits = 8;          // CTAs per (sequence, group) in the selector
+constexpr int kSelSlice = 16384;       // most ranked keys one selector CTA stages
 constexpr int kSelMaxRanked = 1024;    // k - w handled by the split selector
+constexpr int kMergeCap = 8192;        // candidate keys the merge holds at once
+
+// CTAs per (sequence, group) in the split selector: slices of at most
+// kSelSlice keys, and enough CTAs for about two per SM of a 148-SM part
+// (slices not shorter than 2048 keys).
+static int sel_splits(const KParams& p) {
+    const int units = p.batch * p.hkv;
+    const int by_len = (p.t_kv + kSelSlice - 1) / kSelSlice;
+    const int by_fill = min((296 + units - 1) / units, (p.t_kv + 2047) / 2048);
+    return max(1, max(by_len, by_fill));
+}
 
 struct DecodeWs {
     float* logits;    // [batch*hkv][t_kv][16]
     float* part;      // [batch*hkv][n_split][16][D+2]
     float* lse2;      // [batch*hq]
-    uint64_t* cand;   // [batch*hkv][kSelSplits][kSelMaxRanked] selection keys
-    int* cand_n;      // [batch*hkv][kSelSplits]
-    int n_split;
+    uint64_t* cand;   // [batch*hkv][n_sel][kSelMaxRanked] selection keys
+    int* cand_n;      // [batch*hkv][n_sel]
+    int n_split, n_sel;
 };
 
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -50,11 +62,12 @@ static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 static DecodeWs decode_ws_layout(const KParams& p, void* base) {
     DecodeWs w;
     w.n_split = (p.t_kv + kDecodeKeys - 1) / kDecodeKeys;
+    w.n_sel = sel_splits(p);
     const size_t units = (size_t)p.batch * p.hkv;
     const size_t logits_b = align256(units * p.t_kv * 16 * sizeof(float));
     const size_t part_b = align256(units * w.n_split * 16 * (p.head_dim + 2) * sizeof(float));
     const size_t lse_b = align256((size_t)p.batch * p.hq * sizeof(float));
-    const size_t cand_b = align256(units * kSelSplits * kSelMaxRanked * sizeof(uint64_t));
+    const size_t cand_b = align256(units * w.n_sel * kSelMaxRanked * sizeof(uint64_t));
     char* c = static_cast<char*>(base);
     w.logits = reinterpret_cast<float*>(c);
     w.part = reinterpret_cast<float*>(c + logits_b);
@@ -70,8 +83,8 @@ size_t decode_full_workspace(const KParams& p) {
     return align256(units * p.t_kv * 16 * sizeof(float)) +
            align256(units * n_split * 16 * (p.head_dim + 2) * sizeof(float)) +
            align256((size_t)p.batch * p.hq * sizeof(float)) +
-           align256(units * kSelSplits * kSelMaxRanked * sizeof(uint64_t)) +
-           align256(units * kSelSplits * sizeof(int));
+           align256(units * sel_splits(p) * kSelMaxRanked * sizeof(uint64_t)) +
+           align256(units * sel_splits(p) * sizeof(int));
 }
 
 // Writes every head's scaled logit a2 = scale_log2 * q.k of the chunk's keys.
@@ -223,57 +236,84 @@ __device__ __forceinline__ float group_score(const float* lg_row, const float* l
     return s;
 }
 
-// Stage 1 of the split selector: CTA (unit, split) keeps the exact top-(k-w)
-// of its slice of the ranked keys 0..t-w and writes them out unsorted.  The
-// group's top-(k-w) is contained in the union of the slices' top-(k-w).
+// Stage 1 of the split selector: CTA (unit, slice) stages the group scores of
+// its slice of the ranked keys 0..t-w in shared memory (as order bits), finds
+// the slice's (k-w)-th largest selection key with a CTA-wide bucket select,
+// and writes the slice's top-(k-w) keys out unsorted.  The group's top-(k-w)
+// is contained in the union of the slices' top-(k-w).
 __global__ void __launch_bounds__(kSelectThreads)
     decode_select_split_kernel(KParams p, const int32_t* __restrict__ seq_len, DecodeWs ws) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    __shared__ int s_count;
-    __shared__ unsigned long long s_thresh;
+    __shared__ CtaSelectSmem cs;
     __shared__ float s_lse2[16];
-    const int unit = blockIdx.x / kSelSplits, sp = blockIdx.x % kSelSplits;
+    __shared__ int s_n;
+    uint32_t* bits = reinterpret_cast<uint32_t*>(smem_raw);  // [kSelSlice]
+    const int unit = blockIdx.x / ws.n_sel, sp = blockIdx.x % ws.n_sel;
     const int u = unit % p.hkv, b = unit / p.hkv;
     const int g = p.group;
     const int L = seq_len[b];
     const int Kc = p.k - p.window;
-    int* out_n = ws.cand_n + (size_t)unit * kSelSplits + sp;
+    int* out_n = ws.cand_n + (size_t)unit * ws.n_sel + sp;
     if (L < 1 || L > p.t_kv || L <= p.k || Kc <= 0) {  // nothing ranked here
         if (threadIdx.x == 0) *out_n = 0;
         return;
     }
     const int lo = L - p.window;  // ranked keys 0..lo-1
-    const int per = (lo + kSelSplits - 1) / kSelSplits;
-    const int i0 = sp * per, i1 = min(lo, i0 + per);
-    BlockTopK topk;
-    topk.setup(smem_raw, Kc, blockDim.x, &s_count, &s_thresh);
+    const int per = (lo + ws.n_sel - 1) / ws.n_sel;  // <= kSelSlice
+    const int i0 = sp * per;
+    const int n = max(0, min(lo, i0 + per) - i0);
     if (threadIdx.x < 16) s_lse2[threadIdx.x] = threadIdx.x < g ? ws.lse2[b * p.hq + u * g + threadIdx.x] : 0.f;
     __syncthreads();
     const float* lg = ws.logits + (size_t)unit * p.t_kv * 16;
-    for (int c0 = i0; c0 < i1; c0 += blockDim.x) {
-        const int i = c0 + threadIdx.x;
-        if (i < i1) topk.offer(group_score(lg + (size_t)i * 16, s_lse2, g), (uint32_t)i);
-        topk.end_round();
+#pragma unroll 4
+    for (int i = threadIdx.x; i < n; i += blockDim.x)
+        bits[i] = float_order(group_score(lg + (size_t)(i0 + i) * 16, s_lse2, g));
+    __syncthreads();
+    auto key = [&](int i) -> uint64_t {
+        return ((uint64_t)bits[i] << 32) | (uint64_t)(0xffffffffu - (uint32_t)(i0 + i));
+    };
+    uint64_t* dst = ws.cand + ((size_t)unit * ws.n_sel + sp) * kSelMaxRanked;
+    if (n <= Kc) {
+        for (int i = threadIdx.x; i < n; i += blockDim.x) dst[i] = key(i);
+        if (threadIdx.x == 0) *out_n = n;
+        return;
+    }
+    const uint64_t kth = cta_kth_largest(key, n, Kc, cs);
+    if (threadIdx.x == 0) s_n = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const uint64_t v = key(i);
+        if (v >= kth) dst[atomicAdd(&s_n, 1)] = v;
     }
     __syncthreads();
-    if (threadIdx.x >= 32) return;
-    int n = *topk.count;
-    if (n > Kc) { warp_cut_to_k(topk.buf, n, Kc, topk.hist); n = Kc; }
-    __syncwarp();
-    uint64_t* dst = ws.cand + ((size_t)unit * kSelSplits + sp) * kSelMaxRanked;
-    for (int x = threadIdx.x; x < n; x += 32) dst[x] = topk.buf[x];
-    if (threadIdx.x == 0) *out_n = n;
+    if (threadIdx.x == 0) *out_n = s_n;  // exactly Kc: the keys are distinct
 }
 
-// Stage 2: per unit, the final top-(k-w) of the slices' candidates, sorted by
-// id, then the forced window; or every key when the budget covers them all.
+// Keep the K largest of buf[0..n) (n > K), in buf[0..K); tmp holds K keys.
+__device__ int cta_cut(uint64_t* buf, int n, int K, uint64_t* tmp, CtaSelectSmem& cs,
+                       int* s_n) {
+    const uint64_t kth = cta_kth_largest([&](int i) { return buf[i]; }, n, K, cs);
+    if (threadIdx.x == 0) *s_n = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x)
+        if (buf[i] >= kth) tmp[atomicAdd(s_n, 1)] = buf[i];
+    __syncthreads();
+    for (int i = threadIdx.x; i < K; i += blockDim.x) buf[i] = tmp[i];
+    __syncthreads();
+    return K;
+}
+
+// Stage 2: per unit, the final top-(k-w) of the slices' candidates (cut to
+// k-w whenever the buffer would overflow), sorted by id, then the forced
+// window; or every key when the budget covers them all.
 __global__ void __launch_bounds__(kSelectThreads)
     decode_select_merge_kernel(KParams p, const int32_t* __restrict__ seq_len, DecodeWs ws,
                                int32_t* __restrict__ idx, int32_t* __restrict__ cnt,
                                float* __restrict__ sel) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
+    __shared__ CtaSelectSmem cs;
     __shared__ float s_lse2[16];
-    __shared__ int s_base[kSelSplits + 1];
+    __shared__ int s_n;
     const int unit = blockIdx.x;
     const int u = unit % p.hkv, b = unit / p.hkv;
     const int g = p.group;
@@ -291,14 +331,6 @@ __global__ void __launch_bounds__(kSelectThreads)
     const int t = L - 1;
     const int Kc = p.k - p.window;
     if (threadIdx.x < 16) s_lse2[threadIdx.x] = threadIdx.x < g ? ws.lse2[b * p.hq + u * g + threadIdx.x] : 0.f;
-    if (threadIdx.x == 0) {
-        int acc = 0;
-        for (int sp = 0; sp < kSelSplits; ++sp) {
-            s_base[sp] = acc;
-            acc += ws.cand_n[(size_t)unit * kSelSplits + sp];
-        }
-        s_base[kSelSplits] = acc;
-    }
     __syncthreads();
     const float* lg = ws.logits + (size_t)unit * p.t_kv * 16;
     if (t + 1 <= p.k) {  // the budget covers every key
@@ -314,33 +346,32 @@ __global__ void __launch_bounds__(kSelectThreads)
     if (srow)
         for (int x = threadIdx.x; x <= t - lo; x += blockDim.x)
             srow[Kc + x] = exp2f(group_score(lg + (size_t)(lo + x) * 16, s_lse2, g));
-    uint64_t* buf = reinterpret_cast<uint64_t*>(smem_raw);          // [kSplits * Kc]
-    uint64_t* sortb = buf + kSelSplits * kSelMaxRanked;              // [next_pow2(Kc)]
-    uint32_t* hist = reinterpret_cast<uint32_t*>(sortb + kSelMaxRanked);
-    const int total = s_base[kSelSplits];
-    for (int sp = 0; sp < kSelSplits; ++sp) {
-        const uint64_t* src = ws.cand + ((size_t)unit * kSelSplits + sp) * kSelMaxRanked;
-        const int n = s_base[sp + 1] - s_base[sp];
-        for (int x = threadIdx.x; x < n; x += blockDim.x) buf[s_base[sp] + x] = src[x];
+    uint64_t* buf = reinterpret_cast<uint64_t*>(smem_raw);  // [kMergeCap]
+    uint64_t* tmp = buf + kMergeCap;                         // [kSelMaxRanked]
+    int n = 0;
+    if (Kc > 0) {
+        for (int sp = 0; sp < ws.n_sel; ++sp) {
+            const int c = ws.cand_n[(size_t)unit * ws.n_sel + sp];
+            if (n + c > kMergeCap) n = cta_cut(buf, n, Kc, tmp, cs, &s_n);
+            const uint64_t* src = ws.cand + ((size_t)unit * ws.n_sel + sp) * kSelMaxRanked;
+            for (int x = threadIdx.x; x < c; x += blockDim.x) buf[n + x] = src[x];
+            n += c;
+            __syncthreads();
+        }
+        if (n > Kc) n = cta_cut(buf, n, Kc, tmp, cs, &s_n);
     }
-    __syncthreads();
-    if (threadIdx.x >= 32) return;
-    int n = total;
-    if (Kc > 0 && n > Kc) { warp_cut_to_k(buf, n, Kc, hist); n = Kc; }
-    if (Kc <= 0) n = 0;
-    __syncwarp();
     const int sort_n = next_pow2(Kc > 0 ? Kc : 1);
-    for (int x = threadIdx.x; x < sort_n; x += 32)
-        sortb[x] = x < n ? (((uint64_t)sel_key_id(buf[x]) << 32) | (buf[x] >> 32)) : ~0ull;
-    __syncwarp();
-    warp_bitonic_sort(sortb, sort_n);
-    for (int x = threadIdx.x; x < n; x += 32) {
-        irow[x] = (int32_t)(sortb[x] >> 32);
-        if (srow) srow[x] = exp2f(order_float((uint32_t)(sortb[x] & 0xffffffffu)));
+    for (int x = threadIdx.x; x < sort_n; x += blockDim.x)
+        tmp[x] = x < n ? (((uint64_t)sel_key_id(buf[x]) << 32) | (buf[x] >> 32)) : ~0ull;
+    __syncthreads();
+    cta_bitonic_sort(tmp, sort_n);
+    for (int x = threadIdx.x; x < n; x += blockDim.x) {
+        irow[x] = (int32_t)(tmp[x] >> 32);
+        if (srow) srow[x] = exp2f(order_float((uint32_t)(tmp[x] & 0xffffffffu)));
     }
-    for (int x = threadIdx.x; x <= t - lo; x += 32) irow[n + x] = lo + x;
+    for (int x = threadIdx.x; x <= t - lo; x += blockDim.x) irow[n + x] = lo + x;
     const int n_out = n + (t - lo + 1);
-    for (int x = n_out + threadIdx.x; x < p.ksel; x += 32) {
+    for (int x = n_out + threadIdx.x; x < p.ksel; x += blockDim.x) {
         irow[x] = -1;
         if (srow) srow[x] = 0.f;
     }
@@ -372,15 +403,14 @@ static cudaError_t launch_decode_full_t(const KParams& p, const void* q, const v
         return e;
     const int Kc = p.k - p.window;
     if (Kc <= kSelMaxRanked) {
-        const size_t s1 = BlockTopK::smem_bytes(Kc, kSelectThreads);
+        const size_t s1 = sizeof(uint32_t) * kSelSlice;
         e = cudaFuncSetAttribute(decode_select_split_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1);
         if (e != cudaSuccess) return e;
-        decode_select_split_kernel<<<p.batch * p.hkv * kSelSplits, kSelectThreads, s1, st>>>(
+        decode_select_split_kernel<<<p.batch * p.hkv * w.n_sel, kSelectThreads, s1, st>>>(
             p, seq_len, w);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        const size_t s2 = sizeof(uint64_t) * (kSelSplits * kSelMaxRanked + kSelMaxRanked) +
-                          sizeof(uint32_t) * 256;
+        const size_t s2 = sizeof(uint64_t) * (kMergeCap + kSelMaxRanked);
         e = cudaFuncSetAttribute(decode_select_merge_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2);
         if (e != cudaSuccess) return e;

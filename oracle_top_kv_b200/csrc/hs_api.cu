@@ -207,7 +207,7 @@ hs_status hs_decode_step(const hs_params* p, int32_t kind, const void* q, const 
                                           lse, sel_scores, workspace, st);
         });
     }
-    return launched(2, [&] {
+    return launched(1, [&] {
         return hs::launch_decode_sparse(kp, q, k_cache, v_cache, seq_len, idx, idx_count, o, lse,
                                         workspace, st);
     });
@@ -224,7 +224,7 @@ hs_status hs_decode_sparse_noalloc(const hs_params* p, const void* q, const void
     if (!ok_ptr(q) || !ok_ptr(k_cache) || !ok_ptr(v_cache) || !ok_ptr(seq_len) || !ok_ptr(idx) ||
         !ok_ptr(idx_count) || !ok_ptr(o) || !ok_opt(lse))
         return HS_ERR_INVALID_ARG;
-    if (hs::decode_sparse_workspace(kp) > hs::noalloc_scratch_bytes()) return HS_ERR_WORKSPACE;
+    if (hs::decode_sparse_split_workspace(kp) > hs::noalloc_scratch_bytes()) return HS_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return launched(2, [&] {
         return hs::launch_decode_sparse_noalloc(kp, q, k_cache, v_cache, seq_len, idx, idx_count,

@@ -49,9 +49,16 @@ size_t decode_sparse_workspace(const KParams& p);
 cudaError_t launch_decode_full(const KParams& p, const void* q, const void* kc, const void* vc,
                                const int32_t* seq_len, int32_t* idx, int32_t* cnt, void* o,
                                float* lse, float* sel, void* ws, cudaStream_t st);
+// One clustered kernel per sparse step; ws is unused (the workspace size is 0).
 cudaError_t launch_decode_sparse(const KParams& p, const void* q, const void* kc, const void* vc,
                                  const int32_t* seq_len, const int32_t* idx, const int32_t* cnt,
                                  void* o, float* lse, void* ws, cudaStream_t st);
+// Split-k sparse step (split kernel + combine) with partials in `ws`.
+size_t decode_sparse_split_workspace(const KParams& p);
+cudaError_t launch_decode_sparse_split(const KParams& p, const void* q, const void* kc,
+                                       const void* vc, const int32_t* seq_len, const int32_t* idx,
+                                       const int32_t* cnt, void* o, float* lse, void* ws,
+                                       cudaStream_t st);
 
 // Token-mode selection on the tensor cores (bf16, d = 128, 16 heads per group,
 // k - w <= 1024); reads lse from the attention pass.

@@ -4,10 +4,10 @@
 // Some callers are handed only their input and output buffers: a plugin
 // inside an inference engine whose memory planner owns every device byte, or
 // a latency-critical decode loop where a cudaMalloc (which can synchronise
-// the device) is not allowed.  Such a caller cannot provide the split-k
-// workspace that hs_decode_step(HS_DECODE_SPARSE) needs.  This entry point
-// runs the very same kernels with their scratch in a fixed file-scope device
-// array instead; it allocates nothing.
+// the device) is not allowed.  This entry point runs the split-k form of the
+// sparse decode step (a split kernel writing per-split partials, then a
+// combine kernel) with its scratch in a fixed file-scope device array instead
+// of a caller workspace; it allocates nothing.
 //
 // The array exists once per device for as long as the library stays loaded
 // (every GPU that loads the library holds it until exit).  Host code cannot
@@ -62,7 +62,7 @@ cudaError_t launch_decode_sparse_noalloc(const KParams& p, const void* q, const 
     void* scratch = nullptr;
     cudaError_t e = noalloc_scratch(&scratch);
     if (e != cudaSuccess) return e;
-    return launch_decode_sparse(p, q, kc, vc, seq_len, idx, cnt, o, lse, scratch, st);
+    return launch_decode_sparse_split(p, q, kc, vc, seq_len, idx, cnt, o, lse, scratch, st);
 }
 
 }  // namespace hs

@@ -16,6 +16,8 @@
 //                       the 16 MMA rows, so each gathered row is read once.
 //   decode_sparse_*     bf16 decode: the selected rows of one (sequence, group)
 //                       split across warps, then an exact log-sum-exp merge.
+#include <atomic>
+
 #include "attend_mma.cuh"
 #include "hs_common.cuh"
 #include "hs_kernels.cuh"
@@ -366,55 +368,62 @@ __global__ void __launch_bounds__(kSparseWarps * 32)
 }
 
 // Exact merge of split partials: M = max m_s, l = sum l_s 2^(m_s - M),
-// o = sum O_s 2^(m_s - M) / l.  One warp per (sequence, head).
+// o = sum O_s 2^(m_s - M) / l.  One CTA of D threads per (sequence, head);
+// thread d accumulates element d over all splits.
 template <int D>
-__global__ void decode_combine_kernel(KParams p, const float* __restrict__ part, int n_split,
-                                      const int32_t* __restrict__ seq_len,
-                                      __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
-                                      float* __restrict__ lse2_out) {
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (warp >= p.batch * p.hq) return;
-    const int h = warp % p.hq, b = warp / p.hq;
+__global__ void __launch_bounds__(D)
+    decode_combine_kernel(KParams p, const float* __restrict__ part, int n_split,
+                          const int32_t* __restrict__ seq_len, __nv_bfloat16* __restrict__ o,
+                          float* __restrict__ lse, float* __restrict__ lse2_out) {
+    __shared__ float red_m[D / 32], red_l[D / 32];
+    const int row = blockIdx.x;  // b * hq + h
+    const int h = row % p.hq, b = row / p.hq;
     const int g = p.group, u = h / g, hh = h % g;
     const int unit = b * p.hkv + u;
+    const int d = threadIdx.x, lane = d & 31, warp = d >> 5;
     const int L = seq_len[b];
-    constexpr int E = D / 32;
+    constexpr size_t S = 16 * (D + 2);  // floats between consecutive splits
+    const float* base = part + (size_t)unit * n_split * S + (size_t)hh * (D + 2);
     float M = -INFINITY;
-    for (int s = 0; s < n_split; ++s)
-        M = fmaxf(M, part[((size_t)unit * n_split + s) * 16 * (D + 2) + hh * (D + 2)]);
+    for (int s = d; s < n_split; s += D) M = fmaxf(M, base[s * S]);
+    M = warp_max(M);
+    if (lane == 0) red_m[warp] = M;
+    __syncthreads();
+#pragma unroll
+    for (int w = 0; w < D / 32; ++w) M = fmaxf(M, red_m[w]);
     const float Mu = M == -INFINITY ? 0.f : M;
-    float l = 0.f, acc[E];
+    float l = 0.f;
+    for (int s = d; s < n_split; s += D) l += base[s * S + 1] * exp2f(base[s * S] - Mu);
+    l = warp_sum(l);
+    if (lane == 0) red_l[warp] = l;
+    float acc = 0.f;
+#pragma unroll 8
+    for (int s = 0; s < n_split; ++s) acc += base[s * S + 2 + d] * exp2f(base[s * S] - Mu);
+    __syncthreads();
+    l = 0.f;
 #pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = 0.f;
-    for (int s = 0; s < n_split; ++s) {
-        const float* ph = part + ((size_t)unit * n_split + s) * 16 * (D + 2) + hh * (D + 2);
-        const float w = exp2f(ph[0] - Mu);
-        l += ph[1] * w;
-#pragma unroll
-        for (int e = 0; e < E; ++e) acc[e] += ph[2 + lane * E + e] * w;
-    }
+    for (int w = 0; w < D / 32; ++w) l += red_l[w];
     const bool ok = L >= 1 && L <= p.t_kv && l > 0.f;
-    const float inv = ok ? 1.f / l : 0.f;
-#pragma unroll
-    for (int e = 0; e < E; ++e) o[(size_t)warp * D + lane * E + e] = __float2bfloat16_rn(acc[e] * inv);
-    if (lane == 0) {
+    o[(size_t)row * D + d] = __float2bfloat16_rn(ok ? acc / l : 0.f);
+    if (d == 0) {
         const float l2 = ok ? M + log2f(l) : -INFINITY;
-        if (lse) lse[warp] = l2 * kLn2;
-        if (lse2_out) lse2_out[warp] = l2;
+        if (lse) lse[row] = l2 * kLn2;
+        if (lse2_out) lse2_out[row] = l2;
     }
 }
 
-size_t decode_sparse_workspace(const KParams& p) {
+size_t decode_sparse_split_workspace(const KParams& p) {
     const int n_split = (p.ksel + kDecodeSparseRows - 1) / kDecodeSparseRows;
     return (size_t)p.batch * p.hkv * n_split * 16 * (p.head_dim + 2) * sizeof(float);
 }
 
+// The split-k pair above with its partials in caller-provided scratch (used by
+// the allocation-free entry point, whose scratch is a library array).
 template <int D>
-static cudaError_t launch_decode_sparse_t(const KParams& p, const void* q, const void* kc,
-                                          const void* vc, const int32_t* seq_len,
-                                          const int32_t* idx, const int32_t* cnt, void* o,
-                                          float* lse, void* ws, cudaStream_t st) {
+static cudaError_t launch_decode_sparse_split_t(const KParams& p, const void* q, const void* kc,
+                                                const void* vc, const int32_t* seq_len,
+                                                const int32_t* idx, const int32_t* cnt, void* o,
+                                                float* lse, void* ws, cudaStream_t st) {
     const int n_split = (p.ksel + kDecodeSparseRows - 1) / kDecodeSparseRows;
     const size_t smem = (size_t)kSparseWarps * WarpSmem<D>::kBytes + 1024;
     auto kern = decode_sparse_split_kernel<D>;
@@ -426,32 +435,251 @@ static cudaError_t launch_decode_sparse_t(const KParams& p, const void* q, const
         p, (const __nv_bfloat16*)q, (const __nv_bfloat16*)kc, (const __nv_bfloat16*)vc, seq_len,
         idx, cnt, (float*)ws, n_split);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const int warps = p.batch * p.hq;
-    decode_combine_kernel<D><<<(warps + 7) / 8, 256, 0, st>>>(p, (const float*)ws, n_split,
-                                                              seq_len, (__nv_bfloat16*)o, lse,
-                                                              nullptr);
+    decode_combine_kernel<D><<<p.batch * p.hq, D, 0, st>>>(p, (const float*)ws, n_split, seq_len,
+                                                           (__nv_bfloat16*)o, lse, nullptr);
     return cudaGetLastError();
+}
+
+cudaError_t launch_decode_sparse_split(const KParams& p, const void* q, const void* kc,
+                                       const void* vc, const int32_t* seq_len, const int32_t* idx,
+                                       const int32_t* cnt, void* o, float* lse, void* ws,
+                                       cudaStream_t st) {
+    if (p.head_dim == 64)
+        return launch_decode_sparse_split_t<64>(p, q, kc, vc, seq_len, idx, cnt, o, lse, ws, st);
+    return launch_decode_sparse_split_t<128>(p, q, kc, vc, seq_len, idx, cnt, o, lse, ws, st);
+}
+
+// ---------------------------------------------- decode, one kernel per step
+// One (sequence, group) unit per thread-block cluster of `csize` CTAs of
+// kSparseWarps warps.  The unit's selected rows are dealt out to the
+// 6 * csize warps in 32-row chunks (warp w takes chunks w, w + W, ...); each
+// warp attends its chunks with the same cp.async gather ring as the prefill
+// kernel, the CTA merges its warps' partials in shared memory, and CTA 0 of
+// the cluster merges the CTAs' partials read through distributed shared
+// memory and writes o and lse.  Every merge is the exact one of split-k
+// attention: M = max m_s, l = sum l_s 2^(m_s - M), o = sum O_s 2^(m_s - M) / l.
+// Nothing goes through global memory, so the step needs no workspace.
+
+// Rows of the unit's index list owned by one warp: its chunk cc is the
+// list's chunk first + cc * stride.
+struct StridedGather {
+    static constexpr bool kContig = false;
+    const int32_t* ids;
+    int n_rows, t, first, stride;
+    __device__ __forceinline__ int key(int r) const {
+        const int row = (first + (r >> 5) * stride) * kChunk + (r & 31);
+        if (row >= n_rows) return -1;
+        const int key = ids[row];
+        if (key < 0 || key > t) { set_status(HS_ERR_BOUNDS); return -1; }
+        return key;
+    }
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+                 ::: "memory");
+}
+
+// fp32 at shared address `a` of cluster CTA `rank`.
+__device__ __forceinline__ float ld_cluster_f32(uint32_t a, uint32_t rank) {
+    uint32_t ra;
+    float v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+    return v;
+}
+
+template <int D>
+struct DecodeSmem {
+    static constexpr int kPart = 16 * (D + 2);  // floats of one partial [16][D + 2]
+    static constexpr size_t kRing = (size_t)kSparseWarps * WarpSmem<D>::kBytes;
+    static constexpr size_t kBytes = kRing + kPart * sizeof(float) + 32 * sizeof(float) + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kSparseWarps * 32)
+    decode_sparse_cluster_kernel(KParams p, const __nv_bfloat16* __restrict__ q,
+                                 const __nv_bfloat16* __restrict__ kc,
+                                 const __nv_bfloat16* __restrict__ vc,
+                                 const int32_t* __restrict__ seq_len,
+                                 const int32_t* __restrict__ idx,
+                                 const int32_t* __restrict__ cnt, int csize,
+                                 __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    using S = DecodeSmem<D>;
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    unsigned char* gbase = smem_raw + (base - raw);
+    float* cta_part = reinterpret_cast<float*>(gbase + S::kRing);  // [16][D + 2]
+    float* s_ml = cta_part + S::kPart;                              // M[16], l[16]
+    const int warp = threadIdx.x >> 5;
+    const int crank = csize > 1 ? (int)cluster_rank() : 0;
+    const int unit = blockIdx.x / csize;  // b * hkv + u
+    const int u = unit % p.hkv, b = unit / p.hkv;
+    const int g = p.group;
+    const int L = seq_len[b];
+    const bool valid = L >= 1 && L <= p.t_kv;
+    float* wpart = reinterpret_cast<float*>(gbase + (size_t)warp * WarpSmem<D>::kBytes);
+
+    AttnState<D> st;
+    st.init();
+    if (valid) {
+        const int t = L - 1;
+        const int c = clamp_count(cnt[unit], p.ksel);
+        const int n_chunks = (c + kChunk - 1) / kChunk;
+        const int W = kSparseWarps * csize;
+        const int wg = crank * kSparseWarps + warp;
+        const int mine = wg < n_chunks ? (n_chunks - 1 - wg) / W + 1 : 0;
+        uint32_t qf[D / 16][4];
+        load_q_frags<D>(qf, q + ((size_t)b * p.hq + u * g) * D, D, g);
+        const StridedGather keys{idx + (size_t)unit * p.ksel, c, t, wg, W};
+        const size_t kvoff = (size_t)unit * p.t_kv * D;
+        attend_rows<D>(st, qf, kc + kvoff, vc + kvoff, mine, keys,
+                       base + warp * WarpSmem<D>::kBytes, p.scale_log2, NoHook{});
+    } else if (crank == 0 && threadIdx.x == 0) {
+        set_status(HS_ERR_BOUNDS);
+    }
+    __syncwarp();
+    store_partial<D>(st, wpart, g);  // the warp's ring is drained: reuse it
+    __syncthreads();
+
+    // CTA merge of the warps' partials.
+    constexpr int P = D + 2;
+    if (threadIdx.x < g) {
+        const int h = threadIdx.x;
+        float M = -INFINITY;
+        for (int w = 0; w < kSparseWarps; ++w)
+            M = fmaxf(M, reinterpret_cast<const float*>(gbase + (size_t)w * WarpSmem<D>::kBytes)[h * P]);
+        const float Mu = M == -INFINITY ? 0.f : M;
+        float l = 0.f;
+        for (int w = 0; w < kSparseWarps; ++w) {
+            const float* ph = reinterpret_cast<const float*>(gbase + (size_t)w * WarpSmem<D>::kBytes) + h * P;
+            l += ph[1] * exp2f(ph[0] - Mu);
+        }
+        s_ml[h] = M;
+        s_ml[16 + h] = l;
+        cta_part[h * P] = M;
+        cta_part[h * P + 1] = l;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < g * D; e += blockDim.x) {
+        const int h = e / D, d = e % D;
+        const float M = s_ml[h];
+        const float Mu = M == -INFINITY ? 0.f : M;
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kSparseWarps; ++w) {
+            const float* ph = reinterpret_cast<const float*>(gbase + (size_t)w * WarpSmem<D>::kBytes) + h * P;
+            acc += ph[2 + d] * exp2f(ph[0] - Mu);
+        }
+        cta_part[h * P + 2 + d] = acc;
+    }
+    if (csize > 1) cluster_sync_all();  // the CTAs' partials are visible cluster-wide
+    else __syncthreads();
+
+    if (crank == 0) {
+        const uint32_t part_addr = base + (uint32_t)S::kRing;
+        auto rd = [&](int r, int off) -> float {
+            return csize > 1 ? ld_cluster_f32(part_addr + 4u * off, (uint32_t)r) : cta_part[off];
+        };
+        for (int e = threadIdx.x; e < g * D; e += blockDim.x) {
+            const int h = e / D, d = e % D;
+            float M = -INFINITY;
+            for (int r = 0; r < csize; ++r) M = fmaxf(M, rd(r, h * P));
+            const float Mu = M == -INFINITY ? 0.f : M;
+            float l = 0.f, acc = 0.f;
+            for (int r = 0; r < csize; ++r) {
+                const float w = exp2f(rd(r, h * P) - Mu);
+                l += rd(r, h * P + 1) * w;
+                acc += rd(r, h * P + 2 + d) * w;
+            }
+            const bool ok = valid && l > 0.f;
+            const size_t orow = (size_t)b * p.hq + u * g + h;
+            o[orow * D + d] = __float2bfloat16_rn(ok ? acc / l : 0.f);
+            if (d == 0 && lse) lse[orow] = ok ? (M + log2f(l)) * kLn2 : -INFINITY;
+        }
+    }
+    if (csize > 1) cluster_sync_all();  // peers keep their shared memory until CTA 0 is done
+}
+
+size_t decode_sparse_workspace(const KParams&) { return 0; }
+
+template <int D>
+static cudaError_t launch_decode_sparse_t(const KParams& p, const void* q, const void* kc,
+                                          const void* vc, const int32_t* seq_len,
+                                          const int32_t* idx, const int32_t* cnt, void* o,
+                                          float* lse, cudaStream_t st) {
+    auto kern = decode_sparse_cluster_kernel<D>;
+    const size_t smem = DecodeSmem<D>::kBytes;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+    // Widest cluster (<= 8 CTAs, one per SM) that still fits the units in one wave.
+    const int units = p.batch * p.hkv;
+    const int chunks = (p.ksel + kChunk - 1) / kChunk;
+    int csize = 1;
+    while (csize < 8 && units * csize * 2 <= sms && kSparseWarps * csize < chunks) csize *= 2;
+    for (;; csize /= 2) {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        cfg.gridDim = dim3((unsigned)(units * csize));
+        cfg.blockDim = dim3(kSparseWarps * 32);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)csize;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = csize > 1 ? 1 : 0;
+        if (csize > 1) {  // can the device co-schedule a cluster this wide? (cached)
+            static std::atomic<int> fits[64][4];  // 0 unknown, 1 yes, -1 no
+            const int lvl = csize == 2 ? 1 : csize == 4 ? 2 : 3;
+            int f = dev < 64 ? fits[dev][lvl].load(std::memory_order_relaxed) : 0;
+            if (f == 0) {
+                int n = 0;
+                f = cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n >= 1 ? 1
+                                                                                             : -1;
+                (void)cudaGetLastError();
+                if (dev < 64) fits[dev][lvl].store(f, std::memory_order_relaxed);
+            }
+            if (f < 0) continue;
+        }
+        return cudaLaunchKernelEx(&cfg, kern, p, (const __nv_bfloat16*)q,
+                                  (const __nv_bfloat16*)kc, (const __nv_bfloat16*)vc, seq_len,
+                                  idx, cnt, csize, (__nv_bfloat16*)o, lse);
+    }
 }
 
 cudaError_t launch_decode_sparse(const KParams& p, const void* q, const void* kc, const void* vc,
                                  const int32_t* seq_len, const int32_t* idx, const int32_t* cnt,
-                                 void* o, float* lse, void* ws, cudaStream_t st) {
+                                 void* o, float* lse, void*, cudaStream_t st) {
     if (p.head_dim == 64)
-        return launch_decode_sparse_t<64>(p, q, kc, vc, seq_len, idx, cnt, o, lse, ws, st);
-    return launch_decode_sparse_t<128>(p, q, kc, vc, seq_len, idx, cnt, o, lse, ws, st);
+        return launch_decode_sparse_t<64>(p, q, kc, vc, seq_len, idx, cnt, o, lse, st);
+    return launch_decode_sparse_t<128>(p, q, kc, vc, seq_len, idx, cnt, o, lse, st);
 }
 
 // Shared with decode_full.cu.
 cudaError_t launch_decode_combine(const KParams& p, const float* part, int n_split,
                                   const int32_t* seq_len, void* o, float* lse, float* lse2,
                                   cudaStream_t st) {
-    const int warps = p.batch * p.hq;
+    const int rows = p.batch * p.hq;
     if (p.head_dim == 64)
-        decode_combine_kernel<64><<<(warps + 7) / 8, 256, 0, st>>>(
-            p, part, n_split, seq_len, (__nv_bfloat16*)o, lse, lse2);
+        decode_combine_kernel<64><<<rows, 64, 0, st>>>(p, part, n_split, seq_len,
+                                                       (__nv_bfloat16*)o, lse, lse2);
     else
-        decode_combine_kernel<128><<<(warps + 7) / 8, 256, 0, st>>>(
-            p, part, n_split, seq_len, (__nv_bfloat16*)o, lse, lse2);
+        decode_combine_kernel<128><<<rows, 128, 0, st>>>(p, part, n_split, seq_len,
+                                                         (__nv_bfloat16*)o, lse, lse2);
     return cudaGetLastError();
 }
 

@@ -114,6 +114,7 @@ def test_workspace_sizes(lib):
     assert hs.hs_workspace_size(_p(), hs.HS_WS_FULL) == 0
     assert hs.hs_workspace_size(_p(), hs.HS_WS_SPARSE) == 0
     p = _p(t_q=1, t_kv=1024, mode="token", block_size=1)
-    assert hs.hs_workspace_size(p, hs.HS_WS_DECODE_SPARSE) > 0
+    assert hs.hs_workspace_size(p, hs.HS_WS_DECODE_SPARSE) == 0  # merged on chip
+    assert hs.hs_workspace_size(p, hs.HS_WS_DECODE_FULL) > 0
     with pytest.raises(hs.HsError):
         hs.hs_workspace_size(_p(hq=30), hs.HS_WS_FULL)

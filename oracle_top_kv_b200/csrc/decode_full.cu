@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
     if (L >= 1 && L <= p.t_kv && first < L) {
         const int last = min(L - 1, first + kDecodeKeys - 1);
         const uint32_t sbase = base + warp * WarpSmem<D>::kBytes;
-        TmaRing ring{base + kDecodeWarps * WarpSmem<D>::kBytes + 16u * warp, {0u, 0u}};
+        TmaRing ring{base + kDecodeWarps * WarpSmem<D>::kBytes + 16u * warp, 0u};
         if (lane == 0) {
             tc::mbar_init(ring.bar, 1);
             tc::mbar_init(ring.bar + 8, 1);

@@ -12,8 +12,10 @@
 //
 // Kernels
 //   sparse_simt_kernel  fp32 / any shape: one CTA per row, one warp per head.
-//   sparse_mma_kernel   bf16: one warp per (row, group); the group's heads are
-//                       the 16 MMA rows, so each gathered row is read once.
+//   sparse_mma_kernel   bf16: one warp per (row, group), so each gathered row
+//                       is read once for all the group's heads; the heads are
+//                       the 16 MMA rows (groups of 9-16 heads), or the keys
+//                       are (S^T = K Q^T, groups of at most 8 heads).
 //   decode_sparse_*     bf16 decode: the selected rows of one (sequence, group)
 //                       split across warps, then an exact log-sum-exp merge.
 #include <atomic>
@@ -210,14 +212,16 @@ __device__ __forceinline__ void store_rows(const AttnState<D>& st, __nv_bfloat16
     }
 }
 
-// Dynamic shared memory: per warp a 2-stage K/V ring, then per warp 2 mbarriers.
-template <int D>
+// Dynamic shared memory: per warp an S-stage K/V ring, then per warp S mbarriers.
+template <int D, int W, int S>
 constexpr size_t sparse_smem_bytes() {
-    return (size_t)kSparseWarps * WarpSmem<D>::kBytes + kSparseWarps * 16 + 1024;
+    return (size_t)W * WarpSmem<D, S>::kBytes + (size_t)W * 8 * S + 1024;
 }
 
-template <int D>
-__global__ void __launch_bounds__(kSparseWarps * 32)
+// W warps per CTA, each attending one (row, group) task through an S-stage
+// ring.  kT: keys-as-rows form (groups of at most 8 heads); else heads as rows.
+template <int D, bool kT, int W, int S>
+__global__ void __launch_bounds__(W * 32)
     sparse_mma_kernel(const __grid_constant__ CUtensorMap tm_kf,
                       const __grid_constant__ CUtensorMap tm_vf,
                       const __grid_constant__ CUtensorMap tm_kl,
@@ -231,7 +235,7 @@ __global__ void __launch_bounds__(kSparseWarps * 32)
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long task = (long long)blockIdx.x * kSparseWarps + warp;
+    const long long task = (long long)blockIdx.x * W + warp;
     const long long n_tasks = (long long)p.batch * p.hkv * p.t_q;
     if (task >= n_tasks) return;
     const int j = (int)(task % p.t_q);
@@ -239,36 +243,61 @@ __global__ void __launch_bounds__(kSparseWarps * 32)
     const int b = (int)(task / ((long long)p.t_q * p.hkv));
     const int g = p.group;
     const int t = p.q_offset + j;
-    const uint32_t sbase = base + warp * WarpSmem<D>::kBytes;
-    TmaRing ring{base + kSparseWarps * WarpSmem<D>::kBytes + 16u * warp, {0u, 0u}};
+    const uint32_t sbase = base + warp * WarpSmem<D, S>::kBytes;
+    TmaRing ring{base + W * WarpSmem<D, S>::kBytes + 8u * S * warp, 0u};
     if (lane == 0) {
-        tc::mbar_init(ring.bar, 1);
-        tc::mbar_init(ring.bar + 8, 1);
+#pragma unroll
+        for (int i = 0; i < S; ++i) tc::mbar_init(ring.bar + 8u * i, 1);
         tc::fence_mbar_init();
     }
     __syncwarp();
 
     const size_t head_stride = (size_t)p.t_q * D;
     const size_t q0 = (((size_t)b * p.hq + u * g) * p.t_q + j);  // row of head u*g
-    uint32_t qf[D / 16][4];
-    load_q_frags<D>(qf, q + q0 * D, head_stride, g);
-
     const int unit = b * p.hkv + u;
     const size_t row = (size_t)unit * p.t_q + j;
     const size_t kvoff = (size_t)unit * p.t_kv * D;
     const int c = clamp_count(cnt[row], p.ksel);
     const int n_rows = p.mode == 0 ? c * p.block_size : c;
+    if constexpr (kT) {
+        uint32_t qb[D / 16][2];
+        load_qt_frags<D>(qb, q + q0 * D, head_stride, g);
+        AttnStateT<D> st;
+        st.init();
+        if (p.mode == 0 && p.block_size % kChunk == 0) {
+            BlockChunks src{idx + row * p.ksel, p.block_size, t};
+            attend_rows_tma_t<D, S>(st, qb, &tm_kf, &tm_vf, unit, c * (p.block_size / kChunk),
+                                    src, sbase, ring, p.scale_log2);
+        } else {
+            GatherKeys keys{idx + row * p.ksel, n_rows, p.block_size, t, p.mode};
+            attend_rows_t<D, S>(st, qb, kf + kvoff, vf + kvoff, (n_rows + kChunk - 1) / kChunk,
+                                keys, sbase, p.scale_log2);
+        }
+        store_rows_t<D>(st, og + q0 * D, head_stride, lseg + q0, p.t_q, g);
+        if (has_local) {
+            const int first = max(0, t - p.window + 1);
+            AttnStateT<D> sl;
+            sl.init();
+            const ContiguousKeys win{first, t};
+            attend_rows_tma_t<D, S>(sl, qb, &tm_kl, &tm_vl, unit, win.n_chunks(), win, sbase,
+                                    ring, p.scale_log2);
+            store_rows_t<D>(sl, ol + q0 * D, head_stride, lsel + q0, p.t_q, g);
+        }
+        return;
+    }
+    uint32_t qf[D / 16][4];
+    load_q_frags<D>(qf, q + q0 * D, head_stride, g);
 
     AttnState<D> st;
     st.init();
     if (p.mode == 0 && p.block_size % kChunk == 0) {
         BlockChunks src{idx + row * p.ksel, p.block_size, t};
-        attend_rows_tma<D>(st, qf, &tm_kf, &tm_vf, unit, c * (p.block_size / kChunk), src, sbase,
-                           ring, p.scale_log2, NoHook{});
+        attend_rows_tma<D, S>(st, qf, &tm_kf, &tm_vf, unit, c * (p.block_size / kChunk), src,
+                              sbase, ring, p.scale_log2, NoHook{});
     } else {
         GatherKeys keys{idx + row * p.ksel, n_rows, p.block_size, t, p.mode};
-        attend_rows<D>(st, qf, kf + kvoff, vf + kvoff, (n_rows + kChunk - 1) / kChunk, keys,
-                       sbase, p.scale_log2, NoHook{});
+        attend_rows<D, S>(st, qf, kf + kvoff, vf + kvoff, (n_rows + kChunk - 1) / kChunk, keys,
+                          sbase, p.scale_log2, NoHook{});
     }
     store_rows<D>(st, og + q0 * D, head_stride, lseg + q0, p.t_q, g);
     if (has_local) {
@@ -276,10 +305,31 @@ __global__ void __launch_bounds__(kSparseWarps * 32)
         AttnState<D> sl;
         sl.init();
         const ContiguousKeys win{first, t};
-        attend_rows_tma<D>(sl, qf, &tm_kl, &tm_vl, unit, win.n_chunks(), win, sbase, ring,
-                           p.scale_log2, NoHook{});
+        attend_rows_tma<D, S>(sl, qf, &tm_kl, &tm_vl, unit, win.n_chunks(), win, sbase, ring,
+                              p.scale_log2, NoHook{});
         store_rows<D>(sl, ol + q0 * D, head_stride, lsel + q0, p.t_q, g);
     }
+}
+
+template <int D, bool kT, int W, int S>
+static cudaError_t launch_sparse_cfg(const KParams& p, const CUtensorMap& mk,
+                                     const CUtensorMap& mv, const CUtensorMap& mkl,
+                                     const CUtensorMap& mvl, const void* q, const void* kf,
+                                     const void* vf, const int32_t* idx, const int32_t* cnt,
+                                     bool has_local, void* og, float* lseg, void* ol, float* lsel,
+                                     cudaStream_t st) {
+    constexpr size_t smem = sparse_smem_bytes<D, W, S>();
+    auto kern = sparse_mma_kernel<D, kT, W, S>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const long long n_tasks = (long long)p.batch * p.hkv * p.t_q;
+    const unsigned grid = (unsigned)((n_tasks + W - 1) / W);
+    kern<<<grid, W * 32, smem, st>>>(mk, mv, mkl, mvl, p, (const __nv_bfloat16*)q,
+                                     (const __nv_bfloat16*)kf, (const __nv_bfloat16*)vf, idx, cnt,
+                                     has_local ? 1 : 0, (__nv_bfloat16*)og, lseg,
+                                     (__nv_bfloat16*)ol, lsel);
+    return cudaGetLastError();
 }
 
 template <int D>
@@ -287,7 +337,6 @@ static cudaError_t launch_sparse_mma_t(const KParams& p, const void* q, const vo
                                        const void* vf, const int32_t* idx, const int32_t* cnt,
                                        const void* kl, const void* vl, void* og, float* lseg,
                                        void* ol, float* lsel, cudaStream_t st) {
-    const size_t smem = sparse_smem_bytes<D>();
     CUtensorMap mk, mv, mkl, mvl;
     const long long units = (long long)p.batch * p.hkv;
     if (!tc::encode_rows(&mk, kf, D, p.t_kv, units, kChunk) ||
@@ -301,17 +350,14 @@ static cudaError_t launch_sparse_mma_t(const KParams& p, const void* q, const vo
         mkl = mk;
         mvl = mv;
     }
-    auto kern = sparse_mma_kernel<D>;
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    const long long n_tasks = (long long)p.batch * p.hkv * p.t_q;
-    const unsigned grid = (unsigned)((n_tasks + kSparseWarps - 1) / kSparseWarps);
-    kern<<<grid, kSparseWarps * 32, smem, st>>>(
-        mk, mv, mkl, mvl, p, (const __nv_bfloat16*)q, (const __nv_bfloat16*)kf,
-        (const __nv_bfloat16*)vf, idx, cnt, kl ? 1 : 0, (__nv_bfloat16*)og, lseg,
-        (__nv_bfloat16*)ol, lsel);
-    return cudaGetLastError();
+    // 6 warps x 2 stages fills the shared memory (192 KB at d = 128); deeper
+    // rings with fewer warps were slower: the warps' own instruction latency,
+    // not the load lookahead, bounds the rate.
+    if (p.group <= 8)
+        return launch_sparse_cfg<D, true, kSparseWarps, 2>(p, mk, mv, mkl, mvl, q, kf, vf, idx,
+                                                           cnt, kl, og, lseg, ol, lsel, st);
+    return launch_sparse_cfg<D, false, kSparseWarps, 2>(p, mk, mv, mkl, mvl, q, kf, vf, idx, cnt,
+                                                        kl, og, lseg, ol, lsel, st);
 }
 
 cudaError_t launch_sparse_mma(const KParams& p, const void* q, const void* kf, const void* vf,

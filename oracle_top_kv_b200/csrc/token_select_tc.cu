@@ -15,9 +15,11 @@
 // the fp32 lse.  Each position keeps an exact streaming top-(k-w) buffer in
 // shared memory (admission threshold = the k-w-th best key after each cut).
 //
-// Warps: 0 TMA (Q once, K tiles of 128 keys through a 3-stage ring), 1 TMEM +
-// MMA issuer (S^T double-buffered in TMEM), 2..9 scorers in two sets of four
-// (each set covers the 128 TMEM lanes = keys, and 4 of the 8 positions).
+// Warps: 0 TMA (Q once, K tiles of 128 keys through a 2-stage ring), 1 TMEM +
+// MMA issuer (S^T in 4 TMEM buffers), 2..9 scorers in two sets of four (each
+// set covers the 128 TMEM lanes = keys, and 4 of the 8 positions).  The sets
+// only meet at the TMEM buffers, so one set's buffer cut does not stall the
+// other for up to 3 tiles.
 #include "hs_common.cuh"
 #include "hs_kernels.cuh"
 #include "tc_ptx.cuh"
@@ -31,21 +33,28 @@ constexpr int kG = 16;          // heads per group handled here
 constexpr int kPos = 8;         // positions per CTA
 constexpr int kKeys = 128;      // keys per K tile (= MMA M)
 constexpr int kHd = 128;
-constexpr int kStages = 3;
+constexpr int kStages = 2;       // K ring (the MMA is far ahead of the scorers)
+constexpr int kSBufs = 4;        // S^T buffers in TMEM: the two scorer sets may drift 3 tiles
 constexpr int kThreads = 64 + 256;
 constexpr int kMaxRanked = 1024;            // k - w handled here
-constexpr int kCap = kMaxRanked + 2 * kKeys; // per-position buffer entries
+// Per-position buffer entries: the k - w kept, one tile of admissions, and
+// 6 tiles' worth of headroom between cuts (what shared memory holds).
+constexpr int kCap = kMaxRanked + 7 * kKeys;
+constexpr int kBitmapKeys = 65536;  // finalize by id bitmap (8 KB per position) below this
 
 constexpr uint32_t kQOff = 0;                         // 2 x 16 KB
 constexpr uint32_t kKOff = 32768;                     // kStages x 32 KB (sort scratch later)
 constexpr uint32_t kBufOff = kKOff + kStages * 32768; // kPos x kCap x 8
 constexpr uint32_t kHistOff = kBufOff + kPos * kCap * 8;   // 8 warps x 1 KB
 constexpr uint32_t kBarOff = kHistOff + 8 * 1024;
-enum { BQ = 0, BKF = 1, BKE = BKF + kStages, BSF = BKE + kStages, BSE = BSF + 2, BDRAIN = BSE + 2,
-       BCOUNT = BDRAIN + 1 };
+enum { BQ = 0, BKF = 1, BKE = BKF + kStages, BSF = BKE + kStages, BSE = BSF + kSBufs,
+       BDRAIN = BSE + kSBufs, BCOUNT = BDRAIN + 1 };
 constexpr uint32_t kMiscOff = kBarOff + BCOUNT * 8;  // tmem(4) abort(4) cnt[8](32) thresh[8](64)
 constexpr uint32_t kSmemBytes = kMiscOff + 8 + 32 + 64 + 1024;
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemCols = 128 * kSBufs;
+static_assert(kStages * 32768 >= 8 * kMaxRanked * 8, "sort scratch fits in the K ring");
+static_assert(kStages * 32768 >= 8 * (kBitmapKeys / 8), "id bitmaps fit in the K ring");
+static_assert(kSmemBytes <= 232448, "shared memory");
 
 struct Args {
     KParams p;
@@ -92,7 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         mbar_init(bar(BQ), 1);
         for (int i = 0; i < kStages; ++i) { mbar_init(bar(BKF + i), 1); mbar_init(bar(BKE + i), 1); }
-        for (int i = 0; i < 2; ++i) { mbar_init(bar(BSF + i), 1); mbar_init(bar(BSE + i), 8); }
+        for (int i = 0; i < kSBufs; ++i) { mbar_init(bar(BSF + i), 1); mbar_init(bar(BSE + i), 8); }
         mbar_init(bar(BDRAIN), 1);
         *abort_flag = 0;
         for (int i = 0; i < kPos; ++i) { s_cnt[i] = 0; s_th[i] = 0ull; }
@@ -135,9 +144,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = mbar_wait(bar(BQ), 0, abort_flag);
             tc_fence_after();
             for (int j = 0; ok && j < nt; ++j) {
-                const int st = j % kStages, s = j & 1;
+                const int st = j % kStages, s = j % kSBufs;
                 if (!mbar_wait(bar(BKF + st), (j / kStages) & 1, abort_flag)) break;
-                if (j >= 2 && !mbar_wait(bar(BSE + s), ((j >> 1) - 1) & 1, abort_flag)) break;
+                if (j >= kSBufs && !mbar_wait(bar(BSE + s), ((j / kSBufs) - 1) & 1, abort_flag))
+                    break;
                 tc_fence_after();
                 const uint32_t kb = base + kKOff + st * 32768;
 #pragma unroll
@@ -160,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16) + set * 64;
         const float sl2 = p.scale_log2;
         // this thread's 4 positions: lse (log2 domain) of their 16 heads
-        float lse2[4][kG];
+        float nlse2[4][kG];  // -lse2
         int tpos[4];
         bool live[4], all_sel[4];
 #pragma unroll
@@ -171,8 +181,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             all_sel[i] = tpos[i] + 1 <= p.k;
 #pragma unroll
             for (int hh = 0; hh < kG; ++hh)
-                lse2[i][hh] = live[i] ? a.lse[((size_t)b * p.hq + u * kG + hh) * p.t_q + r] * kLog2e
-                                      : 0.f;
+                nlse2[i][hh] = live[i] ? -a.lse[((size_t)b * p.hq + u * kG + hh) * p.t_q + r] * kLog2e
+                                       : 0.f;
         }
         uint64_t* bufs = reinterpret_cast<uint64_t*>(gb + kBufOff);
         uint32_t* hist = reinterpret_cast<uint32_t*>(gb + kHistOff + wid * 1024);
@@ -181,8 +191,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Every warp runs every iteration (the set meets at named barriers);
         // after an abort the waits fail at once and the work is skipped.
         for (int j = 0; j < nt; ++j) {
-            const int s = j & 1;
-            bool got = ok && mbar_wait(bar(BSF + s), (j >> 1) & 1, abort_flag);
+            const int s = j % kSBufs;
+            bool got = ok && mbar_wait(bar(BSF + s), (j / kSBufs) & 1, abort_flag);
             got = __all_sync(0xffffffffu, got);
             if (!got) ok = false;
             if (got) {
@@ -201,10 +211,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 4; ++i) {
                 const uint32_t* rr = i < 2 ? r0 : r1;
                 const int c0 = (i & 1) * 16;
-                float sc = -INFINITY;
+                // a2 - lse2 of the 16 heads (packed FMA), then their max (3-input max)
+                float v[kG];
 #pragma unroll
-                for (int hh = 0; hh < kG; ++hh)
-                    sc = fmaxf(sc, fmaf(__uint_as_float(rr[c0 + hh]), sl2, -lse2[i][hh]));
+                for (int hh = 0; hh < kG; hh += 2) {
+                    const float2 r2 = ffma2(make_float2(__uint_as_float(rr[c0 + hh]),
+                                                        __uint_as_float(rr[c0 + hh + 1])),
+                                            make_float2(sl2, sl2),
+                                            make_float2(nlse2[i][hh], nlse2[i][hh + 1]));
+                    v[hh] = r2.x;
+                    v[hh + 1] = r2.y;
+                }
+                const float sc = fmaxf(max3f(max3f(v[0], v[1], v[2]), max3f(v[3], v[4], v[5]),
+                                             max3f(v[6], v[7], v[8])),
+                                       max3f(max3f(v[9], v[10], v[11]),
+                                             max3f(v[12], v[13], v[14]), v[15]));
                 const int t = tpos[i];
                 const bool visible = live[i] && key <= t;
                 const int pos = set * 4 + i;
@@ -269,15 +290,48 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int n = Kc > 0 ? s_cnt[pos] : 0;
                 if (n > Kc) { warp_cut_to_k(buf, n, Kc, hist); n = Kc; }
                 __syncwarp();
-                const int sort_n = next_pow2(Kc > 0 ? Kc : 1);
-                uint64_t* sb = reinterpret_cast<uint64_t*>(gb + kKOff) + (size_t)wid * kMaxRanked;
-                for (int x = lane; x < sort_n; x += 32)
-                    sb[x] = x < n ? (((uint64_t)sel_key_id(buf[x]) << 32) | (buf[x] >> 32)) : ~0ull;
-                __syncwarp();
-                warp_bitonic_sort(sb, sort_n);
-                for (int x = lane; x < n; x += 32) {
-                    irow[x] = (int32_t)(sb[x] >> 32);
-                    if (srow) srow[x] = exp2f(order_float((uint32_t)(sb[x] & 0xffffffffu)));
+                if (!srow && t < kBitmapKeys) {
+                    // ascending ids without sorting: mark the winners in a bitmap
+                    // over 0..t, then read the set bits out in word order
+                    uint32_t* bm = reinterpret_cast<uint32_t*>(gb + kKOff) + (size_t)wid * (kBitmapKeys / 32);
+                    const int words = (t >> 5) + 1;
+                    const int per = (words + 31) >> 5;  // words per lane, consecutive
+                    for (int x = lane; x < per * 32; x += 32) bm[x] = 0u;
+                    __syncwarp();
+                    for (int x = lane; x < n; x += 32) {
+                        const uint32_t id = sel_key_id(buf[x]);
+                        atomicOr(&bm[id >> 5], 1u << (id & 31));
+                    }
+                    __syncwarp();
+                    int cnt_l = 0;
+                    for (int x = 0; x < per; ++x) cnt_l += __popc(bm[lane * per + x]);
+                    int incl = cnt_l;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                        if (lane >= o) incl += y;
+                    }
+                    int at = incl - cnt_l;
+                    for (int x = 0; x < per; ++x) {
+                        const int wi = lane * per + x;
+                        uint32_t m = bm[wi];
+                        while (m) {
+                            const int bit = __ffs(m) - 1;
+                            irow[at++] = wi * 32 + bit;
+                            m &= m - 1u;
+                        }
+                    }
+                } else {
+                    const int sort_n = next_pow2(Kc > 0 ? Kc : 1);
+                    uint64_t* sb = reinterpret_cast<uint64_t*>(gb + kKOff) + (size_t)wid * kMaxRanked;
+                    for (int x = lane; x < sort_n; x += 32)
+                        sb[x] = x < n ? (((uint64_t)sel_key_id(buf[x]) << 32) | (buf[x] >> 32)) : ~0ull;
+                    __syncwarp();
+                    warp_bitonic_sort(sb, sort_n);
+                    for (int x = lane; x < n; x += 32) {
+                        irow[x] = (int32_t)(sb[x] >> 32);
+                        if (srow) srow[x] = exp2f(order_float((uint32_t)(sb[x] & 0xffffffffu)));
+                    }
                 }
                 const int lo = t - p.window + 1;
                 for (int x = lane; x <= t - lo; x += 32) irow[n + x] = lo + x;

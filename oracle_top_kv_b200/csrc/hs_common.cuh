@@ -235,6 +235,64 @@ __device__ __forceinline__ uint64_t warp_cut_to_k(uint64_t* buf, int n, int K, u
     return kth;
 }
 
+// Ascending bitonic sort of 64 values held two per lane (a = element lane,
+// b = element lane + 32), in registers.
+__device__ __forceinline__ void warp_sort64(uint64_t& a, uint64_t& b) {
+    const int lane = threadIdx.x & 31;
+    for (int size = 2; size <= 64; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            if (stride == 32) {  // a <-> b of the same lane
+                const bool up = true;  // size == 64
+                if ((a > b) == up) { const uint64_t t = a; a = b; b = t; }
+                continue;
+            }
+            // element e = lane (+32 for b); partner e ^ stride is in the same half
+            const uint64_t pa = shfl_xor_u64(a, stride), pb = shfl_xor_u64(b, stride);
+            const bool lower = (lane & stride) == 0;
+            const bool up_a = (lane & size) == 0, up_b = ((lane + 32) & size) == 0;
+            // the lower element keeps min when ascending, max when descending
+            a = (lower == up_a) ? (a < pa ? a : pa) : (a > pa ? a : pa);
+            b = (lower == up_b) ? (b < pb ? b : pb) : (b > pb ? b : pb);
+        }
+    }
+}
+
+// Cut a streaming buffer by a sampled quantile: sort 64 evenly spaced keys,
+// take the one a little below the K-th best's expected sample rank as the
+// threshold, count the keys at or above it and, if that keeps at least K
+// (so the K best are all kept) and frees at least `min_free` slots, compact;
+// otherwise move the threshold down the sample and count again, and fall
+// back to the exact cut when the sample runs out.  No shared atomics, and
+// outlying scores do not bunch the rest up.  Returns the surviving count;
+// *thresh gets an admission threshold (a key must exceed it) that is at most
+// the K-th best key.  Requires n > K.
+__device__ __forceinline__ int warp_cut_sampled(uint64_t* buf, int n, int K, int min_free,
+                                                uint32_t* hist, uint64_t* thresh) {
+    const int lane = threadIdx.x & 31;
+    uint64_t a = buf[(int)(((long long)(2 * lane) * n) >> 6)];
+    uint64_t b = buf[(int)(((long long)(2 * lane + 1) * n) >> 6)];
+    warp_sort64(a, b);  // ascending: element e = a of lane e, b of lane e - 32
+    // expected descending sample rank of the K-th best, plus 3 samples of slack
+    int q = (int)(((long long)K * 64 + n - 1) / n) + 3;
+    for (; q < 64; q += 4) {
+        const int e = 63 - q;  // ascending index
+        const uint64_t thr = __shfl_sync(0xffffffffu, (uint32_t)(e < 32 ? a : b), e & 31) |
+                             ((uint64_t)__shfl_sync(0xffffffffu, (uint32_t)((e < 32 ? a : b) >> 32),
+                                                    e & 31) << 32);
+        int c = 0;
+        for (int i = lane; i < n; i += 32) c += buf[i] >= thr;
+        c = __reduce_add_sync(0xffffffffu, c);
+        if (c < K) continue;            // too high: a top-K key would go
+        if (n - c < min_free) break;    // keeps too much: exact cut instead
+        const int m = warp_keep_at_least(buf, n, thr);
+        *thresh = thr ? thr - 1ull : 0ull;
+        return m;
+    }
+    const uint64_t kth = warp_cut_to_k(buf, n, K, hist);
+    *thresh = kth;
+    return K;
+}
+
 // In-place ascending bitonic sort of n_pow2 values by one warp.
 template <typename U>
 __device__ __forceinline__ void warp_bitonic_sort(U* a, int n_pow2) {

@@ -266,8 +266,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int pos = set * 4 + quad;
                 const int n = s_cnt[pos];
                 if (n > kCap - kKeys) {
-                    const uint64_t th = warp_cut_to_k(bufs + (size_t)pos * kCap, n, Kc, hist);
-                    if (lane == 0) { s_th[pos] = th; s_cnt[pos] = Kc; }
+                    uint64_t th;
+                    const int m = warp_cut_sampled(bufs + (size_t)pos * kCap, n, Kc,
+                                                   (kCap - kKeys - Kc) / 2, hist, &th);
+                    if (lane == 0) {
+                        s_th[pos] = th > s_th[pos] ? th : s_th[pos];
+                        s_cnt[pos] = m;
+                    }
                 }
             }
             asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");

@@ -246,9 +246,22 @@ __device__ __forceinline__ void gather_pipeline(const __nv_bfloat16* kbase,
                                                 const Src& src, uint32_t smem_base,
                                                 Consume&& consume) {
     static_assert(!Src::kContig, "gathered rows");
-    static_assert(S >= 2 && S <= 4, "ring depth");
+    static_assert(S >= 1 && S <= 4, "ring depth");
     const int lane = threadIdx.x & 31;
-    uint32_t mq[S - 1];  // masks of chunks c .. c+S-2
+    if constexpr (S == 1) {  // no lookahead: load, wait, compute
+        for (int c = 0; c < n_chunks; ++c) {
+            const int key = src.key(c * kChunk + lane);
+            const uint32_t mask = __ballot_sync(0xffffffffu, key >= 0);
+            load_chunk<D>(smem_base, kbase, vbase, key);
+            cp_async_commit();
+            cp_async_wait<0>();
+            __syncwarp();
+            consume(c, smem_base, mask, 0);
+            __syncwarp();
+        }
+        return;
+    }
+    uint32_t mq[S > 1 ? S - 1 : 1];  // masks of chunks c .. c+S-2
     auto issue = [&](int c) -> uint32_t {
         const uint32_t sb = smem_base + (uint32_t)(c % S) * WarpSmem<D, S>::kStageBytes;
         const int key = src.key(c * kChunk + lane);
@@ -296,13 +309,13 @@ __device__ __forceinline__ bool tma_pipeline(const CUtensorMap* tk, const CUtens
                                              uint32_t smem_base, TmaRing& ring,
                                              Consume&& consume) {
     static_assert(Src::kContig, "consecutive keys");
-    static_assert(S >= 2 && S <= 4, "ring depth");
+    static_assert(S >= 1 && S <= 4, "ring depth");
     constexpr uint32_t kHalf = kChunk * 128;          // one d-half box
     constexpr uint32_t kTx = 2 * (D / 64) * kHalf;    // K and V, all halves
     const int lane = threadIdx.x & 31;
     const uint32_t k0 = ring.next;
-    uint32_t mq[S - 1];  // masks and first keys of chunks c .. c+S-2
-    int kq[S - 1];
+    uint32_t mq[S > 1 ? S - 1 : 1];  // masks and first keys of chunks c .. c+S-2
+    int kq[S > 1 ? S - 1 : 1];
     int dummy = 0;
     volatile int* no_abort = &dummy;
     auto issue = [&](int c, int& key0) -> uint32_t {
@@ -326,6 +339,7 @@ __device__ __forceinline__ bool tma_pipeline(const CUtensorMap* tk, const CUtens
         kq[i] = 0;
         mq[i] = i < n_chunks ? issue(i, kq[i]) : 0u;
     }
+    if constexpr (S == 1) { mq[0] = 0u; kq[0] = 0; }
     int issued = min(n_chunks, S - 1), failed = -1;
     for (int c = 0; c < n_chunks; ++c) {
         int knext = 0;
@@ -334,15 +348,18 @@ __device__ __forceinline__ bool tma_pipeline(const CUtensorMap* tk, const CUtens
             mnext = issue(c + S - 1, knext);
             issued = c + S;
         }
+        if constexpr (S == 1) { mq[0] = mnext; kq[0] = knext; }
         const uint32_t k = k0 + (uint32_t)c, st = k % S;
         // poll: a suspended warp wakes up late on this short critical path
         const bool got = tc::mbar_wait(ring.bar + 8u * st, (k / S) & 1u, no_abort, false);
         if (!__all_sync(0xffffffffu, got)) { failed = c; break; }
         consume(c, smem_base + st * WarpSmem<D, S>::kStageBytes, mq[0], kq[0]);
+        if constexpr (S > 1) {
 #pragma unroll
-        for (int i = 0; i < S - 2; ++i) { mq[i] = mq[i + 1]; kq[i] = kq[i + 1]; }
-        mq[S - 2] = mnext;
-        kq[S - 2] = knext;
+            for (int i = 0; i < S - 2; ++i) { mq[i] = mq[i + 1]; kq[i] = kq[i + 1]; }
+            mq[S - 2] = mnext;
+            kq[S - 2] = knext;
+        }
         __syncwarp();  // the stage is refilled by the next iteration
     }
     if (failed >= 0) {

@@ -187,7 +187,7 @@ cudaError_t launch_sparse_simt(const KParams& p, int dtype, const void* q, const
 }
 
 // ------------------------------------------------------------ tensor-core path
-constexpr int kSparseWarps = 6;
+constexpr int kSparseWarps = 6;  // decode kernels: warps per CTA, 2-stage rings
 
 // Normalise and store rows < g of a finished warp state.
 template <int D>
@@ -350,14 +350,18 @@ static cudaError_t launch_sparse_mma_t(const KParams& p, const void* q, const vo
         mkl = mk;
         mvl = mv;
     }
-    // 6 warps x 2 stages fills the shared memory (192 KB at d = 128); deeper
-    // rings with fewer warps were slower: the warps' own instruction latency,
-    // not the load lookahead, bounds the rate.
+    // The rate follows the number of resident warps: each warp's own chain of
+    // dependent MMA, shuffle and exp2 steps is long, and other warps hide it
+    // better than a deeper per-warp load lookahead does.  So one stage per
+    // warp and as many warps as shared memory (16 KB each at d = 128) and
+    // registers allow: 14 for the keys-as-rows form (126 registers), 12 for
+    // the heads-as-rows form (168).  At d = 128 these beat 6 warps x 2 stages
+    // by 1.6x and 1.4x; 4 x 3 and 3 x 4 were slower still.
     if (p.group <= 8)
-        return launch_sparse_cfg<D, true, kSparseWarps, 2>(p, mk, mv, mkl, mvl, q, kf, vf, idx,
-                                                           cnt, kl, og, lseg, ol, lsel, st);
-    return launch_sparse_cfg<D, false, kSparseWarps, 2>(p, mk, mv, mkl, mvl, q, kf, vf, idx, cnt,
-                                                        kl, og, lseg, ol, lsel, st);
+        return launch_sparse_cfg<D, true, 14, 1>(p, mk, mv, mkl, mvl, q, kf, vf, idx, cnt, kl,
+                                                 og, lseg, ol, lsel, st);
+    return launch_sparse_cfg<D, false, 12, 1>(p, mk, mv, mkl, mvl, q, kf, vf, idx, cnt, kl, og,
+                                              lseg, ol, lsel, st);
 }
 
 cudaError_t launch_sparse_mma(const KParams& p, const void* q, const void* kf, const void* vf,

@@ -98,6 +98,33 @@ __device__ uint64_t cta_kth_largest(Get get, int n, int k, CtaSelectSmem& sh) {
     return lo;
 }
 
+// Exclusive prefix sum of one int per thread over the CTA (thread order);
+// `scratch` is one shared int per warp plus one.  All threads call.
+__device__ __forceinline__ int cta_exclusive_sum(int v, int* scratch) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    __syncthreads();
+    if (lane == 31) scratch[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < nw ? scratch[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += y;
+        }
+        if (lane < nw) scratch[lane] = wi - w;  // exclusive warp offsets
+    }
+    __syncthreads();
+    return scratch[warp] + incl - v;
+}
+
 // Ascending bitonic sort of a[0 .. n) in shared memory, n a power of two.
 template <typename U>
 __device__ void cta_bitonic_sort(U* a, int n) {

@@ -37,6 +37,8 @@ constexpr int kSelectThreads = 512;
 constexpr int kSelSlice = 16384;       // most ranked keys one selector CTA stages
 constexpr int kSelMaxRanked = 1024;    // k - w handled by the split selector
 constexpr int kMergeCap = 8192;        // candidate keys the merge holds at once
+// The merge writes ids through a bitmap over 0..t below this (in its buffer).
+constexpr int kBitmapKeys = (kMergeCap - kSelMaxRanked) * 64;
 
 // CTAs per (sequence, group) in the split selector: slices of at most
 // kSelSlice keys, and enough CTAs for about two per SM of a 148-SM part
@@ -241,7 +243,7 @@ __device__ __forceinline__ float group_score(const float* lg_row, const float* l
 // the slice's (k-w)-th largest selection key with a CTA-wide bucket select,
 // and writes the slice's top-(k-w) keys out unsorted.  The group's top-(k-w)
 // is contained in the union of the slices' top-(k-w).
-__global__ void __launch_bounds__(kSelectThreads)
+__global__ void __launch_bounds__(kSelectThreads, 2)
     decode_select_split_kernel(KParams p, const int32_t* __restrict__ seq_len, DecodeWs ws) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     __shared__ CtaSelectSmem cs;
@@ -265,9 +267,45 @@ __global__ void __launch_bounds__(kSelectThreads)
     if (threadIdx.x < 16) s_lse2[threadIdx.x] = threadIdx.x < g ? ws.lse2[b * p.hq + u * g + threadIdx.x] : 0.f;
     __syncthreads();
     const float* lg = ws.logits + (size_t)unit * p.t_kv * 16;
-#pragma unroll 4
-    for (int i = threadIdx.x; i < n; i += blockDim.x)
-        bits[i] = float_order(group_score(lg + (size_t)(i0 + i) * 16, s_lse2, g));
+    if (g == 16) {
+        // two keys per thread per round, all 8 loads issued before any use
+        // (the logits are read once: streaming loads)
+        float nl[16];
+#pragma unroll
+        for (int h = 0; h < 16; ++h) nl[h] = -s_lse2[h];
+        const float4* l4 = reinterpret_cast<const float4*>(lg + (size_t)i0 * 16);
+        constexpr int U = 2;
+        for (int base = threadIdx.x; base < n; base += U * blockDim.x) {
+            float4 r[U][4];
+#pragma unroll
+            for (int k = 0; k < U; ++k) {
+                const int i = base + k * blockDim.x;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4)
+                    r[k][q4] = i < n ? __ldcs(l4 + (size_t)i * 4 + q4) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int k = 0; k < U; ++k) {
+                const int i = base + k * blockDim.x;
+                float v[16];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    v[4 * q4] = r[k][q4].x + nl[4 * q4];
+                    v[4 * q4 + 1] = r[k][q4].y + nl[4 * q4 + 1];
+                    v[4 * q4 + 2] = r[k][q4].z + nl[4 * q4 + 2];
+                    v[4 * q4 + 3] = r[k][q4].w + nl[4 * q4 + 3];
+                }
+                const float sc = fmaxf(
+                    tc::max3f(tc::max3f(v[0], v[1], v[2]), tc::max3f(v[3], v[4], v[5]),
+                              tc::max3f(v[6], v[7], v[8])),
+                    tc::max3f(tc::max3f(v[9], v[10], v[11]), tc::max3f(v[12], v[13], v[14]), v[15]));
+                if (i < n) bits[i] = float_order(sc);
+            }
+        }
+    } else {
+        for (int i = threadIdx.x; i < n; i += blockDim.x)
+            bits[i] = float_order(group_score(lg + (size_t)(i0 + i) * 16, s_lse2, g));
+    }
     __syncthreads();
     auto key = [&](int i) -> uint64_t {
         return ((uint64_t)bits[i] << 32) | (uint64_t)(0xffffffffu - (uint32_t)(i0 + i));
@@ -314,6 +352,7 @@ __global__ void __launch_bounds__(kSelectThreads)
     __shared__ CtaSelectSmem cs;
     __shared__ float s_lse2[16];
     __shared__ int s_n;
+    __shared__ int s_scan[33];
     const int unit = blockIdx.x;
     const int u = unit % p.hkv, b = unit / p.hkv;
     const int g = p.group;
@@ -360,14 +399,42 @@ __global__ void __launch_bounds__(kSelectThreads)
         }
         if (n > Kc) n = cta_cut(buf, n, Kc, tmp, cs, &s_n);
     }
-    const int sort_n = next_pow2(Kc > 0 ? Kc : 1);
-    for (int x = threadIdx.x; x < sort_n; x += blockDim.x)
-        tmp[x] = x < n ? (((uint64_t)sel_key_id(buf[x]) << 32) | (buf[x] >> 32)) : ~0ull;
-    __syncthreads();
-    cta_bitonic_sort(tmp, sort_n);
-    for (int x = threadIdx.x; x < n; x += blockDim.x) {
-        irow[x] = (int32_t)(tmp[x] >> 32);
-        if (srow) srow[x] = exp2f(order_float((uint32_t)(tmp[x] & 0xffffffffu)));
+    if (!srow && t < kBitmapKeys) {
+        // ascending ids without sorting: mark the winners in a bitmap over
+        // 0..t (in the free part of buf), then each thread reads out a run of
+        // consecutive words at its prefix-sum offset
+        uint32_t* bm = reinterpret_cast<uint32_t*>(buf + kSelMaxRanked);
+        const int words = (t >> 5) + 1;
+        const int per = (words + blockDim.x - 1) / blockDim.x;
+        for (int x = threadIdx.x; x < per * (int)blockDim.x; x += blockDim.x) bm[x] = 0u;
+        __syncthreads();
+        for (int x = threadIdx.x; x < n; x += blockDim.x) {
+            const uint32_t id = sel_key_id(buf[x]);
+            atomicOr(&bm[id >> 5], 1u << (id & 31));
+        }
+        __syncthreads();
+        const int w0 = threadIdx.x * per;
+        int c = 0;
+        for (int x = 0; x < per; ++x) c += __popc(bm[w0 + x]);
+        const int at = cta_exclusive_sum(c, s_scan);
+        int o = at;
+        for (int x = 0; x < per; ++x) {
+            uint32_t m = bm[w0 + x];
+            while (m) {
+                irow[o++] = (w0 + x) * 32 + (__ffs(m) - 1);
+                m &= m - 1u;
+            }
+        }
+    } else {
+        const int sort_n = next_pow2(Kc > 0 ? Kc : 1);
+        for (int x = threadIdx.x; x < sort_n; x += blockDim.x)
+            tmp[x] = x < n ? (((uint64_t)sel_key_id(buf[x]) << 32) | (buf[x] >> 32)) : ~0ull;
+        __syncthreads();
+        cta_bitonic_sort(tmp, sort_n);
+        for (int x = threadIdx.x; x < n; x += blockDim.x) {
+            irow[x] = (int32_t)(tmp[x] >> 32);
+            if (srow) srow[x] = exp2f(order_float((uint32_t)(tmp[x] & 0xffffffffu)));
+        }
     }
     for (int x = threadIdx.x; x <= t - lo; x += blockDim.x) irow[n + x] = lo + x;
     const int n_out = n + (t - lo + 1);

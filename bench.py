@@ -236,8 +236,8 @@ def traffic_for(kernel, workload):
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
-    d = json.load(open(path)).get(kernel)
-    if not d or d.get("workload") != workload:
+    d = json.load(open(path)).get(f"{kernel}@{workload}")
+    if not d:
         return None
     h = hashlib.sha256()
     for f in d.get("sources", []):
@@ -511,7 +511,7 @@ def cpu_value(w, t_step):
     return ideal / t_step
 
 
-def run_reference(args, w):
+def run_reference(args, w, world):
     inputs = oracle_inputs(w)
     for s in range(args.warmup):
         oracle_sample_time(w, inputs, budget_rows=12, seed=1000 + s)
@@ -522,7 +522,7 @@ def run_reference(args, w):
         times.append(t)
     t_step = statistics.mean(times)
     v = cpu_value(w, t_step)
-    return {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": 0, "steps": args.steps,
+    return {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
@@ -552,7 +552,7 @@ def main():
 
     if args.impl == "reference":
         if rank == 0:
-            print(json.dumps(run_reference(args, w)), flush=True)
+            print(json.dumps(run_reference(args, w, world)), flush=True)
         return
 
     torch.cuda.set_device(local)
@@ -561,7 +561,15 @@ def main():
         hdist.init("nccl", device)
     line = run_ours(args, rank, world, device)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t, sample, cores = oracle_sample_time(w, oracle_inputs(w))
+        # a small sample sizes the real one to about 10 s of oracle work
+        inputs = oracle_inputs(w)
+        t_probe = time.perf_counter()
+        t, sample, cores = oracle_sample_time(w, inputs, budget_rows=48, seed=7)
+        t_probe = time.perf_counter() - t_probe
+        max_rows = w.batch * w.hkv * 8 if w.decode else min(w.tq, 8192)
+        rows = min(max_rows, int(48 * 10.0 / max(t_probe, 1e-3)))
+        if rows > 48:
+            t, sample, cores = oracle_sample_time(w, inputs, budget_rows=rows)
         line["cpu_baseline"] = {"value": cpu_value(w, t), "unit": UNIT, "cores": cores,
                                 "kind": "oracle", "sample": sample,
                                 "ms_per_step_extrapolated": t * 1e3}

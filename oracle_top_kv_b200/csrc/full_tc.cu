@@ -403,10 +403,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (a.capture) {
             // ---- group merge.  Rows hh*P + pr of the g heads share position
-            // pr; each row's list is sorted by (score desc, id asc).  One
-            // thread per position k-way merges the g lists in that order and
-            // skips ids already taken: an id's first occurrence carries its
-            // largest listed score, so this is the union rule's top-k.
+            // pr; each row's list is sorted by (score desc, id asc).  The g
+            // lists of a position are k-way merged in that order, skipping ids
+            // already taken: an id's first occurrence carries its largest
+            // listed score, so this is the union rule's top-k.  The merge runs
+            // on all 128 threads: a group of g consecutive lanes per position,
+            // lane hh holding the front of head hh's list; each step the group
+            // finds its best front with in-group shuffles and that lane moves on.
             unsigned char* reg = gbase + kPOff + q * 32768;    // this tile's P buffers
             float* cs = reinterpret_cast<float*>(reg);         // [128][kList]
             int* ci = reinterpret_cast<int*>(reg + 128 * kList * 4);
@@ -417,44 +420,47 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ci[row * kList + i] = ok ? li[i] : -1;
             }
             asm volatile("bar.sync %0, 128;" ::"r"(1 + q) : "memory");
-            const int pp = row;  // position handled by this thread
-            if (ok && pp < P && qrow0 + pp < p.t_q) {
-                int ptr[16];
+            const int wl = row >> 5;                  // warp within the warpgroup
+            const int gh = lane % g;                  // head of this lane's list
+            const int pp = wl * (32 / g) + lane / g;  // position of this lane's group
+            const int* lid = ci + (gh * P + pp) * kList;
+            const float* lsc = cs + (gh * P + pp) * kList;
+            int ptr = 0;
+            float fv = lsc[0];
+            int fid = lid[0] >= 0 ? lid[0] : 0x7fffffff;
+            if (lid[0] < 0) fv = -INFINITY;
+            int sid[kList];
+            float ssc[kList];
+            int nsel = 0;
+            const int ksel = p.ksel;
+            // warp-uniform trip count: every group of the warp takes part in the shuffles
+            for (int step = 0; step < g * kList; ++step) {
+                float bv = fv;
+                int bid = fid;
+                for (int o = 1; o < g; o <<= 1) {
+                    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                    const int oid = __shfl_xor_sync(0xffffffffu, bid, o);
+                    if (ov > bv || (ov == bv && oid < bid)) { bv = ov; bid = oid; }
+                }
+                const bool live = bv > -INFINITY && nsel < ksel;
+                if (live && fv == bv && fid == bid) {  // this lane's front was taken
+                    ++ptr;
+                    if (ptr < kList && lid[ptr] >= 0) { fv = lsc[ptr]; fid = lid[ptr]; }
+                    else { fv = -INFINITY; fid = 0x7fffffff; }
+                }
+                bool dup = false;
 #pragma unroll
-                for (int h2 = 0; h2 < 16; ++h2) ptr[h2] = 0;
-                int sid[kList];
-                float ssc[kList];
-                int nsel = 0;
-                for (int guard = 0; guard < 16 * kList && nsel < p.ksel; ++guard) {
-                    float best = -INFINITY;
-                    int best_id = 0x7fffffff, bh = -1;
-#pragma unroll
-                    for (int h2 = 0; h2 < 16; ++h2) {
-                        if (h2 < g && ptr[h2] < kList) {
-                            const int e = (h2 * P + pp) * kList + ptr[h2];
-                            const float v = cs[e];
-                            const int id = ci[e];
-                            if (id >= 0 && (v > best || (v == best && id < best_id))) {
-                                best = v;
-                                best_id = id;
-                                bh = h2;
-                            }
-                        }
-                    }
-                    if (bh < 0) break;  // every list exhausted
-#pragma unroll
-                    for (int h2 = 0; h2 < 16; ++h2)
-                        if (h2 == bh) ++ptr[h2];
-                    bool dup = false;
+                for (int x = 0; x < kList; ++x)
+                    if (x < nsel && sid[x] == bid) dup = true;
+                if (live && !dup) {
 #pragma unroll
                     for (int x = 0; x < kList; ++x)
-                        if (x < nsel && sid[x] == best_id) dup = true;
-                    if (dup) continue;
-#pragma unroll
-                    for (int x = 0; x < kList; ++x)
-                        if (x == nsel) { sid[x] = best_id; ssc[x] = best; }
+                        if (x == nsel) { sid[x] = bid; ssc[x] = bv; }
                     ++nsel;
                 }
+                if (__all_sync(0xffffffffu, !live)) break;
+            }
+            if (ok && gh == 0 && pp < P && qrow0 + pp < p.t_q) {
                 // write in ascending id order
                 const size_t orow_i = ((size_t)b * p.hkv + u) * p.t_q + qrow0 + pp;
                 int32_t* irow = a.idx + orow_i * p.ksel;

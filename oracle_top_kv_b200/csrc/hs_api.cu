@@ -16,6 +16,7 @@
 #include "decode_full.cu"
 #include "full_simt.cu"
 #include "full_tc.cu"
+#include "sparse_tc.cu"
 #include "token_select_tc.cu"
 #include "noalloc.cu"
 #include "sparse.cu"
@@ -163,6 +164,16 @@ hs_status hs_sparse_attn_reuse(const hs_params* p, const void* q_sparse, const v
                                           local ? k_local : nullptr, v_local, o_global,
                                           lse_global, o_local, lse_local, st);
         });
+    if (hs::sparse_tc_supported(kp, p->dtype)) {
+        // global branch on the tensor cores; the window branch (if any) in the gather kernel
+        return launched(local ? 2 : 1, [&] {
+            cudaError_t e = hs::launch_sparse_tc(kp, q_sparse, k_f, v_f, idx, idx_count, o_global,
+                                                 lse_global, st);
+            if (e != cudaSuccess || !local) return e;
+            return hs::launch_sparse_mma(kp, q_sparse, k_f, v_f, idx, idx_count, k_local, v_local,
+                                         o_global, lse_global, o_local, lse_local, st, false);
+        });
+    }
     return launched(1, [&] {
         return hs::launch_sparse_mma(kp, q_sparse, k_f, v_f, idx, idx_count,
                                      local ? k_local : nullptr, v_local, o_global, lse_global,

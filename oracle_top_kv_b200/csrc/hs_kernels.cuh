@@ -37,11 +37,18 @@ cudaError_t launch_sparse_simt(const KParams& p, int dtype, const void* q, const
                                const void* kl, const void* vl, void* og, float* lseg, void* ol,
                                float* lsel, cudaStream_t st);
 
-// bf16 tensor-core paths (mma.sync fragments; d = 64 or 128).
+// bf16 tensor-core paths (mma.sync fragments; d = 64 or 128).  global = false:
+// the window branch only (the global branch is computed by sparse_tc).
 cudaError_t launch_sparse_mma(const KParams& p, const void* q, const void* kf, const void* vf,
                               const int32_t* idx, const int32_t* cnt, const void* kl,
                               const void* vl, void* og, float* lseg, void* ol, float* lsel,
-                              cudaStream_t st);
+                              cudaStream_t st, bool global = true);
+
+// Block-mode global branch on tcgen05 (row-grouped block-sparse attention).
+bool sparse_tc_supported(const KParams& p, int dtype);
+cudaError_t launch_sparse_tc(const KParams& p, const void* q, const void* kf, const void* vf,
+                             const int32_t* idx, const int32_t* cnt, void* og, float* lseg,
+                             cudaStream_t st);
 
 // Decode (bf16, token mode).
 size_t decode_full_workspace(const KParams& p);

@@ -257,14 +257,18 @@ __global__ void __launch_bounds__(W * 32)
     const int unit = b * p.hkv + u;
     const size_t row = (size_t)unit * p.t_q + j;
     const size_t kvoff = (size_t)unit * p.t_kv * D;
-    const int c = clamp_count(cnt[row], p.ksel);
+    // has_local: bit 0 = run the window branch, bit 1 = skip the global branch
+    // (computed by another kernel)
+    const bool do_global = !(has_local & 2);
+    const int c = do_global ? clamp_count(cnt[row], p.ksel) : 0;
     const int n_rows = p.mode == 0 ? c * p.block_size : c;
     if constexpr (kT) {
         uint32_t qb[D / 16][2];
         load_qt_frags<D>(qb, q + q0 * D, head_stride, g);
         AttnStateT<D> st;
         st.init();
-        if (p.mode == 0 && p.block_size % kChunk == 0) {
+        if (!do_global) {
+        } else if (p.mode == 0 && p.block_size % kChunk == 0) {
             BlockChunks src{idx + row * p.ksel, p.block_size, t};
             attend_rows_tma_t<D, S>(st, qb, &tm_kf, &tm_vf, unit, c * (p.block_size / kChunk),
                                     src, sbase, ring, p.scale_log2);
@@ -273,8 +277,8 @@ __global__ void __launch_bounds__(W * 32)
             attend_rows_t<D, S>(st, qb, kf + kvoff, vf + kvoff, (n_rows + kChunk - 1) / kChunk,
                                 keys, sbase, p.scale_log2);
         }
-        store_rows_t<D>(st, og + q0 * D, head_stride, lseg + q0, p.t_q, g);
-        if (has_local) {
+        if (do_global) store_rows_t<D>(st, og + q0 * D, head_stride, lseg + q0, p.t_q, g);
+        if (has_local & 1) {
             const int first = max(0, t - p.window + 1);
             AttnStateT<D> sl;
             sl.init();
@@ -290,7 +294,8 @@ __global__ void __launch_bounds__(W * 32)
 
     AttnState<D> st;
     st.init();
-    if (p.mode == 0 && p.block_size % kChunk == 0) {
+    if (!do_global) {
+    } else if (p.mode == 0 && p.block_size % kChunk == 0) {
         BlockChunks src{idx + row * p.ksel, p.block_size, t};
         attend_rows_tma<D, S>(st, qf, &tm_kf, &tm_vf, unit, c * (p.block_size / kChunk), src,
                               sbase, ring, p.scale_log2, NoHook{});
@@ -299,8 +304,8 @@ __global__ void __launch_bounds__(W * 32)
         attend_rows<D, S>(st, qf, kf + kvoff, vf + kvoff, (n_rows + kChunk - 1) / kChunk, keys,
                           sbase, p.scale_log2, NoHook{});
     }
-    store_rows<D>(st, og + q0 * D, head_stride, lseg + q0, p.t_q, g);
-    if (has_local) {
+    if (do_global) store_rows<D>(st, og + q0 * D, head_stride, lseg + q0, p.t_q, g);
+    if (has_local & 1) {
         const int first = max(0, t - p.window + 1);
         AttnState<D> sl;
         sl.init();
@@ -316,7 +321,7 @@ static cudaError_t launch_sparse_cfg(const KParams& p, const CUtensorMap& mk,
                                      const CUtensorMap& mv, const CUtensorMap& mkl,
                                      const CUtensorMap& mvl, const void* q, const void* kf,
                                      const void* vf, const int32_t* idx, const int32_t* cnt,
-                                     bool has_local, void* og, float* lseg, void* ol, float* lsel,
+                                     int has_local, void* og, float* lseg, void* ol, float* lsel,
                                      cudaStream_t st) {
     constexpr size_t smem = sparse_smem_bytes<D, W, S>();
     auto kern = sparse_mma_kernel<D, kT, W, S>;
@@ -327,7 +332,7 @@ static cudaError_t launch_sparse_cfg(const KParams& p, const CUtensorMap& mk,
     const unsigned grid = (unsigned)((n_tasks + W - 1) / W);
     kern<<<grid, W * 32, smem, st>>>(mk, mv, mkl, mvl, p, (const __nv_bfloat16*)q,
                                      (const __nv_bfloat16*)kf, (const __nv_bfloat16*)vf, idx, cnt,
-                                     has_local ? 1 : 0, (__nv_bfloat16*)og, lseg,
+                                     has_local, (__nv_bfloat16*)og, lseg,
                                      (__nv_bfloat16*)ol, lsel);
     return cudaGetLastError();
 }
@@ -336,7 +341,8 @@ template <int D>
 static cudaError_t launch_sparse_mma_t(const KParams& p, const void* q, const void* kf,
                                        const void* vf, const int32_t* idx, const int32_t* cnt,
                                        const void* kl, const void* vl, void* og, float* lseg,
-                                       void* ol, float* lsel, cudaStream_t st) {
+                                       void* ol, float* lsel, bool global, cudaStream_t st) {
+    const int flags = (kl ? 1 : 0) | (global ? 0 : 2);
     CUtensorMap mk, mv, mkl, mvl;
     const long long units = (long long)p.batch * p.hkv;
     if (!tc::encode_rows(&mk, kf, D, p.t_kv, units, kChunk) ||
@@ -358,19 +364,21 @@ static cudaError_t launch_sparse_mma_t(const KParams& p, const void* q, const vo
     // the heads-as-rows form (168).  At d = 128 these beat 6 warps x 2 stages
     // by 1.6x and 1.4x; 4 x 3 and 3 x 4 were slower still.
     if (p.group <= 8)
-        return launch_sparse_cfg<D, true, 14, 1>(p, mk, mv, mkl, mvl, q, kf, vf, idx, cnt, kl,
+        return launch_sparse_cfg<D, true, 14, 1>(p, mk, mv, mkl, mvl, q, kf, vf, idx, cnt, flags,
                                                  og, lseg, ol, lsel, st);
-    return launch_sparse_cfg<D, false, 12, 1>(p, mk, mv, mkl, mvl, q, kf, vf, idx, cnt, kl, og,
+    return launch_sparse_cfg<D, false, 12, 1>(p, mk, mv, mkl, mvl, q, kf, vf, idx, cnt, flags, og,
                                               lseg, ol, lsel, st);
 }
 
 cudaError_t launch_sparse_mma(const KParams& p, const void* q, const void* kf, const void* vf,
                               const int32_t* idx, const int32_t* cnt, const void* kl,
                               const void* vl, void* og, float* lseg, void* ol, float* lsel,
-                              cudaStream_t st) {
+                              cudaStream_t st, bool global) {
     if (p.head_dim == 64)
-        return launch_sparse_mma_t<64>(p, q, kf, vf, idx, cnt, kl, vl, og, lseg, ol, lsel, st);
-    return launch_sparse_mma_t<128>(p, q, kf, vf, idx, cnt, kl, vl, og, lseg, ol, lsel, st);
+        return launch_sparse_mma_t<64>(p, q, kf, vf, idx, cnt, kl, vl, og, lseg, ol, lsel, global,
+                                       st);
+    return launch_sparse_mma_t<128>(p, q, kf, vf, idx, cnt, kl, vl, og, lseg, ol, lsel, global,
+                                    st);
 }
 
 // ------------------------------------------------------------------- decode

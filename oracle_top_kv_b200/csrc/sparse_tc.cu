@@ -1,0 +1,464 @@
+// sparse_tc.cu -- the HySparse block-mode sparse layer on the tcgen05 tensor
+// cores: row-grouped block-sparse attention.
+//
+// Query row t of a sparse layer attends over the keys of the blocks its index
+// set selects, clipped to keys <= t ("HySparse: ..." 3.3; "跨层 KV Cache 复用
+// 怎样成立"; the in-block causal mask of "工程实现中的关键约束" item 4):
+//     o_h = sum_{i in R_t} softmax_{R_t}(tau q'_h . k_i) v_i.
+// Nearby rows select overlapping block sets: on the HySparse-7B-shaped inputs
+// the 64 positions of a CTA's two Q tiles select about 70 distinct 64-key
+// blocks between them (16 each).  So a CTA forms the union of its rows'
+// selected blocks and streams each union block once through the same tcgen05
+// flash pipeline as the full layer: S = Q K^T for all 128 rows of a Q tile,
+// each row keeping only the blocks it selected (and keys <= t), online
+// softmax, O += P V.  A row pays tensor and exp work for union blocks it did
+// not select (masked to -inf), but each K/V block is read once per CTA
+// instead of once per row, and both contractions run on the tensor cores.
+//
+// Warp roles as in full_tc.cu: warp 0 TMA producer (Q once, union blocks
+// through a 2-stage K/V ring), warp 1 TMEM owner and MMA issuer, warps 2..9
+// two softmax warpgroups (one thread per row).  Supported: bf16, d = 128,
+// block mode with B = 64 (= the key tile), 128 % g == 0, and a union of at
+// most kMaxUnion blocks (2 * (128/g) positions x k/B ids).  The window branch
+// over the layer's own K'/V' runs in sparse_mma_kernel.
+#include "cta_select.cuh"
+#include "hs_common.cuh"
+#include "hs_kernels.cuh"
+#include "tc_ptx.cuh"
+
+namespace hs {
+namespace stc {
+
+using namespace tc;
+
+constexpr int kBM = 128;       // rows per Q tile
+constexpr int kNQ = 2;         // Q tiles per CTA
+constexpr int kBN = 64;        // keys per tile = block size
+constexpr int kD = 128;
+constexpr int kKV = 2;         // K/V ring stages
+constexpr int kMaxSel = 16;    // selected blocks per row held in registers
+constexpr int kMaxUnion = 1024;
+constexpr int kThreads = 64 + 128 * kNQ;
+
+constexpr uint32_t kQOff = 0;                          // kNQ x 32 KB
+constexpr uint32_t kKOff = kNQ * 32768;                // kKV x 16 KB
+constexpr uint32_t kVOff = kKOff + kKV * 16384;        // kKV x 16 KB
+constexpr uint32_t kPOff = kVOff + kKV * 16384;        // kNQ x 2 x 16 KB (block bitmap first)
+constexpr uint32_t kUOff = kPOff + kNQ * 2 * 16384;    // union block ids, kMaxUnion ints
+constexpr uint32_t kBarOff = kUOff + kMaxUnion * 4;
+enum {
+    BQ = 0,
+    BKVF = 1,
+    BKVE = BKVF + kKV,
+    BSF = BKVE + kKV,  // [q][s]
+    BSE = BSF + 2 * kNQ,
+    BPF = BSE + 2 * kNQ,
+    BPVD = BPF + 2 * kNQ,
+    BOF = BPVD + 2 * kNQ,
+    BDRAIN = BOF + 1,
+    BCOUNT = BDRAIN + 1
+};
+constexpr uint32_t kMiscOff = kBarOff + BCOUNT * 8;  // tmem(4) abort(4) U(4) pad(4) scan[16]
+constexpr uint32_t kSmemBytes = kMiscOff + 16 + 64 + 1024;
+constexpr uint32_t kTmemCols = 256 * kNQ;
+constexpr uint32_t kBitmapWords = kNQ * 2 * 16384 / 4;  // blocks the union bitmap covers / 32
+static_assert(kSmemBytes <= 232448, "shared memory");
+
+struct Args {
+    KParams p;
+    const int32_t* idx;
+    const int32_t* cnt;
+    __nv_bfloat16* o;
+    float* lse;
+    int n_ctas_q;
+    int P;  // positions per Q tile (128 / g)
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    sparse_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                     const __grid_constant__ CUtensorMap tmap_k,
+                     const __grid_constant__ CUtensorMap tmap_v, Args a) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    unsigned char* gbase = smem_raw + (base - raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const KParams& p = a.p;
+    const int g = p.group, P = a.P;
+
+    const int bu_n = p.batch * p.hkv;
+    const int qc = a.n_ctas_q - 1 - (int)(blockIdx.x / bu_n);  // latest rows first
+    const int bu = (int)(blockIdx.x % bu_n);
+    const int b = bu / p.hkv, u = bu % p.hkv;
+    const int row0 = qc * kNQ * P;  // first query row of the CTA
+    const int last_row = min(p.t_q, row0 + kNQ * P) - 1;
+    const int n_blocks = (p.q_offset + last_row) / kBN + 1;  // blocks any row may select
+
+    auto bar = [&](int i) { return base + kBarOff + 8u * i; };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kMiscOff);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + kMiscOff + 4);
+    int* s_union = reinterpret_cast<int*>(gbase + kMiscOff + 8);
+    int* s_scan = reinterpret_cast<int*>(gbase + kMiscOff + 16);
+    uint32_t* bitmap = reinterpret_cast<uint32_t*>(gbase + kPOff);  // prologue only
+    int* ulist = reinterpret_cast<int*>(gbase + kUOff);
+    const int words = (n_blocks + 31) >> 5;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(BQ), 1);
+        for (int i = 0; i < kKV; ++i) { mbar_init(bar(BKVF + i), 1); mbar_init(bar(BKVE + i), 1); }
+        for (int i = 0; i < 2 * kNQ; ++i) {
+            mbar_init(bar(BSF + i), 1);
+            mbar_init(bar(BSE + i), 4);
+            mbar_init(bar(BPF + i), 4);
+            mbar_init(bar(BPVD + i), 1);
+        }
+        mbar_init(bar(BOF), 1);
+        mbar_init(bar(BDRAIN), 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(base + kMiscOff, kTmemCols);
+        tmem_relinquish();
+    }
+    for (int x = threadIdx.x; x < words; x += blockDim.x) bitmap[x] = 0u;
+
+    // This thread's row (softmax warps): its position's selected block ids.
+    const bool is_row = warp >= 2;
+    const int q = is_row ? (warp - 2) >> 2 : 0;
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const int hh = row / P, pr = row % P;
+    const int qrow0 = row0 + q * P;
+    const int pos = p.q_offset + qrow0 + pr;
+    const bool row_valid = is_row && qrow0 + pr < p.t_q;
+    int sid[kMaxSel];
+    int nsel = 0;
+#pragma unroll
+    for (int x = 0; x < kMaxSel; ++x) sid[x] = -1;
+    __syncthreads();  // bitmap zeroed
+    if (row_valid) {
+        const size_t irow = ((size_t)b * p.hkv + u) * p.t_q + qrow0 + pr;
+        int c = a.cnt[irow];
+        if (c < 0 || c > p.ksel) { if (hh == 0) set_status(HS_ERR_BOUNDS); c = c < 0 ? 0 : p.ksel; }
+        const int32_t* ids = a.idx + irow * p.ksel;
+#pragma unroll
+        for (int x = 0; x < kMaxSel; ++x) {
+            if (x < c) {
+                const int id = ids[x];
+                if (id < 0 || id > pos / kBN) {
+                    if (hh == 0) set_status(HS_ERR_BOUNDS);
+                } else {
+                    sid[x] = id;
+                    if (hh == 0) atomicOr(&bitmap[id >> 5], 1u << (id & 31));
+                }
+            }
+        }
+        nsel = c;
+    }
+    __syncthreads();  // bitmap complete
+    {
+        // union list, ascending: each thread reads out a run of words
+        const int per = (words + blockDim.x - 1) / blockDim.x;
+        const int w0 = threadIdx.x * per;
+        int cbits = 0;
+        for (int x = 0; x < per; ++x)
+            if (w0 + x < words) cbits += __popc(bitmap[w0 + x]);
+        int at = cta_exclusive_sum(cbits, s_scan);
+        for (int x = 0; x < per; ++x) {
+            if (w0 + x >= words) break;
+            uint32_t m = bitmap[w0 + x];
+            while (m) {
+                if (at < kMaxUnion) ulist[at] = (w0 + x) * 32 + (__ffs(m) - 1);
+                ++at;
+                m &= m - 1u;
+            }
+        }
+        if (threadIdx.x == blockDim.x - 1) *s_union = min(at, kMaxUnion);
+    }
+    tc_fence_before();
+    __syncthreads();  // union ready; the P region is free again
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int U = *s_union;
+    int ntq[kNQ];
+#pragma unroll
+    for (int qq = 0; qq < kNQ; ++qq) ntq[qq] = row0 + qq * P < p.t_q ? U : 0;
+    const int nt = U;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tmap(&tmap_q);
+            prefetch_tmap(&tmap_k);
+            prefetch_tmap(&tmap_v);
+            mbar_arrive_expect_tx(bar(BQ), kNQ * 32768);
+#pragma unroll
+            for (int qq = 0; qq < kNQ; ++qq) {
+                tma_load_4d(base + kQOff + qq * 32768, &tmap_q, bar(BQ), 0, row0 + qq * P, u * g, b);
+                tma_load_4d(base + kQOff + qq * 32768 + 16384, &tmap_q, bar(BQ), 64,
+                            row0 + qq * P, u * g, b);
+            }
+            int issued = 0;
+            for (int j = 0; j < nt; ++j) {
+                const int st = j % kKV;
+                if (j >= kKV && !mbar_wait(bar(BKVE + st), ((j / kKV) - 1) & 1, abort_flag, false))
+                    break;
+                const uint32_t f = bar(BKVF + st);
+                mbar_arrive_expect_tx(f, 4 * 8192);
+                const uint32_t kd = base + kKOff + st * 16384, vd = base + kVOff + st * 16384;
+                const int key0 = ulist[j] * kBN;
+                tma_load_3d(kd, &tmap_k, f, 0, key0, bu);
+                tma_load_3d(kd + 8192, &tmap_k, f, 64, key0, bu);
+                tma_load_3d(vd, &tmap_v, f, 0, key0, bu);
+                tma_load_3d(vd + 8192, &tmap_v, f, 64, key0, bu);
+                issued = j + 1;
+            }
+            mbar_drain(bar(BQ), 0);
+            for (int j = max(0, issued - kKV); j < issued; ++j)
+                mbar_drain(bar(BKVF + j % kKV), (j / kKV) & 1);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t id_s = idesc_bf16(kBM, kBN, false, false);
+            const uint32_t id_o = idesc_bf16(kBM, kD, false, true);
+            bool ok = mbar_wait(bar(BQ), 0, abort_flag, false);
+            tc_fence_after();
+            for (int j = 0; ok && j <= nt; ++j) {
+                if (j < nt) {
+                    const int st = j % kKV, s = j & 1;
+                    if (!mbar_wait(bar(BKVF + st), (j / kKV) & 1, abort_flag, false)) break;
+                    const uint32_t kb = base + kKOff + st * 16384;
+#pragma unroll
+                    for (int qq = 0; qq < kNQ; ++qq) {
+                        if (j >= ntq[qq]) continue;
+                        if (j >= 2 && !mbar_wait(bar(BSE + 2 * qq + s), ((j >> 1) - 1) & 1,
+                                                 abort_flag, false)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t qb = base + kQOff + qq * 32768;
+#pragma unroll
+                        for (int kk = 0; kk < kD / 16; ++kk) {
+                            const uint64_t ad = sw128_desc(qb + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                            const uint64_t bd = sw128_desc(kb + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+                            umma_ss(tmem + qq * 256 + 64 * s, ad, bd, id_s, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(bar(BSF + 2 * qq + s));
+                    }
+                    if (!ok) break;
+                }
+                if (j >= 1) {
+                    const int jj = j - 1, sp = jj & 1, stp = jj % kKV;
+                    const uint32_t vb = base + kVOff + stp * 16384;
+#pragma unroll
+                    for (int qq = 0; qq < kNQ; ++qq) {
+                        if (jj >= ntq[qq]) continue;
+                        if (!mbar_wait(bar(BPF + 2 * qq + sp), (jj >> 1) & 1, abort_flag, false)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t pb = base + kPOff + (2 * qq + sp) * 16384;
+#pragma unroll
+                        for (int kk = 0; kk < kBN / 16; ++kk) {
+                            const uint64_t ad = sw128_desc(pb + kk * 32, 16, 1024);
+                            const uint64_t bd = sw128_desc(vb + kk * 2048, 8192, 1024);
+                            umma_ss(tmem + qq * 256 + 128, ad, bd, id_o, (jj > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit(bar(BPVD + 2 * qq + sp));
+                    }
+                    if (!ok) break;
+                    umma_commit(bar(BKVE + stp));
+                }
+            }
+            umma_commit(bar(BOF));
+            umma_commit(bar(BDRAIN));
+            mbar_drain(bar(BDRAIN), 0);
+        }
+    } else {
+        // ------------------------------------------------------ softmax
+        const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16) + q * 256;
+        const int nt_me = ntq[q];
+        const float sl2 = p.scale_log2;
+        float m_ref = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nt_me; ++j) {
+            const int s = j & 1;
+            if (!warp_wait(bar(BSF + 2 * q + s), (j >> 1) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t r[64];
+            tmem_ld32(trow + 64 * s, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+            tmem_ld32(trow + 64 * s + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(BSE + 2 * q + s));
+
+            // this row keeps the block only if it selected it, and keys <= t
+            const int blk = ulist[j];
+            const int key0 = blk * kBN;
+            bool sel = false;
+#pragma unroll
+            for (int x = 0; x < kMaxSel; ++x) sel |= (x < nsel) & (sid[x] == blk);
+            const int lim = (sel && row_valid) ? pos - key0 : -1;  // last kept column
+            float x[64];
+#pragma unroll
+            for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(r[c]);
+            if (lim < kBN - 1) {
+#pragma unroll
+                for (int c = 0; c < 64; ++c) x[c] = c <= lim ? x[c] : -INFINITY;
+            }
+            float m3[22];
+#pragma unroll
+            for (int c = 0; c < 21; ++c) m3[c] = max3f(x[3 * c], x[3 * c + 1], x[3 * c + 2]);
+            m3[21] = x[63];
+#pragma unroll
+            for (int c = 0; c < 7; ++c) m3[c] = max3f(m3[3 * c], m3[3 * c + 1], m3[3 * c + 2]);
+            const float mt = max3f(max3f(m3[0], m3[1], m3[2]), max3f(m3[3], m3[4], m3[5]),
+                                   fmaxf(m3[6], m3[21])) * sl2;  // -inf stays -inf
+            // lazy rescale; a row may see no kept key for a while (m_ref = -inf)
+            bool resc = false;
+            float corr = 1.f;
+            if (mt > m_ref + 8.f) {
+                corr = ex2(m_ref - mt);  // 0 while nothing was kept
+                resc = m_ref > -INFINITY;
+                m_ref = mt;
+                l *= corr;
+            }
+            const float mu = m_ref == -INFINITY ? 0.f : m_ref;
+            const float2 s2 = make_float2(sl2, sl2), n2 = make_float2(-mu, -mu);
+            float e[64];
+            float2 acc[8];
+#pragma unroll
+            for (int c2 = 0; c2 < 32; ++c2) {
+                const float2 y = ffma2(make_float2(x[2 * c2], x[2 * c2 + 1]), s2, n2);
+                e[2 * c2] = ex2(y.x);
+                e[2 * c2 + 1] = ex2(y.y);
+                const float2 ev = make_float2(e[2 * c2], e[2 * c2 + 1]);
+                acc[c2 & 7] = c2 < 8 ? ev : fadd2(acc[c2 & 7], ev);
+            }
+#pragma unroll
+            for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+                for (int c = 0; c < w; ++c) acc[c] = fadd2(acc[c], acc[c + w]);
+            l += acc[0].x + acc[0].y;
+            uint32_t pk[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(e[2 * c], e[2 * c + 1]);
+            // P buffer s is free once the PV of tile j-2 is done
+            if (j >= 2 && !warp_wait(bar(BPVD + 2 * q + s), ((j >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+            unsigned char* prow = gbase + kPOff + (2 * q + s) * 16384 + row * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint4 v4 = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) = v4;
+            }
+            fence_proxy_async_smem();
+            if (__any_sync(0xffffffffu, resc)) {
+                // O may only be touched once the PV of tile j-1 has finished
+                if (!warp_wait(bar(BPVD + 2 * q + (s ^ 1)), ((j - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const float cf = resc ? corr : 1.f;
+#pragma unroll
+                for (int c4 = 0; c4 < kD / 32; ++c4) {
+                    uint32_t ro[32];
+                    tmem_ld32(trow + 128 + 32 * c4, ro);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) ro[c] = __float_as_uint(__uint_as_float(ro[c]) * cf);
+                    tmem_st32(trow + 128 + 32 * c4, ro);
+                }
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(BPF + 2 * q + s));
+        }
+        if (ok && nt_me > 0) ok = warp_wait(bar(BOF), 0, abort_flag);
+        const size_t orow = ((size_t)b * p.hq + u * g + hh) * p.t_q + qrow0 + pr;
+        if (ok) {  // warp-uniform; the TMEM loads run on every lane of the warp
+            if (nt_me > 0) tc_fence_after();
+            const bool any = l > 0.f;
+            const float inv = any ? 1.f / l : 0.f;
+            __nv_bfloat16* og = a.o + orow * kD;
+#pragma unroll
+            for (int c4 = 0; c4 < kD / 32; ++c4) {
+                uint32_t ro[32];
+                if (nt_me > 0) {
+                    tmem_ld32(trow + 128 + 32 * c4, ro);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) ro[c] = 0u;
+                }
+                if (row_valid) {
+#pragma unroll
+                    for (int c = 0; c < 32; c += 8) {
+                        uint4 v4;
+                        v4.x = pack_bf16(__uint_as_float(ro[c]) * inv, __uint_as_float(ro[c + 1]) * inv);
+                        v4.y = pack_bf16(__uint_as_float(ro[c + 2]) * inv, __uint_as_float(ro[c + 3]) * inv);
+                        v4.z = pack_bf16(__uint_as_float(ro[c + 4]) * inv, __uint_as_float(ro[c + 5]) * inv);
+                        v4.w = pack_bf16(__uint_as_float(ro[c + 6]) * inv, __uint_as_float(ro[c + 7]) * inv);
+                        *reinterpret_cast<uint4*>(og + c4 * 32 + c) = v4;
+                    }
+                }
+            }
+            if (row_valid) a.lse[orow] = any ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace stc
+
+bool sparse_tc_supported(const KParams& p, int dtype) {
+    if (dtype != HS_BF16 || p.head_dim != stc::kD || p.mode != 0) return false;
+    if (p.block_size != stc::kBN || p.ksel > stc::kMaxSel || 128 % p.group != 0) return false;
+    const int P = stc::kBM / p.group;
+    if (stc::kNQ * P * p.ksel > stc::kMaxUnion) return false;  // the union always fits
+    return (long long)(p.t_kv / stc::kBN + 1) <= (long long)stc::kBitmapWords * 32;
+}
+
+cudaError_t launch_sparse_tc(const KParams& p, const void* q, const void* kf, const void* vf,
+                             const int32_t* idx, const int32_t* cnt, void* og, float* lseg,
+                             cudaStream_t st) {
+    const int g = p.group, P = stc::kBM / g;
+    CUtensorMap mq, mk, mv;
+    const cuuint64_t qd[4] = {(cuuint64_t)stc::kD, (cuuint64_t)p.t_q, (cuuint64_t)p.hq,
+                              (cuuint64_t)p.batch};
+    const cuuint64_t qs[3] = {(cuuint64_t)stc::kD * 2, (cuuint64_t)p.t_q * stc::kD * 2,
+                              (cuuint64_t)p.hq * p.t_q * stc::kD * 2};
+    const cuuint32_t qb[4] = {64, (cuuint32_t)P, (cuuint32_t)g, 1};
+    const cuuint64_t kdims[3] = {(cuuint64_t)stc::kD, (cuuint64_t)p.t_kv, (cuuint64_t)p.hkv * p.batch};
+    const cuuint64_t ks[2] = {(cuuint64_t)stc::kD * 2, (cuuint64_t)p.t_kv * stc::kD * 2};
+    const cuuint32_t kb[3] = {64, (cuuint32_t)stc::kBN, 1};
+    if (!tc::encode(&mq, q, 4, qd, qs, qb) || !tc::encode(&mk, kf, 3, kdims, ks, kb) ||
+        !tc::encode(&mv, vf, 3, kdims, ks, kb))
+        return cudaErrorInvalidValue;
+    stc::Args a;
+    a.p = p;
+    a.idx = idx;
+    a.cnt = cnt;
+    a.o = (__nv_bfloat16*)og;
+    a.lse = lseg;
+    a.P = P;
+    a.n_ctas_q = (p.t_q + stc::kNQ * P - 1) / (stc::kNQ * P);
+    cudaError_t e = cudaFuncSetAttribute(stc::sparse_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, stc::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const long long grid = (long long)a.n_ctas_q * p.batch * p.hkv;
+    stc::sparse_tc_kernel<<<(unsigned)grid, stc::kThreads, stc::kSmemBytes, st>>>(mq, mk, mv, a);
+    return cudaGetLastError();
+}
+
+}  // namespace hs

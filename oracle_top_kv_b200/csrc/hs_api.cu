@@ -165,13 +165,13 @@ hs_status hs_sparse_attn_reuse(const hs_params* p, const void* q_sparse, const v
                                           lse_global, o_local, lse_local, st);
         });
     if (hs::sparse_tc_supported(kp, p->dtype)) {
-        // global branch on the tensor cores; the window branch (if any) in the gather kernel
+        // global branch, then the window branch, on the tensor cores
         return launched(local ? 2 : 1, [&] {
             cudaError_t e = hs::launch_sparse_tc(kp, q_sparse, k_f, v_f, idx, idx_count, o_global,
-                                                 lse_global, st);
+                                                 lse_global, false, st);
             if (e != cudaSuccess || !local) return e;
-            return hs::launch_sparse_mma(kp, q_sparse, k_f, v_f, idx, idx_count, k_local, v_local,
-                                         o_global, lse_global, o_local, lse_local, st, false);
+            return hs::launch_sparse_tc(kp, q_sparse, k_local, v_local, idx, idx_count, o_local,
+                                        lse_local, true, st);
         });
     }
     return launched(1, [&] {

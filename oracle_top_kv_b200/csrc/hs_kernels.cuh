@@ -46,9 +46,10 @@ cudaError_t launch_sparse_mma(const KParams& p, const void* q, const void* kf, c
 
 // Block-mode global branch on tcgen05 (row-grouped block-sparse attention).
 bool sparse_tc_supported(const KParams& p, int dtype);
+// window = true: the window branch over the layer's own K'/V' (idx unused).
 cudaError_t launch_sparse_tc(const KParams& p, const void* q, const void* kf, const void* vf,
                              const int32_t* idx, const int32_t* cnt, void* og, float* lseg,
-                             cudaStream_t st);
+                             bool window, cudaStream_t st);
 
 // Decode (bf16, token mode).
 size_t decode_full_workspace(const KParams& p);

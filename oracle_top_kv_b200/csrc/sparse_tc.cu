@@ -20,7 +20,8 @@
 // two softmax warpgroups (one thread per row).  Supported: bf16, d = 128,
 // block mode with B = 64 (= the key tile), 128 % g == 0, and a union of at
 // most kMaxUnion blocks (2 * (128/g) positions x k/B ids).  The window branch
-// over the layer's own K'/V' runs in sparse_mma_kernel.
+// over the layer's own K'/V' (keys t-w+1..t) is a second launch of the same
+// kernel whose block list is the contiguous run the CTA's windows touch.
 #include "cta_select.cuh"
 #include "hs_common.cuh"
 #include "hs_kernels.cuh"
@@ -74,6 +75,9 @@ struct Args {
     int P;  // positions per Q tile (128 / g)
 };
 
+// kWin: the window branch -- keys max(0, t-w+1)..t of the layer's own K'/V',
+// so the block list is the contiguous run of blocks the CTA's windows touch.
+template <bool kWin>
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ CUtensorMap tmap_k,
@@ -93,6 +97,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row0 = qc * kNQ * P;  // first query row of the CTA
     const int last_row = min(p.t_q, row0 + kNQ * P) - 1;
     const int n_blocks = (p.q_offset + last_row) / kBN + 1;  // blocks any row may select
+    const int win_b0 = max(0, p.q_offset + row0 - p.window + 1) / kBN;  // first window block
 
     auto bar = [&](int i) { return base + kBarOff + 8u * i; };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kMiscOff);
@@ -101,7 +106,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int* s_scan = reinterpret_cast<int*>(gbase + kMiscOff + 16);
     uint32_t* bitmap = reinterpret_cast<uint32_t*>(gbase + kPOff);  // prologue only
     int* ulist = reinterpret_cast<int*>(gbase + kUOff);
-    const int words = (n_blocks + 31) >> 5;
+    const int words = kWin ? 0 : (n_blocks + 31) >> 5;
 
     if (threadIdx.x == 0) {
         mbar_init(bar(BQ), 1);
@@ -137,7 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int x = 0; x < kMaxSel; ++x) sid[x] = -1;
     __syncthreads();  // bitmap zeroed
-    if (row_valid) {
+    if (row_valid && !kWin) {
         const size_t irow = ((size_t)b * p.hkv + u) * p.t_q + qrow0 + pr;
         int c = a.cnt[irow];
         if (c < 0 || c > p.ksel) { if (hh == 0) set_status(HS_ERR_BOUNDS); c = c < 0 ? 0 : p.ksel; }
@@ -174,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m &= m - 1u;
             }
         }
-        if (threadIdx.x == blockDim.x - 1) *s_union = min(at, kMaxUnion);
+        if (threadIdx.x == blockDim.x - 1) *s_union = kWin ? n_blocks - win_b0 : min(at, kMaxUnion);
     }
     tc_fence_before();
     __syncthreads();  // union ready; the P region is free again
@@ -207,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t f = bar(BKVF + st);
                 mbar_arrive_expect_tx(f, 4 * 8192);
                 const uint32_t kd = base + kKOff + st * 16384, vd = base + kVOff + st * 16384;
-                const int key0 = ulist[j] * kBN;
+                const int key0 = (kWin ? win_b0 + j : ulist[j]) * kBN;
                 tma_load_3d(kd, &tmap_k, f, 0, key0, bu);
                 tma_load_3d(kd + 8192, &tmap_k, f, 64, key0, bu);
                 tma_load_3d(vd, &tmap_v, f, 0, key0, bu);
@@ -297,19 +302,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(BSE + 2 * q + s));
 
-            // this row keeps the block only if it selected it, and keys <= t
-            const int blk = ulist[j];
+            // global: this row keeps the block only if it selected it, and keys
+            // <= t; window: keys t-w+1..t
+            const int blk = kWin ? win_b0 + j : ulist[j];
             const int key0 = blk * kBN;
-            bool sel = false;
+            bool sel = kWin;
+            if (!kWin) {
 #pragma unroll
-            for (int x = 0; x < kMaxSel; ++x) sel |= (x < nsel) & (sid[x] == blk);
+                for (int x = 0; x < kMaxSel; ++x) sel |= (x < nsel) & (sid[x] == blk);
+            }
             const int lim = (sel && row_valid) ? pos - key0 : -1;  // last kept column
+            const int first = kWin ? pos - p.window + 1 - key0 : 0;  // first kept column
             float x[64];
 #pragma unroll
             for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(r[c]);
-            if (lim < kBN - 1) {
+            if (lim < kBN - 1 || first > 0) {
 #pragma unroll
-                for (int c = 0; c < 64; ++c) x[c] = c <= lim ? x[c] : -INFINITY;
+                for (int c = 0; c < 64; ++c) x[c] = (c <= lim && c >= first) ? x[c] : -INFINITY;
             }
             float m3[22];
 #pragma unroll
@@ -431,7 +440,7 @@ bool sparse_tc_supported(const KParams& p, int dtype) {
 
 cudaError_t launch_sparse_tc(const KParams& p, const void* q, const void* kf, const void* vf,
                              const int32_t* idx, const int32_t* cnt, void* og, float* lseg,
-                             cudaStream_t st) {
+                             bool window, cudaStream_t st) {
     const int g = p.group, P = stc::kBM / g;
     CUtensorMap mq, mk, mv;
     const cuuint64_t qd[4] = {(cuuint64_t)stc::kD, (cuuint64_t)p.t_q, (cuuint64_t)p.hq,
@@ -453,11 +462,12 @@ cudaError_t launch_sparse_tc(const KParams& p, const void* q, const void* kf, co
     a.lse = lseg;
     a.P = P;
     a.n_ctas_q = (p.t_q + stc::kNQ * P - 1) / (stc::kNQ * P);
-    cudaError_t e = cudaFuncSetAttribute(stc::sparse_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, stc::kSmemBytes);
+    auto kern = window ? stc::sparse_tc_kernel<true> : stc::sparse_tc_kernel<false>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, stc::kSmemBytes);
     if (e != cudaSuccess) return e;
     const long long grid = (long long)a.n_ctas_q * p.batch * p.hkv;
-    stc::sparse_tc_kernel<<<(unsigned)grid, stc::kThreads, stc::kSmemBytes, st>>>(mq, mk, mv, a);
+    kern<<<(unsigned)grid, stc::kThreads, stc::kSmemBytes, st>>>(mq, mk, mv, a);
     return cudaGetLastError();
 }
 

@@ -123,6 +123,16 @@ SMALL = {
                                  hq=4, hkv=2, t=100, k=128, window=16),
     "bf16_single_token": wl.scaled(wl.WORKLOADS["hysparse2_prefill"], name="bf16_single_token",
                                    hq=4, hkv=2, t=1, k=16, window=4, needles="count:0"),
+    # block mode, B = 64: the row-grouped tensor-core sparse kernel (group of
+    # 16 with a ragged length; group of 2; a chunk at a nonzero offset)
+    "bf16_block_g16_B64_ragged": wl.scaled(wl.WORKLOADS["hysparse_7b_block"],
+                                           name="bf16_block_g16_B64_ragged", batch=1, hq=32,
+                                           hkv=2, t=520, k=1024, window=128),
+    "bf16_block_g2_B64": wl.scaled(wl.WORKLOADS["hysparse_7b_block"], name="bf16_block_g2_B64",
+                                   hq=4, hkv=2, t=400, k=256, window=64),
+    "bf16_block_g4_B64_chunk": wl.scaled(wl.WORKLOADS["hysparse_7b_block"],
+                                         name="bf16_block_g4_B64_chunk", batch=1, hq=8, hkv=2,
+                                         t=900, t_q=250, q_offset=650, k=512, window=64),
 }
 
 
@@ -155,6 +165,74 @@ def test_bounds_error_sets_status_without_fault():
     hs.hs_sparse_attn_reuse(p, qs, full["k"], full["v"], bad, full["cnt"], None, None, og, lg)
     assert hs.hs_device_status() == hs.HS_ERR_BOUNDS
     assert hs.hs_device_status() == 0  # reading clears it
+
+
+def test_block_sparse_custom_index_sets():
+    """Block mode, B = 64, with index sets made up here rather than by the full
+    layer: empty rows, rows of one block, full rows, blocks crossing the row's
+    position, and the window branch -- against the oracle's sparse formula."""
+    w = wl.scaled(wl.WORKLOADS["hysparse_7b_block"], name="block_custom", batch=2, hq=8, hkv=2,
+                  t=700, k=512, window=96)
+    q, k, v, _ = wl.full_layer_inputs(w)
+    q, k, v = _cuda(q, k, v)
+    ks = w.k // w.block_size
+    rng = np.random.default_rng(5)
+    idx = np.full((w.batch, w.hkv, w.tq, ks), -1, np.int32)
+    cnt = np.zeros((w.batch, w.hkv, w.tq), np.int32)
+    for b in range(w.batch):
+        for u in range(w.hkv):
+            for j in range(w.tq):
+                nb = j // w.block_size + 1
+                kind = rng.integers(0, 4)
+                c = 0 if kind == 0 else 1 if kind == 1 else min(ks, nb) if kind == 2 else \
+                    int(rng.integers(1, min(ks, nb) + 1))
+                ids = np.sort(rng.choice(nb, size=c, replace=False)) if c else np.zeros(0, int)
+                if kind == 1:
+                    ids = np.array([nb - 1])  # the block holding the row: in-block causal clip
+                idx[b, u, j, :c] = ids
+                cnt[b, u, j] = c
+    p = P.abi_params(w)
+    qs = wl.sparse_layer_query(w, 0).to(DEV)
+    kl, vl = _cuda(*wl.sparse_layer_local_kv(w, 0))
+    og, ol = torch.empty_like(qs), torch.empty_like(qs)
+    lg = torch.empty(w.batch, w.hq, w.tq, dtype=torch.float32, device=DEV)
+    ll = torch.empty_like(lg)
+    hs.hs_sparse_attn_reuse(p, qs, k, v, torch.from_numpy(idx).to(DEV),
+                            torch.from_numpy(cnt).to(DEV), kl, vl, og, lg, ol, ll)
+    torch.cuda.synchronize()
+    assert hs.hs_device_status() == 0
+    rws = P.all_rows(w)
+    pos = w.q_offset + rws[:, 2]
+    g_idx = idx[rws[:, 0], rws[:, 1], rws[:, 2]]
+    g_cnt = cnt[rws[:, 0], rws[:, 1], rws[:, 2]]
+    sp = P.oracle_sparse_rows(w, qs, k, v, g_idx, g_cnt, rws, pos, kl, vl)
+    g = w.group
+    P.check_o(P.gpu_rows(P.f64(og), rws, True, g), sp["o_g"], w.dtype, "custom o_g")
+    P.check_lse(P.gpu_rows(lg.cpu().double().numpy(), rws, True, g), sp["lse_g"], w.dtype,
+                "custom lse_g")
+    P.check_o(P.gpu_rows(P.f64(ol), rws, True, g), sp["o_l"], w.dtype, "custom o_l")
+    P.check_lse(P.gpu_rows(ll.cpu().double().numpy(), rws, True, g), sp["lse_l"], w.dtype,
+                "custom lse_l")
+    # empty rows: o = 0, lse = -inf
+    e = np.argwhere(cnt == 0)[0]
+    for hh in range(g):
+        h = e[1] * g + hh
+        assert torch.all(og[e[0], h, e[2]] == 0)
+        assert lg[e[0], h, e[2]].item() == -np.inf
+
+
+def test_block_sparse_bounds_status():
+    w = SMALL["bf16_block_g4_B64"]
+    full = run_full(w)
+    bad = full["idx"].clone()
+    bad[0, 0, 5, 0] = 7  # block 7 starts beyond position 5
+    p = P.abi_params(w)
+    qs = wl.sparse_layer_query(w, 0).to(DEV)
+    og = torch.empty_like(qs)
+    lg = torch.empty(w.batch, w.hq, w.tq, dtype=torch.float32, device=DEV)
+    hs.hs_sparse_attn_reuse(p, qs, full["k"], full["v"], bad, full["cnt"], None, None, og, lg)
+    assert hs.hs_device_status() == hs.HS_ERR_BOUNDS
+    assert hs.hs_device_status() == 0
 
 
 # -------------------------------------------------------------------- decode

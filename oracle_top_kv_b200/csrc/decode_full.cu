@@ -50,14 +50,21 @@ static int sel_splits(const KParams& p) {
     return max(1, max(by_len, by_fill));
 }
 
+constexpr int kSelGroup = 8;  // slices a first-level merge CTA folds (many slices)
+
 struct DecodeWs {
     float* logits;    // [batch*hkv][t_kv][16]
     float* part;      // [batch*hkv][n_split][16][D+2]
     float* lse2;      // [batch*hq]
     uint64_t* cand;   // [batch*hkv][n_sel][kSelMaxRanked] selection keys
     int* cand_n;      // [batch*hkv][n_sel]
-    int n_split, n_sel;
+    uint64_t* cand2;  // [batch*hkv][n_grp][kSelMaxRanked] first-level merge output
+    int* cand2_n;     // [batch*hkv][n_grp]
+    int n_split, n_sel, n_grp;
 };
+
+// Many slices (few sequences, long caches) are merged in two levels.
+static int sel_groups(int n_sel) { return n_sel > 2 * kSelGroup ? (n_sel + kSelGroup - 1) / kSelGroup : 0; }
 
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -65,6 +72,7 @@ static DecodeWs decode_ws_layout(const KParams& p, void* base) {
     DecodeWs w;
     w.n_split = (p.t_kv + kDecodeKeys - 1) / kDecodeKeys;
     w.n_sel = sel_splits(p);
+    w.n_grp = sel_groups(w.n_sel);
     const size_t units = (size_t)p.batch * p.hkv;
     const size_t logits_b = align256(units * p.t_kv * 16 * sizeof(float));
     const size_t part_b = align256(units * w.n_split * 16 * (p.head_dim + 2) * sizeof(float));
@@ -76,6 +84,10 @@ static DecodeWs decode_ws_layout(const KParams& p, void* base) {
     w.lse2 = reinterpret_cast<float*>(c + logits_b + part_b);
     w.cand = reinterpret_cast<uint64_t*>(c + logits_b + part_b + lse_b);
     w.cand_n = reinterpret_cast<int*>(c + logits_b + part_b + lse_b + cand_b);
+    const size_t candn_b = align256(units * w.n_sel * sizeof(int));
+    const size_t cand2_b = align256(units * w.n_grp * kSelMaxRanked * sizeof(uint64_t));
+    w.cand2 = reinterpret_cast<uint64_t*>(c + logits_b + part_b + lse_b + cand_b + candn_b);
+    w.cand2_n = reinterpret_cast<int*>(c + logits_b + part_b + lse_b + cand_b + candn_b + cand2_b);
     return w;
 }
 
@@ -86,7 +98,9 @@ size_t decode_full_workspace(const KParams& p) {
            align256(units * n_split * 16 * (p.head_dim + 2) * sizeof(float)) +
            align256((size_t)p.batch * p.hq * sizeof(float)) +
            align256(units * sel_splits(p) * kSelMaxRanked * sizeof(uint64_t)) +
-           align256(units * sel_splits(p) * sizeof(int));
+           align256(units * sel_splits(p) * sizeof(int)) +
+           align256(units * sel_groups(sel_splits(p)) * kSelMaxRanked * sizeof(uint64_t)) +
+           align256(units * sel_groups(sel_splits(p)) * sizeof(int));
 }
 
 // Writes every head's scaled logit a2 = scale_log2 * q.k of the chunk's keys.
@@ -344,9 +358,43 @@ __device__ int cta_cut(uint64_t* buf, int n, int K, uint64_t* tmp, CtaSelectSmem
 // Stage 2: per unit, the final top-(k-w) of the slices' candidates (cut to
 // k-w whenever the buffer would overflow), sorted by id, then the forced
 // window; or every key when the budget covers them all.
+// First level of a two-level merge: CTA (unit, group) folds kSelGroup slices'
+// candidates into their top-(k-w), written out unsorted as one group list.
+__global__ void __launch_bounds__(kSelectThreads)
+    decode_select_group_kernel(KParams p, const int32_t* __restrict__ seq_len, DecodeWs ws) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    __shared__ CtaSelectSmem cs;
+    __shared__ int s_n;
+    const int unit = blockIdx.x / ws.n_grp, grp = blockIdx.x % ws.n_grp;
+    const int b = unit / p.hkv;
+    const int L = seq_len[b];
+    const int Kc = p.k - p.window;
+    int* out_n = ws.cand2_n + (size_t)unit * ws.n_grp + grp;
+    if (L < 1 || L > p.t_kv || L <= p.k || Kc <= 0) {
+        if (threadIdx.x == 0) *out_n = 0;
+        return;
+    }
+    uint64_t* buf = reinterpret_cast<uint64_t*>(smem_raw);  // [kSelGroup * kSelMaxRanked]
+    uint64_t* tmp = buf + kSelGroup * kSelMaxRanked;         // [kSelMaxRanked]
+    int n = 0;
+    const int s0 = grp * kSelGroup, s1 = min(ws.n_sel, s0 + kSelGroup);
+    for (int sp = s0; sp < s1; ++sp) {
+        const int c = ws.cand_n[(size_t)unit * ws.n_sel + sp];
+        const uint64_t* src = ws.cand + ((size_t)unit * ws.n_sel + sp) * kSelMaxRanked;
+        for (int x = threadIdx.x; x < c; x += blockDim.x) buf[n + x] = src[x];
+        n += c;
+    }
+    __syncthreads();
+    if (n > Kc) n = cta_cut(buf, n, Kc, tmp, cs, &s_n);
+    uint64_t* dst = ws.cand2 + ((size_t)unit * ws.n_grp + grp) * kSelMaxRanked;
+    for (int x = threadIdx.x; x < n; x += blockDim.x) dst[x] = buf[x];
+    if (threadIdx.x == 0) *out_n = n;
+}
+
 __global__ void __launch_bounds__(kSelectThreads)
     decode_select_merge_kernel(KParams p, const int32_t* __restrict__ seq_len, DecodeWs ws,
-                               int32_t* __restrict__ idx, int32_t* __restrict__ cnt,
+                               const uint64_t* __restrict__ cand, const int* __restrict__ cand_n,
+                               int n_src, int32_t* __restrict__ idx, int32_t* __restrict__ cnt,
                                float* __restrict__ sel) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     __shared__ CtaSelectSmem cs;
@@ -389,10 +437,10 @@ __global__ void __launch_bounds__(kSelectThreads)
     uint64_t* tmp = buf + kMergeCap;                         // [kSelMaxRanked]
     int n = 0;
     if (Kc > 0) {
-        for (int sp = 0; sp < ws.n_sel; ++sp) {
-            const int c = ws.cand_n[(size_t)unit * ws.n_sel + sp];
+        for (int sp = 0; sp < n_src; ++sp) {
+            const int c = cand_n[(size_t)unit * n_src + sp];
             if (n + c > kMergeCap) n = cta_cut(buf, n, Kc, tmp, cs, &s_n);
-            const uint64_t* src = ws.cand + ((size_t)unit * ws.n_sel + sp) * kSelMaxRanked;
+            const uint64_t* src = cand + ((size_t)unit * n_src + sp) * kSelMaxRanked;
             for (int x = threadIdx.x; x < c; x += blockDim.x) buf[n + x] = src[x];
             n += c;
             __syncthreads();
@@ -477,12 +525,27 @@ static cudaError_t launch_decode_full_t(const KParams& p, const void* q, const v
         decode_select_split_kernel<<<p.batch * p.hkv * w.n_sel, kSelectThreads, s1, st>>>(
             p, seq_len, w);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        const uint64_t* cand = w.cand;
+        const int* cand_n = w.cand_n;
+        int n_src = w.n_sel;
+        if (w.n_grp > 0) {  // many slices: fold groups of them on more CTAs first
+            const size_t sg = sizeof(uint64_t) * (kSelGroup * kSelMaxRanked + kSelMaxRanked);
+            e = cudaFuncSetAttribute(decode_select_group_kernel,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sg);
+            if (e != cudaSuccess) return e;
+            decode_select_group_kernel<<<p.batch * p.hkv * w.n_grp, kSelectThreads, sg, st>>>(
+                p, seq_len, w);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            cand = w.cand2;
+            cand_n = w.cand2_n;
+            n_src = w.n_grp;
+        }
         const size_t s2 = sizeof(uint64_t) * (kMergeCap + kSelMaxRanked);
         e = cudaFuncSetAttribute(decode_select_merge_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s2);
         if (e != cudaSuccess) return e;
-        decode_select_merge_kernel<<<p.batch * p.hkv, kSelectThreads, s2, st>>>(p, seq_len, w, idx,
-                                                                               cnt, sel);
+        decode_select_merge_kernel<<<p.batch * p.hkv, kSelectThreads, s2, st>>>(
+            p, seq_len, w, cand, cand_n, n_src, idx, cnt, sel);
         return cudaGetLastError();
     }
     const size_t sel_smem = BlockTopK::smem_bytes(Kc, kSelectThreads);
@@ -492,6 +555,11 @@ static cudaError_t launch_decode_full_t(const KParams& p, const void* q, const v
     decode_select_kernel<<<p.batch * p.hkv, kSelectThreads, sel_smem, st>>>(p, seq_len, w, idx,
                                                                            cnt, sel);
     return cudaGetLastError();
+}
+
+int decode_full_kernel_count(const KParams& p) {
+    if (p.k - p.window > kSelMaxRanked) return 3;  // split, combine, one-CTA selector
+    return sel_groups(sel_splits(p)) > 0 ? 5 : 4;  // + split selector, (group merge,) merge
 }
 
 cudaError_t launch_decode_full(const KParams& p, const void* q, const void* kc, const void* vc,

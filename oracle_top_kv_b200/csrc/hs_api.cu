@@ -212,7 +212,7 @@ hs_status hs_decode_step(const hs_params* p, int32_t kind, const void* q, const 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (kind == HS_DECODE_FULL_INDEX) {
         if (!lse) return HS_ERR_INVALID_ARG;
-        const int n_kernels = kp.k - kp.window <= 1024 ? 4 : 3;
+        const int n_kernels = hs::decode_full_kernel_count(kp);
         return launched(n_kernels, [&] {
             return hs::launch_decode_full(kp, q, k_cache, v_cache, seq_len, idx, idx_count, o,
                                           lse, sel_scores, workspace, st);

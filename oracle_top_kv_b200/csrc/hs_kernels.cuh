@@ -53,6 +53,7 @@ cudaError_t launch_sparse_tc(const KParams& p, const void* q, const void* kf, co
 
 // Decode (bf16, token mode).
 size_t decode_full_workspace(const KParams& p);
+int decode_full_kernel_count(const KParams& p);  // kernels one full decode step launches
 size_t decode_sparse_workspace(const KParams& p);
 cudaError_t launch_decode_full(const KParams& p, const void* q, const void* kc, const void* vc,
                                const int32_t* seq_len, int32_t* idx, int32_t* cnt, void* o,

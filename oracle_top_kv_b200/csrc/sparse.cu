@@ -426,41 +426,52 @@ __global__ void __launch_bounds__(kSparseWarps * 32)
 }
 
 // Exact merge of split partials: M = max m_s, l = sum l_s 2^(m_s - M),
-// o = sum O_s 2^(m_s - M) / l.  One CTA of D threads per (sequence, head);
-// thread d accumulates element d over all splits.
+// o = sum O_s 2^(m_s - M) / l.  One CTA of parts x D threads per (sequence,
+// head): thread (part, d) accumulates element d over the splits s = part
+// mod parts, and the parts are added in shared memory (parts = 4 when there
+// are many splits -- long caches -- else 1).
+constexpr int kCombineParts = 4;
+static int combine_parts(int n_split) { return n_split >= 256 ? kCombineParts : 1; }
+
 template <int D>
-__global__ void __launch_bounds__(D)
+__global__ void __launch_bounds__(kCombineParts * D)
     decode_combine_kernel(KParams p, const float* __restrict__ part, int n_split,
                           const int32_t* __restrict__ seq_len, __nv_bfloat16* __restrict__ o,
                           float* __restrict__ lse, float* __restrict__ lse2_out) {
-    __shared__ float red_m[D / 32], red_l[D / 32];
+    constexpr int NWMAX = kCombineParts * D / 32;
+    __shared__ float red_m[NWMAX], red_l[NWMAX];
+    const int NW = blockDim.x >> 5, parts = blockDim.x / D;
+    __shared__ float s_acc[kCombineParts][D];
     const int row = blockIdx.x;  // b * hq + h
     const int h = row % p.hq, b = row / p.hq;
     const int g = p.group, u = h / g, hh = h % g;
     const int unit = b * p.hkv + u;
-    const int d = threadIdx.x, lane = d & 31, warp = d >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int d = tid % D, prt = tid / D;
     const int L = seq_len[b];
     constexpr size_t S = 16 * (D + 2);  // floats between consecutive splits
     const float* base = part + (size_t)unit * n_split * S + (size_t)hh * (D + 2);
     float M = -INFINITY;
-    for (int s = d; s < n_split; s += D) M = fmaxf(M, base[s * S]);
+    for (int s = tid; s < n_split; s += blockDim.x) M = fmaxf(M, base[s * S]);
     M = warp_max(M);
     if (lane == 0) red_m[warp] = M;
     __syncthreads();
-#pragma unroll
-    for (int w = 0; w < D / 32; ++w) M = fmaxf(M, red_m[w]);
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, red_m[w]);
     const float Mu = M == -INFINITY ? 0.f : M;
     float l = 0.f;
-    for (int s = d; s < n_split; s += D) l += base[s * S + 1] * exp2f(base[s * S] - Mu);
+    for (int s = tid; s < n_split; s += blockDim.x) l += base[s * S + 1] * exp2f(base[s * S] - Mu);
     l = warp_sum(l);
     if (lane == 0) red_l[warp] = l;
     float acc = 0.f;
-#pragma unroll 8
-    for (int s = 0; s < n_split; ++s) acc += base[s * S + 2 + d] * exp2f(base[s * S] - Mu);
+#pragma unroll 4
+    for (int s = prt; s < n_split; s += parts)
+        acc += base[s * S + 2 + d] * exp2f(base[s * S] - Mu);
+    s_acc[prt][d] = acc;
     __syncthreads();
+    if (prt != 0) return;
     l = 0.f;
-#pragma unroll
-    for (int w = 0; w < D / 32; ++w) l += red_l[w];
+    for (int w = 0; w < NW; ++w) l += red_l[w];
+    for (int x = 1; x < parts; ++x) acc += s_acc[x][d];
     const bool ok = L >= 1 && L <= p.t_kv && l > 0.f;
     o[(size_t)row * D + d] = __float2bfloat16_rn(ok ? acc / l : 0.f);
     if (d == 0) {
@@ -493,8 +504,8 @@ static cudaError_t launch_decode_sparse_split_t(const KParams& p, const void* q,
         p, (const __nv_bfloat16*)q, (const __nv_bfloat16*)kc, (const __nv_bfloat16*)vc, seq_len,
         idx, cnt, (float*)ws, n_split);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    decode_combine_kernel<D><<<p.batch * p.hq, D, 0, st>>>(p, (const float*)ws, n_split, seq_len,
-                                                           (__nv_bfloat16*)o, lse, nullptr);
+    decode_combine_kernel<D><<<p.batch * p.hq, combine_parts(n_split) * D, 0, st>>>(
+        p, (const float*)ws, n_split, seq_len, (__nv_bfloat16*)o, lse, nullptr);
     return cudaGetLastError();
 }
 
@@ -733,11 +744,11 @@ cudaError_t launch_decode_combine(const KParams& p, const float* part, int n_spl
                                   cudaStream_t st) {
     const int rows = p.batch * p.hq;
     if (p.head_dim == 64)
-        decode_combine_kernel<64><<<rows, 64, 0, st>>>(p, part, n_split, seq_len,
-                                                       (__nv_bfloat16*)o, lse, lse2);
+        decode_combine_kernel<64><<<rows, combine_parts(n_split) * 64, 0, st>>>(
+            p, part, n_split, seq_len, (__nv_bfloat16*)o, lse, lse2);
     else
-        decode_combine_kernel<128><<<rows, 128, 0, st>>>(p, part, n_split, seq_len,
-                                                         (__nv_bfloat16*)o, lse, lse2);
+        decode_combine_kernel<128><<<rows, combine_parts(n_split) * 128, 0, st>>>(
+            p, part, n_split, seq_len, (__nv_bfloat16*)o, lse, lse2);
     return cudaGetLastError();
 }
 

@@ -290,6 +290,14 @@ def test_decode_small_ragged():
     run_decode(w, torch.tensor([5000, 1, 200, 4097], dtype=torch.int32))
 
 
+def test_decode_single_sequence_two_level_merge():
+    # one sequence and one KV group: the selector splits the cache into 35
+    # slices, so their candidates are merged in two levels
+    w = wl.scaled(wl.WORKLOADS["hysparse2_decode"], name="decode_one_seq", batch=1, hq=16, hkv=1,
+                  t=70000, k=512, window=64)
+    run_decode(w, torch.tensor([69999], dtype=torch.int32), layers=1)
+
+
 def test_decode_small_g4_d64():
     w = wl.scaled(wl.WORKLOADS["hysparse2_decode"], name="decode_g4", batch=2, hq=8, hkv=2,
                   head_dim=64, t=3000, k=100, window=10)

@@ -1,0 +1,288 @@
+// flash_tc.cuh -- the tcgen05 flash-attention pipeline shared by the full
+// layer (full_tc.cu) and the row-grouped sparse layer (sparse_tc.cu).
+//
+// A CTA runs two 128-row Q tiles over a list of 64-key tiles that both share.
+// Warp 0 is the TMA producer, warp 1 owns TMEM and issues the MMAs from one
+// thread, warps 2..9 are two softmax warpgroups with one thread per row:
+//   S = Q K^T  (M = 128, N = 64, K = 16 x 8) into one of two TMEM buffers,
+//   O += P V   (N = 128, V as the MN-major operand; P from shared memory).
+// The kernels differ in which key tiles they visit, which keys a row keeps,
+// and what they do besides attention (block-score capture, union building).
+#pragma once
+
+#include "hs_common.cuh"
+#include "tc_ptx.cuh"
+
+namespace hs {
+namespace fl {
+
+using namespace tc;
+
+// Shared-memory map and mbarrier indices of a pipeline with a KV-stage ring
+// and `Extra` kernel-specific bytes after the P buffers.
+template <int KV, uint32_t Extra>
+struct Layout {
+    static constexpr int kBM = 128, kNQ = 2, kBN = 64, kD = 128, kKV = KV;
+    static constexpr int kThreads = 64 + 128 * kNQ;
+    static constexpr uint32_t kQOff = 0;                       // kNQ x 32 KB (two d halves)
+    static constexpr uint32_t kKOff = kNQ * 32768;             // KV x 16 KB
+    static constexpr uint32_t kVOff = kKOff + KV * 16384;      // KV x 16 KB
+    static constexpr uint32_t kPOff = kVOff + KV * 16384;      // kNQ x 2 x 16 KB
+    static constexpr uint32_t kExtraOff = kPOff + kNQ * 2 * 16384;
+    static constexpr uint32_t kBarOff = kExtraOff + Extra;
+    enum {
+        BQ = 0,
+        BKVF = 1,
+        BKVE = BKVF + KV,
+        BSF = BKVE + KV,  // [q][s]
+        BSE = BSF + 2 * kNQ,
+        BPF = BSE + 2 * kNQ,
+        BPVD = BPF + 2 * kNQ,
+        BOF = BPVD + 2 * kNQ,
+        BDRAIN = BOF + 1,
+        BCOUNT = BDRAIN + 1
+    };
+    static constexpr uint32_t kMiscOff = kBarOff + BCOUNT * 8;  // tmem slot, abort flag, ...
+    static constexpr uint32_t kTmemCols = 256 * kNQ;            // per Q tile: S0 | S1 | O
+};
+
+// Bounded wait that ignores the abort flag (used to drain in-flight work).
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait_sleep(bar, parity)) {
+        if (clock64() - t0 > kWaitCycles) { set_status(HS_ERR_TIMEOUT); return; }
+    }
+}
+
+// Warp-uniform bounded wait: every lane polls, the warp proceeds only if all saw it.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+    const bool ok = mbar_wait(bar, parity, abort);
+    return __all_sync(0xffffffffu, ok);
+}
+
+template <class L>
+__device__ __forceinline__ void init_barriers(uint32_t bar0) {
+    auto bar = [&](int i) { return bar0 + 8u * i; };
+    mbar_init(bar(L::BQ), 1);
+    for (int i = 0; i < L::kKV; ++i) { mbar_init(bar(L::BKVF + i), 1); mbar_init(bar(L::BKVE + i), 1); }
+    for (int i = 0; i < 2 * L::kNQ; ++i) {
+        mbar_init(bar(L::BSF + i), 1);
+        mbar_init(bar(L::BSE + i), 4);
+        mbar_init(bar(L::BPF + i), 4);
+        mbar_init(bar(L::BPVD + i), 1);
+    }
+    mbar_init(bar(L::BOF), 1);
+    mbar_init(bar(L::BDRAIN), 1);
+}
+
+// TMA producer (one thread): both Q tiles once (4-D boxes: 64 d x P positions
+// x g heads), then the key tiles key0_of(j), j < nt, through the ring.
+template <class L, class KeyOf>
+__device__ __forceinline__ void producer(uint32_t base, const CUtensorMap* tq, const CUtensorMap* tk,
+                                         const CUtensorMap* tv, int row0, int P, int head0, int b,
+                                         int bu, int nt, KeyOf key0_of, volatile int* abort) {
+    auto bar = [&](int i) { return base + L::kBarOff + 8u * i; };
+    prefetch_tmap(tq);
+    prefetch_tmap(tk);
+    prefetch_tmap(tv);
+    mbar_arrive_expect_tx(bar(L::BQ), L::kNQ * 32768);
+#pragma unroll
+    for (int q = 0; q < L::kNQ; ++q) {
+        tma_load_4d(base + L::kQOff + q * 32768, tq, bar(L::BQ), 0, row0 + q * P, head0, b);
+        tma_load_4d(base + L::kQOff + q * 32768 + 16384, tq, bar(L::BQ), 64, row0 + q * P, head0, b);
+    }
+    int issued = 0;
+    for (int j = 0; j < nt; ++j) {
+        const int st = j % L::kKV;
+        if (j >= L::kKV && !mbar_wait(bar(L::BKVE + st), ((j / L::kKV) - 1) & 1, abort, false))
+            break;
+        const uint32_t f = bar(L::BKVF + st);
+        mbar_arrive_expect_tx(f, 4 * 8192);
+        const uint32_t kd = base + L::kKOff + st * 16384, vd = base + L::kVOff + st * 16384;
+        const int key0 = key0_of(j);
+        tma_load_3d(kd, tk, f, 0, key0, bu);
+        tma_load_3d(kd + 8192, tk, f, 64, key0, bu);
+        tma_load_3d(vd, tv, f, 0, key0, bu);
+        tma_load_3d(vd + 8192, tv, f, 64, key0, bu);
+        issued = j + 1;
+    }
+    // every issued load must have landed before the CTA may exit
+    mbar_drain(bar(L::BQ), 0);
+    for (int j = max(0, issued - L::kKV); j < issued; ++j)
+        mbar_drain(bar(L::BKVF + j % L::kKV), (j / L::kKV) & 1);
+}
+
+// MMA issuer (one thread): iteration j issues S = Q K^T of tile j for both Q
+// tiles (each waits for its S buffer), then O += P V of tile j-1 (each waits
+// for its P), and releases tile j-1's K/V stage.  Q tile q uses ntq[q] tiles.
+template <class L>
+__device__ __forceinline__ void mma_issuer(uint32_t base, uint32_t tmem, int nt,
+                                           const int (&ntq)[L::kNQ], volatile int* abort) {
+    auto bar = [&](int i) { return base + L::kBarOff + 8u * i; };
+    const uint32_t id_s = idesc_bf16(L::kBM, L::kBN, false, false);
+    const uint32_t id_o = idesc_bf16(L::kBM, L::kD, false, true);
+    bool ok = mbar_wait(bar(L::BQ), 0, abort, false);
+    tc_fence_after();
+    for (int j = 0; ok && j <= nt; ++j) {
+        if (j < nt) {
+            const int st = j % L::kKV, s = j & 1;
+            if (!mbar_wait(bar(L::BKVF + st), (j / L::kKV) & 1, abort, false)) break;
+            const uint32_t kb = base + L::kKOff + st * 16384;
+#pragma unroll
+            for (int q = 0; q < L::kNQ; ++q) {
+                if (j >= ntq[q]) continue;
+                if (j >= 2 && !mbar_wait(bar(L::BSE + 2 * q + s), ((j >> 1) - 1) & 1, abort, false)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t qb = base + L::kQOff + q * 32768;
+#pragma unroll
+                for (int kk = 0; kk < L::kD / 16; ++kk) {
+                    const uint64_t ad = sw128_desc(qb + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bd = sw128_desc(kb + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+                    umma_ss(tmem + q * 256 + 64 * s, ad, bd, id_s, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(bar(L::BSF + 2 * q + s));
+            }
+            if (!ok) break;
+        }
+        if (j >= 1) {
+            const int jj = j - 1, sp = jj & 1, stp = jj % L::kKV;
+            const uint32_t vb = base + L::kVOff + stp * 16384;
+#pragma unroll
+            for (int q = 0; q < L::kNQ; ++q) {
+                if (jj >= ntq[q]) continue;
+                if (!mbar_wait(bar(L::BPF + 2 * q + sp), (jj >> 1) & 1, abort, false)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t pb = base + L::kPOff + (2 * q + sp) * 16384;
+#pragma unroll
+                for (int kk = 0; kk < L::kBN / 16; ++kk) {
+                    const uint64_t ad = sw128_desc(pb + kk * 32, 16, 1024);
+                    const uint64_t bd = sw128_desc(vb + kk * 2048, 8192, 1024);
+                    umma_ss(tmem + q * 256 + 128, ad, bd, id_o, (jj > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(bar(L::BPVD + 2 * q + sp));
+            }
+            if (!ok) break;
+            umma_commit(bar(L::BKVE + stp));
+        }
+    }
+    umma_commit(bar(L::BOF));
+    umma_commit(bar(L::BDRAIN));
+    mbar_drain(bar(L::BDRAIN), 0);
+}
+
+// One 64-key tile of one row: raw logits r[] (TMEM), keep columns first..lim
+// (the rest -> -inf), tile max mt (log2 domain, -inf if nothing kept), lazy
+// rescale (the reference max m_ref moves only when the tile exceeds it by
+// more than 2^8; *corr is then the factor for l and O, and the return value
+// says whether O holds anything to rescale), p = 2^(x*scale_log2 - m_ref)
+// with packed FMA, row sum into l, and P packed to bf16 pairs.
+__device__ __forceinline__ bool softmax_tile(const uint32_t (&r)[64], int first, int lim, float sl2,
+                                             float& m_ref, float& l, float& mt, float& corr,
+                                             uint32_t (&pk)[32]) {
+    float x[64];
+#pragma unroll
+    for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(r[c]);
+    if (lim < 63 || first > 0) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) x[c] = (c <= lim && c >= first) ? x[c] : -INFINITY;
+    }
+    float m3[22];
+#pragma unroll
+    for (int c = 0; c < 21; ++c) m3[c] = max3f(x[3 * c], x[3 * c + 1], x[3 * c + 2]);
+    m3[21] = x[63];
+#pragma unroll
+    for (int c = 0; c < 7; ++c) m3[c] = max3f(m3[3 * c], m3[3 * c + 1], m3[3 * c + 2]);
+    mt = max3f(max3f(m3[0], m3[1], m3[2]), max3f(m3[3], m3[4], m3[5]), fmaxf(m3[6], m3[21])) *
+         sl2;  // -inf stays -inf (sl2 > 0)
+    bool resc = false;
+    corr = 1.f;
+    if (mt > m_ref + 8.f) {
+        corr = ex2(m_ref - mt);  // 0 while nothing was kept
+        resc = m_ref > -INFINITY;
+        m_ref = mt;
+        l *= corr;
+    }
+    const float mu = m_ref == -INFINITY ? 0.f : m_ref;
+    const float2 s2 = make_float2(sl2, sl2), n2 = make_float2(-mu, -mu);
+    float e[64];
+    float2 acc[8];
+#pragma unroll
+    for (int c2 = 0; c2 < 32; ++c2) {
+        const float2 y = ffma2(make_float2(x[2 * c2], x[2 * c2 + 1]), s2, n2);
+        e[2 * c2] = ex2(y.x);
+        e[2 * c2 + 1] = ex2(y.y);
+        const float2 ev = make_float2(e[2 * c2], e[2 * c2 + 1]);
+        acc[c2 & 7] = c2 < 8 ? ev : fadd2(acc[c2 & 7], ev);
+    }
+#pragma unroll
+    for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+        for (int c = 0; c < w; ++c) acc[c] = fadd2(acc[c], acc[c + w]);
+    l += acc[0].x + acc[0].y;
+#pragma unroll
+    for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(e[2 * c], e[2 * c + 1]);
+    return resc;
+}
+
+// P row (64 keys, bf16) into the 128B-swizzled P buffer, made visible to the
+// tensor core's operand reads.
+__device__ __forceinline__ void store_p(unsigned char* pbuf, int row, const uint32_t (&pk)[32]) {
+    unsigned char* prow = pbuf + row * 128;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const uint4 v4 = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) = v4;
+    }
+    fence_proxy_async_smem();
+}
+
+// O row *= cf in TMEM (every lane of the warp calls this).
+__device__ __forceinline__ void rescale_o(uint32_t trow_o, float cf) {
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) {
+        uint32_t ro[32];
+        tmem_ld32(trow_o + 32 * c4, ro);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) ro[c] = __float_as_uint(__uint_as_float(ro[c]) * cf);
+        tmem_st32(trow_o + 32 * c4, ro);
+    }
+    tmem_wait_st();
+}
+
+// O row * inv -> og[0..128) as bf16 (every lane of the warp calls this; only
+// lanes with store = true write; have_o = false writes zeros).
+__device__ __forceinline__ void store_o(uint32_t trow_o, bool have_o, float inv, bool store,
+                                        __nv_bfloat16* og) {
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) {
+        uint32_t ro[32];
+        if (have_o) {
+            tmem_ld32(trow_o + 32 * c4, ro);
+            tmem_wait_ld();
+        } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) ro[c] = 0u;
+        }
+        if (store) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 8) {
+                uint4 v4;
+                v4.x = pack_bf16(__uint_as_float(ro[c]) * inv, __uint_as_float(ro[c + 1]) * inv);
+                v4.y = pack_bf16(__uint_as_float(ro[c + 2]) * inv, __uint_as_float(ro[c + 3]) * inv);
+                v4.z = pack_bf16(__uint_as_float(ro[c + 4]) * inv, __uint_as_float(ro[c + 5]) * inv);
+                v4.w = pack_bf16(__uint_as_float(ro[c + 6]) * inv, __uint_as_float(ro[c + 7]) * inv);
+                *reinterpret_cast<uint4*>(og + c4 * 32 + c) = v4;
+            }
+        }
+    }
+}
+
+}  // namespace fl
+}  // namespace hs

@@ -28,6 +28,7 @@
 //                grows by > 2^8), P to shared memory, block-score capture,
 //                epilogue.
 // All waits are bounded (tc_ptx.cuh); a timeout aborts the CTA cleanly.
+#include "flash_tc.cuh"
 #include "hs_common.cuh"
 #include "hs_kernels.cuh"
 #include "tc_ptx.cuh"
@@ -35,37 +36,11 @@
 namespace hs {
 namespace tc {
 
-constexpr int kBM = 128;      // rows per Q tile (one softmax warpgroup)
-constexpr int kNQ = 2;        // Q tiles per CTA, sharing every K/V tile
-constexpr int kBN = 64;       // keys per K/V tile (= block size B)
-constexpr int kD = 128;
-constexpr int kKV = 3;        // K/V ring stages
+using L = fl::Layout<3, 0>;   // 3-stage K/V ring, nothing beyond the P buffers
+constexpr int kBM = L::kBM, kNQ = L::kNQ, kBN = L::kBN, kD = L::kD;
 constexpr int kList = 16;     // per-row candidate list (>= k/B)
-constexpr int kThreads = 64 + 128 * kNQ;
-// The TMA producer and the MMA issuer are single threads on the critical
-// path: they poll their barriers instead of sleeping.
-constexpr bool kRoleSleep = false;
-
-constexpr uint32_t kQOff = 0;                         // kNQ x 32 KB (two d halves each)
-constexpr uint32_t kKOff = kNQ * 32768;               // kKV x 16 KB
-constexpr uint32_t kVOff = kKOff + kKV * 16384;       // kKV x 16 KB
-constexpr uint32_t kPOff = kVOff + kKV * 16384;       // kNQ x 2 x 16 KB
-constexpr uint32_t kBarOff = kPOff + kNQ * 2 * 16384;
-enum {
-    BQ = 0,
-    BKVF = 1,
-    BKVE = BKVF + kKV,
-    BSF = BKVE + kKV,      // [q][s]
-    BSE = BSF + 2 * kNQ,
-    BPF = BSE + 2 * kNQ,
-    BPVD = BPF + 2 * kNQ,
-    BOF = BPVD + 2 * kNQ,
-    BDRAIN = BOF + 1,
-    BCOUNT = BDRAIN + 1
-};
-constexpr uint32_t kMiscOff = kBarOff + BCOUNT * 8;
-constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;  // + room to align the base to 1 KB
-constexpr uint32_t kTmemCols = 256 * kNQ;              // per Q tile: S0 | S1 | O
+constexpr int kThreads = L::kThreads;
+constexpr uint32_t kSmemBytes = L::kMiscOff + 16 + 1024;  // + room to align the base to 1 KB
 
 struct FullTcArgs {
     KParams p;
@@ -78,20 +53,6 @@ struct FullTcArgs {
     int P;         // positions per Q tile (128 / g)
     int capture;   // 1: block-mode selection
 };
-
-// Bounded wait that ignores the abort flag (used to drain in-flight work).
-__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
-    const long long t0 = clock64();
-    while (!mbar_try_wait_sleep(bar, parity)) {
-        if (clock64() - t0 > kWaitCycles) { set_status(HS_ERR_TIMEOUT); return; }
-    }
-}
-
-// Warp-uniform bounded wait: every lane polls, the warp proceeds only if all saw it.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
-    const bool ok = mbar_wait(bar, parity, abort);
-    return __all_sync(0xffffffffu, ok);
-}
 
 // Insert (v, id) into a list sorted by value descending; equal values keep the
 // earlier (lower) id first.  Static indices only, so the list stays in registers.
@@ -142,26 +103,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int q = 0; q < kNQ; ++q) nt = max(nt, ntq[q]);
 
-    auto bar = [&](int i) { return base + kBarOff + 8u * i; };
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + kMiscOff + 4);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kMiscOff);
+    auto bar = [&](int i) { return base + L::kBarOff + 8u * i; };
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::kMiscOff + 4);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::kMiscOff);
 
     if (threadIdx.x == 0) {
-        mbar_init(bar(BQ), 1);
-        for (int i = 0; i < kKV; ++i) { mbar_init(bar(BKVF + i), 1); mbar_init(bar(BKVE + i), 1); }
-        for (int i = 0; i < 2 * kNQ; ++i) {
-            mbar_init(bar(BSF + i), 1);
-            mbar_init(bar(BSE + i), 4);
-            mbar_init(bar(BPF + i), 4);
-            mbar_init(bar(BPVD + i), 1);
-        }
-        mbar_init(bar(BOF), 1);
-        mbar_init(bar(BDRAIN), 1);
+        fl::init_barriers<L>(base + L::kBarOff);
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(base + kMiscOff, kTmemCols);
+        tmem_alloc(base + L::kMiscOff, L::kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -170,100 +122,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            prefetch_tmap(&tmap_q);
-            prefetch_tmap(&tmap_k);
-            prefetch_tmap(&tmap_v);
-            mbar_arrive_expect_tx(bar(BQ), kNQ * 32768);
-#pragma unroll
-            for (int q = 0; q < kNQ; ++q) {
-                tma_load_4d(base + kQOff + q * 32768, &tmap_q, bar(BQ), 0, row0 + q * P, u * g, b);
-                tma_load_4d(base + kQOff + q * 32768 + 16384, &tmap_q, bar(BQ), 64, row0 + q * P,
-                            u * g, b);
-            }
-            int issued = 0;
-            for (int j = 0; j < nt; ++j) {
-                const int st = j % kKV;
-                if (j >= kKV &&
-                    !mbar_wait(bar(BKVE + st), ((j / kKV) - 1) & 1, abort_flag, kRoleSleep))
-                    break;
-                const uint32_t f = bar(BKVF + st);
-                mbar_arrive_expect_tx(f, 4 * 8192);
-                const uint32_t kd = base + kKOff + st * 16384, vd = base + kVOff + st * 16384;
-                const int key0 = j * kBN;
-                tma_load_3d(kd, &tmap_k, f, 0, key0, bu);
-                tma_load_3d(kd + 8192, &tmap_k, f, 64, key0, bu);
-                tma_load_3d(vd, &tmap_v, f, 0, key0, bu);
-                tma_load_3d(vd + 8192, &tmap_v, f, 64, key0, bu);
-                issued = j + 1;
-            }
-            // every issued load must have landed before the CTA may exit
-            mbar_drain(bar(BQ), 0);
-            for (int j = max(0, issued - kKV); j < issued; ++j)
-                mbar_drain(bar(BKVF + j % kKV), (j / kKV) & 1);
-        }
+        if (lane == 0)
+            fl::producer<L>(base, &tmap_q, &tmap_k, &tmap_v, row0, P, u * g, b, bu, nt,
+                            [](int j) { return j * kBN; }, abort_flag);
     } else if (warp == 1) {
-        // ------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t id_s = idesc_bf16(kBM, kBN, false, false);
-            const uint32_t id_o = idesc_bf16(kBM, kD, false, true);
-            bool ok = mbar_wait(bar(BQ), 0, abort_flag, kRoleSleep);
-            tc_fence_after();
-            for (int j = 0; ok && j <= nt; ++j) {
-                if (j < nt) {
-                    const int st = j % kKV, s = j & 1;
-                    if (!mbar_wait(bar(BKVF + st), (j / kKV) & 1, abort_flag, kRoleSleep)) break;
-                    const uint32_t kb = base + kKOff + st * 16384;
-#pragma unroll
-                    for (int q = 0; q < kNQ; ++q) {
-                        if (j >= ntq[q]) continue;
-                        if (j >= 2 && !mbar_wait(bar(BSE + 2 * q + s), ((j >> 1) - 1) & 1,
-                                                 abort_flag, kRoleSleep)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t qb = base + kQOff + q * 32768;
-#pragma unroll
-                        for (int kk = 0; kk < kD / 16; ++kk) {
-                            const uint64_t ad = sw128_desc(qb + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                            const uint64_t bd = sw128_desc(kb + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-                            umma_ss(tmem + q * 256 + 64 * s, ad, bd, id_s, kk > 0 ? 1u : 0u);
-                        }
-                        umma_commit(bar(BSF + 2 * q + s));
-                    }
-                    if (!ok) break;
-                }
-                if (j >= 1) {
-                    const int jj = j - 1, sp = jj & 1, stp = jj % kKV;
-                    const uint32_t vb = base + kVOff + stp * 16384;
-#pragma unroll
-                    for (int q = 0; q < kNQ; ++q) {
-                        if (jj >= ntq[q]) continue;
-                        if (!mbar_wait(bar(BPF + 2 * q + sp), (jj >> 1) & 1, abort_flag,
-                                       kRoleSleep)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t pb = base + kPOff + (2 * q + sp) * 16384;
-#pragma unroll
-                        for (int kk = 0; kk < kBN / 16; ++kk) {
-                            const uint64_t ad = sw128_desc(pb + kk * 32, 16, 1024);
-                            const uint64_t bd = sw128_desc(vb + kk * 2048, 8192, 1024);
-                            umma_ss(tmem + q * 256 + 128, ad, bd, id_o, (jj > 0 || kk > 0) ? 1u : 0u);
-                        }
-                        umma_commit(bar(BPVD + 2 * q + sp));
-                    }
-                    if (!ok) break;
-                    umma_commit(bar(BKVE + stp));
-                }
-            }
-            umma_commit(bar(BOF));
-            umma_commit(bar(BDRAIN));
-            mbar_drain(bar(BDRAIN), 0);
-        }
+        if (lane == 0) fl::mma_issuer<L>(base, tmem, nt, ntq, abort_flag);
     } else {
         // ------------------------------------------------------ softmax
         const int q = (warp - 2) >> 2;   // warpgroup = Q tile
@@ -272,8 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16) + q * 256;
         const int hh = row / P, pr = row % P;
         const int qrow0 = row0 + q * P;              // first query row of this Q tile
-        const int pos_first = p.q_offset + qrow0;    // its position
-        const int pos = pos_first + pr;
+        const int pos = p.q_offset + qrow0 + pr;
         const int nt_me = ntq[q];
         const float sl2 = p.scale_log2;
         float m_ref = -INFINITY, l = 0.f;
@@ -284,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int j = 0; j < nt_me; ++j) {
             const int s = j & 1;
-            if (!warp_wait(bar(BSF + 2 * q + s), (j >> 1) & 1, abort_flag)) { ok = false; break; }
+            if (!fl::warp_wait(bar(L::BSF + 2 * q + s), (j >> 1) & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             uint32_t r[64];
             tmem_ld32(trow + 64 * s, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
@@ -292,113 +154,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(BSE + 2 * q + s));
+            if (lane == 0) mbar_arrive(bar(L::BSE + 2 * q + s));
 
-            const int key0 = j * kBN;
-            float x[64];
-#pragma unroll
-            for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(r[c]);
-            if (key0 + kBN - 1 > pos_first) {  // diagonal tile: causal mask per row
-                const int lim = pos - key0;
-#pragma unroll
-                for (int c = 0; c < 64; ++c) x[c] = c <= lim ? x[c] : -INFINITY;
-            }
-            // tile max of the raw logits (tree), then to the log2 domain
-            float mx[16];
-#pragma unroll
-            for (int c = 0; c < 16; ++c)
-                mx[c] = fmaxf(fmaxf(x[c], x[c + 16]), fmaxf(x[c + 32], x[c + 48]));
-#pragma unroll
-            for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-                for (int c = 0; c < w; ++c) mx[c] = fmaxf(mx[c], mx[c + w]);
-            const float mt = mx[0] * sl2;  // -inf stays -inf (sl2 > 0)
-            if (a.capture && mt > -INFINITY) list_insert(lv, li, mt, j);
-            // lazy rescale: keep the reference max unless the tile exceeds it by 2^8
-            bool resc = false;
-            float corr = 1.f;
-            if (mt > m_ref + 8.f) {
-                corr = ex2(m_ref - mt);  // 0 on the first tile
-                resc = j > 0;
-                m_ref = mt;
-                l *= corr;
-            }
-            // p = 2^(x * scale_log2 - m): packed FFMA for the arguments and
-            // packed adds for the row sum
-            const float2 s2 = make_float2(sl2, sl2), n2 = make_float2(-m_ref, -m_ref);
-            float e[64];
-            float2 acc[8];
-#pragma unroll
-            for (int c2 = 0; c2 < 32; ++c2) {
-                const float2 y = ffma2(make_float2(x[2 * c2], x[2 * c2 + 1]), s2, n2);
-                e[2 * c2] = ex2(y.x);
-                e[2 * c2 + 1] = ex2(y.y);
-                const float2 ev = make_float2(e[2 * c2], e[2 * c2 + 1]);
-                acc[c2 & 7] = c2 < 8 ? ev : fadd2(acc[c2 & 7], ev);
-            }
-#pragma unroll
-            for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-                for (int c = 0; c < w; ++c) acc[c] = fadd2(acc[c], acc[c + w]);
-            l += acc[0].x + acc[0].y;
+            // causal: keys <= pos (only the diagonal tile masks anything)
+            float mt, corr;
             uint32_t pk[32];
-#pragma unroll
-            for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(e[2 * c], e[2 * c + 1]);
+            const bool resc = fl::softmax_tile(r, 0, pos - j * kBN, sl2, m_ref, l, mt, corr, pk);
+            if (a.capture && mt > -INFINITY) list_insert(lv, li, mt, j);
             // P buffer s of this tile is free once the PV of tile j-2 is done
-            if (j >= 2 && !warp_wait(bar(BPVD + 2 * q + s), ((j >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
-            unsigned char* prow = gbase + kPOff + (2 * q + s) * 16384 + row * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint4 v4 = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-                *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) = v4;
-            }
-            fence_proxy_async_smem();
+            if (j >= 2 && !fl::warp_wait(bar(L::BPVD + 2 * q + s), ((j >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+            fl::store_p(gbase + L::kPOff + (2 * q + s) * 16384, row, pk);
             if (__any_sync(0xffffffffu, resc)) {
                 // O may only be touched once the PV of tile j-1 has finished
-                if (!warp_wait(bar(BPVD + 2 * q + (s ^ 1)), ((j - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+                if (!fl::warp_wait(bar(L::BPVD + 2 * q + (s ^ 1)), ((j - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                const float cf = resc ? corr : 1.f;
-#pragma unroll
-                for (int c4 = 0; c4 < kD / 32; ++c4) {
-                    uint32_t ro[32];
-                    tmem_ld32(trow + 128 + 32 * c4, ro);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) ro[c] = __float_as_uint(__uint_as_float(ro[c]) * cf);
-                    tmem_st32(trow + 128 + 32 * c4, ro);
-                }
-                tmem_wait_st();
+                fl::rescale_o(trow + 128, resc ? corr : 1.f);
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(BPF + 2 * q + s));
+            if (lane == 0) mbar_arrive(bar(L::BPF + 2 * q + s));
         }
-        if (ok && nt_me > 0) ok = warp_wait(bar(BOF), 0, abort_flag);
+        if (ok && nt_me > 0) ok = fl::warp_wait(bar(L::BOF), 0, abort_flag);
         const bool row_ok = nt_me > 0 && qrow0 + pr < p.t_q;
         const int h = u * g + hh;
         const size_t orow = ((size_t)b * p.hq + h) * p.t_q + qrow0 + pr;
         const float lse2 = m_ref + log2f(l);
         if (ok && nt_me > 0) {
             tc_fence_after();
-            const float inv = 1.f / l;
-            __nv_bfloat16* og = a.o + orow * kD;
-#pragma unroll
-            for (int c4 = 0; c4 < kD / 32; ++c4) {
-                uint32_t ro[32];
-                tmem_ld32(trow + 128 + 32 * c4, ro);
-                tmem_wait_ld();
-                if (row_ok) {
-#pragma unroll
-                    for (int c = 0; c < 32; c += 8) {
-                        uint4 v4;
-                        v4.x = pack_bf16(__uint_as_float(ro[c]) * inv, __uint_as_float(ro[c + 1]) * inv);
-                        v4.y = pack_bf16(__uint_as_float(ro[c + 2]) * inv, __uint_as_float(ro[c + 3]) * inv);
-                        v4.z = pack_bf16(__uint_as_float(ro[c + 4]) * inv, __uint_as_float(ro[c + 5]) * inv);
-                        v4.w = pack_bf16(__uint_as_float(ro[c + 6]) * inv, __uint_as_float(ro[c + 7]) * inv);
-                        *reinterpret_cast<uint4*>(og + c4 * 32 + c) = v4;
-                    }
-                }
-            }
+            fl::store_o(trow + 128, true, 1.f / l, row_ok, a.o + orow * kD);
             if (row_ok) a.lse[orow] = lse2 * kLn2;
         }
         if (a.capture) {
@@ -410,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // on all 128 threads: a group of g consecutive lanes per position,
             // lane hh holding the front of head hh's list; each step the group
             // finds its best front with in-group shuffles and that lane moves on.
-            unsigned char* reg = gbase + kPOff + q * 32768;    // this tile's P buffers
+            unsigned char* reg = gbase + L::kPOff + q * 32768;    // this tile's P buffers
             float* cs = reinterpret_cast<float*>(reg);         // [128][kList]
             int* ci = reinterpret_cast<int*>(reg + 128 * kList * 4);
             // every PV has completed (BOF), so the P buffers are free to reuse
@@ -489,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, L::kTmemCols);
     }
 }
 

@@ -23,6 +23,7 @@
 // over the layer's own K'/V' (keys t-w+1..t) is a second launch of the same
 // kernel whose block list is the contiguous run the CTA's windows touch.
 #include "cta_select.cuh"
+#include "flash_tc.cuh"
 #include "hs_common.cuh"
 #include "hs_kernels.cuh"
 #include "tc_ptx.cuh"
@@ -32,36 +33,14 @@ namespace stc {
 
 using namespace tc;
 
-constexpr int kBM = 128;       // rows per Q tile
-constexpr int kNQ = 2;         // Q tiles per CTA
-constexpr int kBN = 64;        // keys per tile = block size
-constexpr int kD = 128;
-constexpr int kKV = 2;         // K/V ring stages
 constexpr int kMaxSel = 16;    // selected blocks per row held in registers
 constexpr int kMaxUnion = 1024;
-constexpr int kThreads = 64 + 128 * kNQ;
-
-constexpr uint32_t kQOff = 0;                          // kNQ x 32 KB
-constexpr uint32_t kKOff = kNQ * 32768;                // kKV x 16 KB
-constexpr uint32_t kVOff = kKOff + kKV * 16384;        // kKV x 16 KB
-constexpr uint32_t kPOff = kVOff + kKV * 16384;        // kNQ x 2 x 16 KB (block bitmap first)
-constexpr uint32_t kUOff = kPOff + kNQ * 2 * 16384;    // union block ids, kMaxUnion ints
-constexpr uint32_t kBarOff = kUOff + kMaxUnion * 4;
-enum {
-    BQ = 0,
-    BKVF = 1,
-    BKVE = BKVF + kKV,
-    BSF = BKVE + kKV,  // [q][s]
-    BSE = BSF + 2 * kNQ,
-    BPF = BSE + 2 * kNQ,
-    BPVD = BPF + 2 * kNQ,
-    BOF = BPVD + 2 * kNQ,
-    BDRAIN = BOF + 1,
-    BCOUNT = BDRAIN + 1
-};
-constexpr uint32_t kMiscOff = kBarOff + BCOUNT * 8;  // tmem(4) abort(4) U(4) pad(4) scan[16]
-constexpr uint32_t kSmemBytes = kMiscOff + 16 + 64 + 1024;
-constexpr uint32_t kTmemCols = 256 * kNQ;
+using L = fl::Layout<2, kMaxUnion * 4>;  // 2-stage K/V ring; the union block list after P
+constexpr int kBM = L::kBM, kNQ = L::kNQ, kBN = L::kBN, kD = L::kD;
+constexpr int kThreads = L::kThreads;
+constexpr uint32_t kUOff = L::kExtraOff;                  // union block ids, kMaxUnion ints
+// misc: tmem(4) abort(4) U(4) pad(4) scan[16]
+constexpr uint32_t kSmemBytes = L::kMiscOff + 16 + 64 + 1024;
 constexpr uint32_t kBitmapWords = kNQ * 2 * 16384 / 4;  // blocks the union bitmap covers / 32
 static_assert(kSmemBytes <= 232448, "shared memory");
 
@@ -99,31 +78,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n_blocks = (p.q_offset + last_row) / kBN + 1;  // blocks any row may select
     const int win_b0 = max(0, p.q_offset + row0 - p.window + 1) / kBN;  // first window block
 
-    auto bar = [&](int i) { return base + kBarOff + 8u * i; };
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kMiscOff);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + kMiscOff + 4);
-    int* s_union = reinterpret_cast<int*>(gbase + kMiscOff + 8);
-    int* s_scan = reinterpret_cast<int*>(gbase + kMiscOff + 16);
-    uint32_t* bitmap = reinterpret_cast<uint32_t*>(gbase + kPOff);  // prologue only
+    auto bar = [&](int i) { return base + L::kBarOff + 8u * i; };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::kMiscOff);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::kMiscOff + 4);
+    int* s_union = reinterpret_cast<int*>(gbase + L::kMiscOff + 8);
+    int* s_scan = reinterpret_cast<int*>(gbase + L::kMiscOff + 16);
+    uint32_t* bitmap = reinterpret_cast<uint32_t*>(gbase + L::kPOff);  // prologue only
     int* ulist = reinterpret_cast<int*>(gbase + kUOff);
     const int words = kWin ? 0 : (n_blocks + 31) >> 5;
 
     if (threadIdx.x == 0) {
-        mbar_init(bar(BQ), 1);
-        for (int i = 0; i < kKV; ++i) { mbar_init(bar(BKVF + i), 1); mbar_init(bar(BKVE + i), 1); }
-        for (int i = 0; i < 2 * kNQ; ++i) {
-            mbar_init(bar(BSF + i), 1);
-            mbar_init(bar(BSE + i), 4);
-            mbar_init(bar(BPF + i), 4);
-            mbar_init(bar(BPVD + i), 1);
-        }
-        mbar_init(bar(BOF), 1);
-        mbar_init(bar(BDRAIN), 1);
+        fl::init_barriers<L>(base + L::kBarOff);
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(base + kMiscOff, kTmemCols);
+        tmem_alloc(base + L::kMiscOff, L::kTmemCols);
         tmem_relinquish();
     }
     for (int x = threadIdx.x; x < words; x += blockDim.x) bitmap[x] = 0u;
@@ -192,97 +162,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nt = U;
 
     if (warp == 0) {
-        // ------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            prefetch_tmap(&tmap_q);
-            prefetch_tmap(&tmap_k);
-            prefetch_tmap(&tmap_v);
-            mbar_arrive_expect_tx(bar(BQ), kNQ * 32768);
-#pragma unroll
-            for (int qq = 0; qq < kNQ; ++qq) {
-                tma_load_4d(base + kQOff + qq * 32768, &tmap_q, bar(BQ), 0, row0 + qq * P, u * g, b);
-                tma_load_4d(base + kQOff + qq * 32768 + 16384, &tmap_q, bar(BQ), 64,
-                            row0 + qq * P, u * g, b);
-            }
-            int issued = 0;
-            for (int j = 0; j < nt; ++j) {
-                const int st = j % kKV;
-                if (j >= kKV && !mbar_wait(bar(BKVE + st), ((j / kKV) - 1) & 1, abort_flag, false))
-                    break;
-                const uint32_t f = bar(BKVF + st);
-                mbar_arrive_expect_tx(f, 4 * 8192);
-                const uint32_t kd = base + kKOff + st * 16384, vd = base + kVOff + st * 16384;
-                const int key0 = (kWin ? win_b0 + j : ulist[j]) * kBN;
-                tma_load_3d(kd, &tmap_k, f, 0, key0, bu);
-                tma_load_3d(kd + 8192, &tmap_k, f, 64, key0, bu);
-                tma_load_3d(vd, &tmap_v, f, 0, key0, bu);
-                tma_load_3d(vd + 8192, &tmap_v, f, 64, key0, bu);
-                issued = j + 1;
-            }
-            mbar_drain(bar(BQ), 0);
-            for (int j = max(0, issued - kKV); j < issued; ++j)
-                mbar_drain(bar(BKVF + j % kKV), (j / kKV) & 1);
-        }
+        if (lane == 0)
+            fl::producer<L>(base, &tmap_q, &tmap_k, &tmap_v, row0, P, u * g, b, bu, nt,
+                            [&](int j) { return (kWin ? win_b0 + j : ulist[j]) * kBN; }, abort_flag);
     } else if (warp == 1) {
-        // ------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t id_s = idesc_bf16(kBM, kBN, false, false);
-            const uint32_t id_o = idesc_bf16(kBM, kD, false, true);
-            bool ok = mbar_wait(bar(BQ), 0, abort_flag, false);
-            tc_fence_after();
-            for (int j = 0; ok && j <= nt; ++j) {
-                if (j < nt) {
-                    const int st = j % kKV, s = j & 1;
-                    if (!mbar_wait(bar(BKVF + st), (j / kKV) & 1, abort_flag, false)) break;
-                    const uint32_t kb = base + kKOff + st * 16384;
-#pragma unroll
-                    for (int qq = 0; qq < kNQ; ++qq) {
-                        if (j >= ntq[qq]) continue;
-                        if (j >= 2 && !mbar_wait(bar(BSE + 2 * qq + s), ((j >> 1) - 1) & 1,
-                                                 abort_flag, false)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t qb = base + kQOff + qq * 32768;
-#pragma unroll
-                        for (int kk = 0; kk < kD / 16; ++kk) {
-                            const uint64_t ad = sw128_desc(qb + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                            const uint64_t bd = sw128_desc(kb + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-                            umma_ss(tmem + qq * 256 + 64 * s, ad, bd, id_s, kk > 0 ? 1u : 0u);
-                        }
-                        umma_commit(bar(BSF + 2 * qq + s));
-                    }
-                    if (!ok) break;
-                }
-                if (j >= 1) {
-                    const int jj = j - 1, sp = jj & 1, stp = jj % kKV;
-                    const uint32_t vb = base + kVOff + stp * 16384;
-#pragma unroll
-                    for (int qq = 0; qq < kNQ; ++qq) {
-                        if (jj >= ntq[qq]) continue;
-                        if (!mbar_wait(bar(BPF + 2 * qq + sp), (jj >> 1) & 1, abort_flag, false)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t pb = base + kPOff + (2 * qq + sp) * 16384;
-#pragma unroll
-                        for (int kk = 0; kk < kBN / 16; ++kk) {
-                            const uint64_t ad = sw128_desc(pb + kk * 32, 16, 1024);
-                            const uint64_t bd = sw128_desc(vb + kk * 2048, 8192, 1024);
-                            umma_ss(tmem + qq * 256 + 128, ad, bd, id_o, (jj > 0 || kk > 0) ? 1u : 0u);
-                        }
-                        umma_commit(bar(BPVD + 2 * qq + sp));
-                    }
-                    if (!ok) break;
-                    umma_commit(bar(BKVE + stp));
-                }
-            }
-            umma_commit(bar(BOF));
-            umma_commit(bar(BDRAIN));
-            mbar_drain(bar(BDRAIN), 0);
-        }
+        if (lane == 0) fl::mma_issuer<L>(base, tmem, nt, ntq, abort_flag);
     } else {
         // ------------------------------------------------------ softmax
         const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16) + q * 256;
@@ -292,7 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int j = 0; j < nt_me; ++j) {
             const int s = j & 1;
-            if (!warp_wait(bar(BSF + 2 * q + s), (j >> 1) & 1, abort_flag)) { ok = false; break; }
+            if (!fl::warp_wait(bar(L::BSF + 2 * q + s), (j >> 1) & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             uint32_t r[64];
             tmem_ld32(trow + 64 * s, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
@@ -300,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(BSE + 2 * q + s));
+            if (lane == 0) mbar_arrive(bar(L::BSE + 2 * q + s));
 
             // global: this row keeps the block only if it selected it, and keys
             // <= t; window: keys t-w+1..t
@@ -313,108 +197,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const int lim = (sel && row_valid) ? pos - key0 : -1;  // last kept column
             const int first = kWin ? pos - p.window + 1 - key0 : 0;  // first kept column
-            float x[64];
-#pragma unroll
-            for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(r[c]);
-            if (lim < kBN - 1 || first > 0) {
-#pragma unroll
-                for (int c = 0; c < 64; ++c) x[c] = (c <= lim && c >= first) ? x[c] : -INFINITY;
-            }
-            float m3[22];
-#pragma unroll
-            for (int c = 0; c < 21; ++c) m3[c] = max3f(x[3 * c], x[3 * c + 1], x[3 * c + 2]);
-            m3[21] = x[63];
-#pragma unroll
-            for (int c = 0; c < 7; ++c) m3[c] = max3f(m3[3 * c], m3[3 * c + 1], m3[3 * c + 2]);
-            const float mt = max3f(max3f(m3[0], m3[1], m3[2]), max3f(m3[3], m3[4], m3[5]),
-                                   fmaxf(m3[6], m3[21])) * sl2;  // -inf stays -inf
-            // lazy rescale; a row may see no kept key for a while (m_ref = -inf)
-            bool resc = false;
-            float corr = 1.f;
-            if (mt > m_ref + 8.f) {
-                corr = ex2(m_ref - mt);  // 0 while nothing was kept
-                resc = m_ref > -INFINITY;
-                m_ref = mt;
-                l *= corr;
-            }
-            const float mu = m_ref == -INFINITY ? 0.f : m_ref;
-            const float2 s2 = make_float2(sl2, sl2), n2 = make_float2(-mu, -mu);
-            float e[64];
-            float2 acc[8];
-#pragma unroll
-            for (int c2 = 0; c2 < 32; ++c2) {
-                const float2 y = ffma2(make_float2(x[2 * c2], x[2 * c2 + 1]), s2, n2);
-                e[2 * c2] = ex2(y.x);
-                e[2 * c2 + 1] = ex2(y.y);
-                const float2 ev = make_float2(e[2 * c2], e[2 * c2 + 1]);
-                acc[c2 & 7] = c2 < 8 ? ev : fadd2(acc[c2 & 7], ev);
-            }
-#pragma unroll
-            for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-                for (int c = 0; c < w; ++c) acc[c] = fadd2(acc[c], acc[c + w]);
-            l += acc[0].x + acc[0].y;
+            // a row may see no kept key for a while (m_ref = -inf)
+            float mt, corr;
             uint32_t pk[32];
-#pragma unroll
-            for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(e[2 * c], e[2 * c + 1]);
+            const bool resc = fl::softmax_tile(r, first, lim, sl2, m_ref, l, mt, corr, pk);
             // P buffer s is free once the PV of tile j-2 is done
-            if (j >= 2 && !warp_wait(bar(BPVD + 2 * q + s), ((j >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
-            unsigned char* prow = gbase + kPOff + (2 * q + s) * 16384 + row * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint4 v4 = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-                *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) = v4;
-            }
-            fence_proxy_async_smem();
+            if (j >= 2 && !fl::warp_wait(bar(L::BPVD + 2 * q + s), ((j >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+            fl::store_p(gbase + L::kPOff + (2 * q + s) * 16384, row, pk);
             if (__any_sync(0xffffffffu, resc)) {
                 // O may only be touched once the PV of tile j-1 has finished
-                if (!warp_wait(bar(BPVD + 2 * q + (s ^ 1)), ((j - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+                if (!fl::warp_wait(bar(L::BPVD + 2 * q + (s ^ 1)), ((j - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                const float cf = resc ? corr : 1.f;
-#pragma unroll
-                for (int c4 = 0; c4 < kD / 32; ++c4) {
-                    uint32_t ro[32];
-                    tmem_ld32(trow + 128 + 32 * c4, ro);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) ro[c] = __float_as_uint(__uint_as_float(ro[c]) * cf);
-                    tmem_st32(trow + 128 + 32 * c4, ro);
-                }
-                tmem_wait_st();
+                fl::rescale_o(trow + 128, resc ? corr : 1.f);
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(BPF + 2 * q + s));
+            if (lane == 0) mbar_arrive(bar(L::BPF + 2 * q + s));
         }
-        if (ok && nt_me > 0) ok = warp_wait(bar(BOF), 0, abort_flag);
+        if (ok && nt_me > 0) ok = fl::warp_wait(bar(L::BOF), 0, abort_flag);
         const size_t orow = ((size_t)b * p.hq + u * g + hh) * p.t_q + qrow0 + pr;
         if (ok) {  // warp-uniform; the TMEM loads run on every lane of the warp
             if (nt_me > 0) tc_fence_after();
             const bool any = l > 0.f;
             const float inv = any ? 1.f / l : 0.f;
-            __nv_bfloat16* og = a.o + orow * kD;
-#pragma unroll
-            for (int c4 = 0; c4 < kD / 32; ++c4) {
-                uint32_t ro[32];
-                if (nt_me > 0) {
-                    tmem_ld32(trow + 128 + 32 * c4, ro);
-                    tmem_wait_ld();
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) ro[c] = 0u;
-                }
-                if (row_valid) {
-#pragma unroll
-                    for (int c = 0; c < 32; c += 8) {
-                        uint4 v4;
-                        v4.x = pack_bf16(__uint_as_float(ro[c]) * inv, __uint_as_float(ro[c + 1]) * inv);
-                        v4.y = pack_bf16(__uint_as_float(ro[c + 2]) * inv, __uint_as_float(ro[c + 3]) * inv);
-                        v4.z = pack_bf16(__uint_as_float(ro[c + 4]) * inv, __uint_as_float(ro[c + 5]) * inv);
-                        v4.w = pack_bf16(__uint_as_float(ro[c + 6]) * inv, __uint_as_float(ro[c + 7]) * inv);
-                        *reinterpret_cast<uint4*>(og + c4 * 32 + c) = v4;
-                    }
-                }
-            }
+            fl::store_o(trow + 128, nt_me > 0, inv, row_valid, a.o + orow * kD);
             if (row_valid) a.lse[orow] = any ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
         }
     }
@@ -424,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, L::kTmemCols);
     }
 }
 

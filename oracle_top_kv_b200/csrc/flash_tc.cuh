@@ -2,8 +2,9 @@
 // layer (full_tc.cu) and the row-grouped sparse layer (sparse_tc.cu).
 //
 // A CTA runs two 128-row Q tiles over a list of 64-key tiles that both share.
-// Warp 0 is the TMA producer, warp 1 owns TMEM and issues the MMAs from one
-// thread, warps 2..9 are two softmax warpgroups with one thread per row:
+// Warp 0 is the TMA producer, warp 1 owns TMEM, warps 2..9 are two softmax
+// warpgroups with one thread per row, and one thread per Q tile (warp 1 for
+// tile 0, warp 10 for tile 1) issues that tile's MMAs:
 //   S = Q K^T  (M = 128, N = 64, K = 16 x 8) into one of two TMEM buffers,
 //   O += P V   (N = 128, V as the MN-major operand; P from shared memory).
 // The kernels differ in which key tiles they visit, which keys a row keeps,
@@ -23,7 +24,8 @@ using namespace tc;
 template <int KV, uint32_t Extra>
 struct Layout {
     static constexpr int kBM = 128, kNQ = 2, kBN = 64, kD = 128, kKV = KV;
-    static constexpr int kThreads = 64 + 128 * kNQ;
+    static constexpr int kIssuer1Warp = 2 + 4 * kNQ;               // issuer of Q tile 1
+    static constexpr int kThreads = 64 + 128 * kNQ + 32 * (kNQ - 1);
     static constexpr uint32_t kQOff = 0;                       // kNQ x 32 KB (two d halves)
     static constexpr uint32_t kKOff = kNQ * 32768;             // KV x 16 KB
     static constexpr uint32_t kVOff = kKOff + KV * 16384;      // KV x 16 KB
@@ -38,12 +40,15 @@ struct Layout {
         BSE = BSF + 2 * kNQ,
         BPF = BSE + 2 * kNQ,
         BPVD = BPF + 2 * kNQ,
-        BOF = BPVD + 2 * kNQ,
-        BDRAIN = BOF + 1,
-        BCOUNT = BDRAIN + 1
+        BOF = BPVD + 2 * kNQ,   // [q]: O of Q tile q is final
+        BDRAIN = BOF + kNQ,     // [q]: issuer q's MMAs are done
+        BCOUNT = BDRAIN + kNQ
     };
     static constexpr uint32_t kMiscOff = kBarOff + BCOUNT * 8;  // tmem slot, abort flag, ...
     static constexpr uint32_t kTmemCols = 256 * kNQ;            // per Q tile: S0 | S1 | O
+    // every operand lies below 256 KB, so a descriptor's 14-bit addr >> 4 field never wraps
+    static_assert(kMiscOff + 1024 <= 232448, "shared memory");
+    static_assert(kNQ == 2, "one issuer warp per Q tile: warps 1 and 2 + 4 kNQ");
 };
 
 // Bounded wait that ignores the abort flag (used to drain in-flight work).
@@ -64,15 +69,15 @@ template <class L>
 __device__ __forceinline__ void init_barriers(uint32_t bar0) {
     auto bar = [&](int i) { return bar0 + 8u * i; };
     mbar_init(bar(L::BQ), 1);
-    for (int i = 0; i < L::kKV; ++i) { mbar_init(bar(L::BKVF + i), 1); mbar_init(bar(L::BKVE + i), 1); }
+    // a K/V stage is free once both issuers' PV MMAs that read it are done
+    for (int i = 0; i < L::kKV; ++i) { mbar_init(bar(L::BKVF + i), 1); mbar_init(bar(L::BKVE + i), L::kNQ); }
     for (int i = 0; i < 2 * L::kNQ; ++i) {
         mbar_init(bar(L::BSF + i), 1);
         mbar_init(bar(L::BSE + i), 4);
         mbar_init(bar(L::BPF + i), 4);
         mbar_init(bar(L::BPVD + i), 1);
     }
-    mbar_init(bar(L::BOF), 1);
-    mbar_init(bar(L::BDRAIN), 1);
+    for (int q = 0; q < L::kNQ; ++q) { mbar_init(bar(L::BOF + q), 1); mbar_init(bar(L::BDRAIN + q), 1); }
 }
 
 // TMA producer (one thread): both Q tiles once (4-D boxes: 64 d x P positions
@@ -112,68 +117,66 @@ __device__ __forceinline__ void producer(uint32_t base, const CUtensorMap* tq, c
         mbar_drain(bar(L::BKVF + j % L::kKV), (j / L::kKV) & 1);
 }
 
-// MMA issuer (one thread): iteration j issues S = Q K^T of tile j for both Q
-// tiles (each waits for its S buffer), then O += P V of tile j-1 (each waits
-// for its P), and releases tile j-1's K/V stage.  Q tile q uses ntq[q] tiles.
+// MMA issuer of Q tile q (one thread): iteration j issues S = Q K^T of tile j
+// (after its S buffer is free), then O += P V of tile j-1 (after its P is
+// ready), and releases tile j-1's K/V stage.  The Q tile uses ntq of the CTA's
+// nt tiles; for the rest it still waits for each stage to fill before
+// releasing it, so its release of a stage can never count towards a later
+// use of that stage than the other issuer's.
+// One thread's instruction stream bounds the MMA rate, hence one issuer per Q
+// tile and shared-memory descriptors built once: a descriptor holds its start
+// address as addr >> 4 in its low 14 bits, and every operand of the CTA lies
+// below 256 KB, so moving an operand by `off` bytes adds off >> 4.
 template <class L>
-__device__ __forceinline__ void mma_issuer(uint32_t base, uint32_t tmem, int nt,
-                                           const int (&ntq)[L::kNQ], volatile int* abort) {
+__device__ __forceinline__ void mma_issuer(uint32_t base, uint32_t tmem, int q, int nt, int ntq,
+                                           volatile int* abort) {
     auto bar = [&](int i) { return base + L::kBarOff + 8u * i; };
     const uint32_t id_s = idesc_bf16(L::kBM, L::kBN, false, false);
     const uint32_t id_o = idesc_bf16(L::kBM, L::kD, false, true);
+    const uint64_t dq = sw128_desc(base + L::kQOff + q * 32768, 16, 1024);
+    const uint64_t dk0 = sw128_desc(base + L::kKOff, 16, 1024);
+    const uint64_t dp0 = sw128_desc(base + L::kPOff + q * 32768, 16, 1024);
+    const uint64_t dv0 = sw128_desc(base + L::kVOff, 8192, 1024);  // V: MN-major, d halves 8 KB apart
+    const uint32_t ts = tmem + q * 256, to = tmem + q * 256 + 128;
     bool ok = mbar_wait(bar(L::BQ), 0, abort, false);
     tc_fence_after();
     for (int j = 0; ok && j <= nt; ++j) {
         if (j < nt) {
             const int st = j % L::kKV, s = j & 1;
             if (!mbar_wait(bar(L::BKVF + st), (j / L::kKV) & 1, abort, false)) break;
-            const uint32_t kb = base + L::kKOff + st * 16384;
-#pragma unroll
-            for (int q = 0; q < L::kNQ; ++q) {
-                if (j >= ntq[q]) continue;
-                if (j >= 2 && !mbar_wait(bar(L::BSE + 2 * q + s), ((j >> 1) - 1) & 1, abort, false)) {
-                    ok = false;
-                    break;
-                }
+            if (j < ntq) {
+                if (j >= 2 && !mbar_wait(bar(L::BSE + 2 * q + s), ((j >> 1) - 1) & 1, abort, false)) break;
                 tc_fence_after();
-                const uint32_t qb = base + L::kQOff + q * 32768;
+                const uint64_t dk = dk0 + (uint64_t)(st * (16384 >> 4));
+                // K step kk: d columns 16kk.. = 32-byte column group kk&3 of d half kk>>2
 #pragma unroll
-                for (int kk = 0; kk < L::kD / 16; ++kk) {
-                    const uint64_t ad = sw128_desc(qb + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                    const uint64_t bd = sw128_desc(kb + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-                    umma_ss(tmem + q * 256 + 64 * s, ad, bd, id_s, kk > 0 ? 1u : 0u);
-                }
+                for (int kk = 0; kk < L::kD / 16; ++kk)
+                    umma_ss(ts + 64 * s, dq + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                            dk + (uint64_t)(((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), id_s,
+                            kk > 0 ? 1u : 0u);
                 umma_commit(bar(L::BSF + 2 * q + s));
             }
-            if (!ok) break;
         }
         if (j >= 1) {
             const int jj = j - 1, sp = jj & 1, stp = jj % L::kKV;
-            const uint32_t vb = base + L::kVOff + stp * 16384;
-#pragma unroll
-            for (int q = 0; q < L::kNQ; ++q) {
-                if (jj >= ntq[q]) continue;
-                if (!mbar_wait(bar(L::BPF + 2 * q + sp), (jj >> 1) & 1, abort, false)) {
-                    ok = false;
-                    break;
-                }
+            if (jj < ntq) {
+                if (!mbar_wait(bar(L::BPF + 2 * q + sp), (jj >> 1) & 1, abort, false)) break;
                 tc_fence_after();
-                const uint32_t pb = base + L::kPOff + (2 * q + sp) * 16384;
+                const uint64_t dp = dp0 + (uint64_t)(sp * (16384 >> 4));
+                const uint64_t dv = dv0 + (uint64_t)(stp * (16384 >> 4));
+                // K step kk: keys 16kk.. = P column group kk, V rows 16kk..
 #pragma unroll
-                for (int kk = 0; kk < L::kBN / 16; ++kk) {
-                    const uint64_t ad = sw128_desc(pb + kk * 32, 16, 1024);
-                    const uint64_t bd = sw128_desc(vb + kk * 2048, 8192, 1024);
-                    umma_ss(tmem + q * 256 + 128, ad, bd, id_o, (jj > 0 || kk > 0) ? 1u : 0u);
-                }
+                for (int kk = 0; kk < L::kBN / 16; ++kk)
+                    umma_ss(to, dp + (uint64_t)((kk * 32) >> 4), dv + (uint64_t)((kk * 2048) >> 4),
+                            id_o, (jj > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(bar(L::BPVD + 2 * q + sp));
             }
-            if (!ok) break;
             umma_commit(bar(L::BKVE + stp));
         }
     }
-    umma_commit(bar(L::BOF));
-    umma_commit(bar(L::BDRAIN));
-    mbar_drain(bar(L::BDRAIN), 0);
+    umma_commit(bar(L::BOF + q));
+    umma_commit(bar(L::BDRAIN + q));
+    mbar_drain(bar(L::BDRAIN + q), 0);
 }
 
 // One 64-key tile of one row: raw logits r[] (TMEM), keep columns first..lim

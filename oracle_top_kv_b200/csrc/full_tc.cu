@@ -20,9 +20,11 @@
 // share every K/V tile; their softmax warpgroups alternate on the tensor core.
 // Warp roles:
 //   warp 0       TMA producer (both Q tiles once; K and V tiles, 3-stage ring)
-//   warp 1       TMEM owner and MMA issuer: per Q tile S = Q K^T into one of
-//                two TMEM buffers, then O += P V (P from shared memory, V
-//                MN-major)
+//   warp 1       TMEM owner and MMA issuer of Q tile 0; warp 10 issues for
+//                Q tile 1: S = Q K^T into one of two TMEM buffers, then
+//                O += P V (P from shared memory, V MN-major).  One issuing
+//                thread per tile: a single thread cannot issue the MMAs of
+//                both tiles as fast as the tensor core runs them.
 //   warps 2..9   two softmax warpgroups, one thread per row (TMEM lane):
 //                online softmax with lazy rescaling of O (only when the max
 //                grows by > 2^8), P to shared memory, block-score capture,
@@ -125,8 +127,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0)
             fl::producer<L>(base, &tmap_q, &tmap_k, &tmap_v, row0, P, u * g, b, bu, nt,
                             [](int j) { return j * kBN; }, abort_flag);
-    } else if (warp == 1) {
-        if (lane == 0) fl::mma_issuer<L>(base, tmem, nt, ntq, abort_flag);
+    } else if (warp == 1 || warp == L::kIssuer1Warp) {
+        if (lane == 0) {
+            const int qi = warp == 1 ? 0 : 1;
+            fl::mma_issuer<L>(base, tmem, qi, nt, qi == 0 ? ntq[0] : ntq[1], abort_flag);
+        }
     } else {
         // ------------------------------------------------------ softmax
         const int q = (warp - 2) >> 2;   // warpgroup = Q tile
@@ -174,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(L::BPF + 2 * q + s));
         }
-        if (ok && nt_me > 0) ok = fl::warp_wait(bar(L::BOF), 0, abort_flag);
+        if (ok && nt_me > 0) ok = fl::warp_wait(bar(L::BOF + q), 0, abort_flag);
         const bool row_ok = nt_me > 0 && qrow0 + pr < p.t_q;
         const int h = u * g + hh;
         const size_t orow = ((size_t)b * p.hq + h) * p.t_q + qrow0 + pr;

@@ -16,7 +16,8 @@
 // instead of once per row, and both contractions run on the tensor cores.
 //
 // Warp roles as in full_tc.cu: warp 0 TMA producer (Q once, union blocks
-// through a 2-stage K/V ring), warp 1 TMEM owner and MMA issuer, warps 2..9
+// through a 2-stage K/V ring), warp 1 TMEM owner and MMA issuer of Q tile 0,
+// warp 10 MMA issuer of Q tile 1, warps 2..9
 // two softmax warpgroups (one thread per row).  Supported: bf16, d = 128,
 // block mode with B = 64 (= the key tile), 128 % g == 0, and a union of at
 // most kMaxUnion blocks (2 * (128/g) positions x k/B ids).  The window branch
@@ -99,7 +100,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int x = threadIdx.x; x < words; x += blockDim.x) bitmap[x] = 0u;
 
     // This thread's row (softmax warps): its position's selected block ids.
-    const bool is_row = warp >= 2;
+    const bool is_row = warp >= 2 && warp < L::kIssuer1Warp;
     const int q = is_row ? (warp - 2) >> 2 : 0;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
@@ -165,8 +166,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0)
             fl::producer<L>(base, &tmap_q, &tmap_k, &tmap_v, row0, P, u * g, b, bu, nt,
                             [&](int j) { return (kWin ? win_b0 + j : ulist[j]) * kBN; }, abort_flag);
-    } else if (warp == 1) {
-        if (lane == 0) fl::mma_issuer<L>(base, tmem, nt, ntq, abort_flag);
+    } else if (warp == 1 || warp == L::kIssuer1Warp) {
+        if (lane == 0) {
+            const int qi = warp == 1 ? 0 : 1;
+            fl::mma_issuer<L>(base, tmem, qi, nt, qi == 0 ? ntq[0] : ntq[1], abort_flag);
+        }
     } else {
         // ------------------------------------------------------ softmax
         const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16) + q * 256;
@@ -214,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(L::BPF + 2 * q + s));
         }
-        if (ok && nt_me > 0) ok = fl::warp_wait(bar(L::BOF), 0, abort_flag);
+        if (ok && nt_me > 0) ok = fl::warp_wait(bar(L::BOF + q), 0, abort_flag);
         const size_t orow = ((size_t)b * p.hq + u * g + hh) * p.t_q + qrow0 + pr;
         if (ok) {  // warp-uniform; the TMEM loads run on every lane of the warp
             if (nt_me > 0) tc_fence_after();

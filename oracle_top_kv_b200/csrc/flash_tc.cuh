@@ -185,6 +185,11 @@ __device__ __forceinline__ void mma_issuer(uint32_t base, uint32_t tmem, int q, 
 // more than 2^8; *corr is then the factor for l and O, and the return value
 // says whether O holds anything to rescale), p = 2^(x*scale_log2 - m_ref)
 // with packed FMA, row sum into l, and P packed to bf16 pairs.
+// kPolyEvery > 0: every kPolyEvery-th pair of exponentials runs on the FMA
+// pipe (exp2_poly2) instead of the MUFU unit, whose throughput otherwise
+// bounds the tile.  That path never returns an exact 0 (2^-125 for masked
+// keys), so only callers whose rows always keep some key may use it.
+template <int kPolyEvery = 0>
 __device__ __forceinline__ bool softmax_tile(const uint32_t (&r)[64], int first, int lim, float sl2,
                                              float& m_ref, float& l, float& mt, float& corr,
                                              uint32_t (&pk)[32]) {
@@ -218,8 +223,14 @@ __device__ __forceinline__ bool softmax_tile(const uint32_t (&r)[64], int first,
 #pragma unroll
     for (int c2 = 0; c2 < 32; ++c2) {
         const float2 y = ffma2(make_float2(x[2 * c2], x[2 * c2 + 1]), s2, n2);
-        e[2 * c2] = ex2(y.x);
-        e[2 * c2 + 1] = ex2(y.y);
+        if (kPolyEvery > 0 && c2 % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
+            const float2 ev = exp2_poly2(y);
+            e[2 * c2] = ev.x;
+            e[2 * c2 + 1] = ev.y;
+        } else {
+            e[2 * c2] = ex2(y.x);
+            e[2 * c2 + 1] = ex2(y.y);
+        }
         const float2 ev = make_float2(e[2 * c2], e[2 * c2 + 1]);
         acc[c2 & 7] = c2 < 8 ? ev : fadd2(acc[c2 & 7], ev);
     }

@@ -161,10 +161,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(L::BSE + 2 * q + s));
 
-            // causal: keys <= pos (only the diagonal tile masks anything)
+            // causal: keys <= pos (only the diagonal tile masks anything).  Key 0
+            // is in every row's first tile, so every row keeps a key and a third
+            // of the exponentials can run on the FMA pipe.
             float mt, corr;
             uint32_t pk[32];
-            const bool resc = fl::softmax_tile(r, 0, pos - j * kBN, sl2, m_ref, l, mt, corr, pk);
+            const bool resc =
+                fl::softmax_tile<3>(r, 0, pos - j * kBN, sl2, m_ref, l, mt, corr, pk);
             if (a.capture && mt > -INFINITY) list_insert(lv, li, mt, j);
             // P buffer s of this tile is free once the PV of tile j-2 is done
             if (j >= 2 && !fl::warp_wait(bar(L::BPVD + 2 * q + s), ((j >> 1) - 1) & 1, abort_flag)) { ok = false; break; }

@@ -106,6 +106,31 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
     return d;
 }
 
+// 2^y for a pair of values on the FMA pipe, to take part of a softmax's
+// exponentials off the MUFU unit (the split FlashAttention-4 makes on
+// Blackwell).  y is clamped to >= -125, so the result is never 0: at most
+// 2^-125 where the exact value is smaller.  Steps: t = y + 1.5*2^23 rounds y to
+// the nearest integer j (held in t's low mantissa bits), f = y - j in
+// [-1/2, 1/2], 2^f from the degree-3 minimax polynomial of exp2_poly.py
+// (relative error <= 7.5e-5), then j is added to the exponent field.  Because
+// every set bit of 1.5*2^23's encoding lies at position >= 22, the float bits
+// of t shifted left by 23 are exactly j << 23 (mod 2^32).
+__device__ __forceinline__ float2 exp2_poly2(float2 y) {
+    constexpr float kShift = 12582912.f;  // 1.5 * 2^23
+    constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f,
+                    c2 = 0.2426111251115799f, c3 = 0.0551716685295105f;
+    y.x = fmaxf(y.x, -125.f);
+    y.y = fmaxf(y.y, -125.f);
+    const float2 t = fadd2(y, make_float2(kShift, kShift));
+    const float2 r = fadd2(t, make_float2(-kShift, -kShift));
+    const float2 f = ffma2(r, make_float2(-1.f, -1.f), y);  // exact: y - rint(y)
+    float2 p = ffma2(make_float2(c3, c3), f, make_float2(c2, c2));
+    p = ffma2(p, f, make_float2(c1, c1));
+    p = ffma2(p, f, make_float2(c0, c0));
+    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int c0, int c1, int c2) {

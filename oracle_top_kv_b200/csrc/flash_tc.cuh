@@ -19,24 +19,28 @@ namespace fl {
 
 using namespace tc;
 
-// Shared-memory map and mbarrier indices of a pipeline with a KV-stage ring
-// and `Extra` kernel-specific bytes after the P buffers.
-template <int KV, uint32_t Extra>
+// Shared-memory map and mbarrier indices of a pipeline with a KS-stage K ring,
+// a VS-stage V ring and `Extra` kernel-specific bytes after the P buffers.
+// K and V have rings of their own: a K stage is free as soon as the S MMAs
+// that read it are done, so K loads run ahead of V loads, which wait for PV.
+template <int KS, int VS, uint32_t Extra>
 struct Layout {
-    static constexpr int kBM = 128, kNQ = 2, kBN = 64, kD = 128, kKV = KV;
+    static constexpr int kBM = 128, kNQ = 2, kBN = 64, kD = 128, kKS = KS, kVS = VS;
     static constexpr int kIssuer1Warp = 2 + 4 * kNQ;               // issuer of Q tile 1
     static constexpr int kThreads = 64 + 128 * kNQ + 32 * (kNQ - 1);
     static constexpr uint32_t kQOff = 0;                       // kNQ x 32 KB (two d halves)
-    static constexpr uint32_t kKOff = kNQ * 32768;             // KV x 16 KB
-    static constexpr uint32_t kVOff = kKOff + KV * 16384;      // KV x 16 KB
-    static constexpr uint32_t kPOff = kVOff + KV * 16384;      // kNQ x 2 x 16 KB
+    static constexpr uint32_t kKOff = kNQ * 32768;             // KS x 16 KB
+    static constexpr uint32_t kVOff = kKOff + KS * 16384;      // VS x 16 KB
+    static constexpr uint32_t kPOff = kVOff + VS * 16384;      // kNQ x 2 x 16 KB
     static constexpr uint32_t kExtraOff = kPOff + kNQ * 2 * 16384;
     static constexpr uint32_t kBarOff = kExtraOff + Extra;
     enum {
         BQ = 0,
-        BKVF = 1,
-        BKVE = BKVF + KV,
-        BSF = BKVE + KV,  // [q][s]
+        BKF = 1,          // K stage full / empty
+        BKE = BKF + KS,
+        BVF = BKE + KS,   // V stage full / empty
+        BVE = BVF + VS,
+        BSF = BVE + VS,   // [q][s]
         BSE = BSF + 2 * kNQ,
         BPF = BSE + 2 * kNQ,
         BPVD = BPF + 2 * kNQ,
@@ -69,8 +73,9 @@ template <class L>
 __device__ __forceinline__ void init_barriers(uint32_t bar0) {
     auto bar = [&](int i) { return bar0 + 8u * i; };
     mbar_init(bar(L::BQ), 1);
-    // a K/V stage is free once both issuers' PV MMAs that read it are done
-    for (int i = 0; i < L::kKV; ++i) { mbar_init(bar(L::BKVF + i), 1); mbar_init(bar(L::BKVE + i), L::kNQ); }
+    // a K (V) stage is free once both issuers' S (PV) MMAs that read it are done
+    for (int i = 0; i < L::kKS; ++i) { mbar_init(bar(L::BKF + i), 1); mbar_init(bar(L::BKE + i), L::kNQ); }
+    for (int i = 0; i < L::kVS; ++i) { mbar_init(bar(L::BVF + i), 1); mbar_init(bar(L::BVE + i), L::kNQ); }
     for (int i = 0; i < 2 * L::kNQ; ++i) {
         mbar_init(bar(L::BSF + i), 1);
         mbar_init(bar(L::BSE + i), 4);
@@ -81,7 +86,9 @@ __device__ __forceinline__ void init_barriers(uint32_t bar0) {
 }
 
 // TMA producer (one thread): both Q tiles once (4-D boxes: 64 d x P positions
-// x g heads), then the key tiles key0_of(j), j < nt, through the ring.
+// x g heads), then K and V of the key tiles key0_of(j), j < nt, in the order
+// the MMAs need them: K(j) before V(j-1), since S of tile j is issued before
+// PV of tile j-1.
 template <class L, class KeyOf>
 __device__ __forceinline__ void producer(uint32_t base, const CUtensorMap* tq, const CUtensorMap* tk,
                                          const CUtensorMap* tv, int row0, int P, int head0, int b,
@@ -96,33 +103,45 @@ __device__ __forceinline__ void producer(uint32_t base, const CUtensorMap* tq, c
         tma_load_4d(base + L::kQOff + q * 32768, tq, bar(L::BQ), 0, row0 + q * P, head0, b);
         tma_load_4d(base + L::kQOff + q * 32768 + 16384, tq, bar(L::BQ), 64, row0 + q * P, head0, b);
     }
-    int issued = 0;
-    for (int j = 0; j < nt; ++j) {
-        const int st = j % L::kKV;
-        if (j >= L::kKV && !mbar_wait(bar(L::BKVE + st), ((j / L::kKV) - 1) & 1, abort, false))
-            break;
-        const uint32_t f = bar(L::BKVF + st);
-        mbar_arrive_expect_tx(f, 4 * 8192);
-        const uint32_t kd = base + L::kKOff + st * 16384, vd = base + L::kVOff + st * 16384;
-        const int key0 = key0_of(j);
-        tma_load_3d(kd, tk, f, 0, key0, bu);
-        tma_load_3d(kd + 8192, tk, f, 64, key0, bu);
-        tma_load_3d(vd, tv, f, 0, key0, bu);
-        tma_load_3d(vd + 8192, tv, f, 64, key0, bu);
-        issued = j + 1;
+    int k_issued = 0, v_issued = 0, key_next = nt > 0 ? key0_of(0) : 0, key_prev = 0;
+    for (int j = 0; j <= nt; ++j) {
+        if (j < nt) {
+            const int st = j % L::kKS;
+            if (j >= L::kKS && !mbar_wait(bar(L::BKE + st), ((j / L::kKS) - 1) & 1, abort, false))
+                break;
+            const uint32_t f = bar(L::BKF + st), kd = base + L::kKOff + st * 16384;
+            mbar_arrive_expect_tx(f, 16384);
+            tma_load_3d(kd, tk, f, 0, key_next, bu);
+            tma_load_3d(kd + 8192, tk, f, 64, key_next, bu);
+            k_issued = j + 1;
+        }
+        if (j >= 1) {
+            const int jj = j - 1, st = jj % L::kVS;
+            if (jj >= L::kVS && !mbar_wait(bar(L::BVE + st), ((jj / L::kVS) - 1) & 1, abort, false))
+                break;
+            const uint32_t f = bar(L::BVF + st), vd = base + L::kVOff + st * 16384;
+            mbar_arrive_expect_tx(f, 16384);
+            tma_load_3d(vd, tv, f, 0, key_prev, bu);
+            tma_load_3d(vd + 8192, tv, f, 64, key_prev, bu);
+            v_issued = j;
+        }
+        key_prev = key_next;
+        if (j + 1 < nt) key_next = key0_of(j + 1);
     }
     // every issued load must have landed before the CTA may exit
     mbar_drain(bar(L::BQ), 0);
-    for (int j = max(0, issued - L::kKV); j < issued; ++j)
-        mbar_drain(bar(L::BKVF + j % L::kKV), (j / L::kKV) & 1);
+    for (int j = max(0, k_issued - L::kKS); j < k_issued; ++j)
+        mbar_drain(bar(L::BKF + j % L::kKS), (j / L::kKS) & 1);
+    for (int j = max(0, v_issued - L::kVS); j < v_issued; ++j)
+        mbar_drain(bar(L::BVF + j % L::kVS), (j / L::kVS) & 1);
 }
 
 // MMA issuer of Q tile q (one thread): iteration j issues S = Q K^T of tile j
-// (after its S buffer is free), then O += P V of tile j-1 (after its P is
-// ready), and releases tile j-1's K/V stage.  The Q tile uses ntq of the CTA's
-// nt tiles; for the rest it still waits for each stage to fill before
-// releasing it, so its release of a stage can never count towards a later
-// use of that stage than the other issuer's.
+// (after its S buffer is free) and releases tile j's K stage, then issues
+// O += P V of tile j-1 (after its P is ready) and releases tile j-1's V stage.
+// The Q tile uses ntq of the CTA's nt tiles; for the rest it still waits for
+// each stage to fill before releasing it, so its release of a stage can never
+// count towards a later use of that stage than the other issuer's.
 // One thread's instruction stream bounds the MMA rate, hence one issuer per Q
 // tile and shared-memory descriptors built once: a descriptor holds its start
 // address as addr >> 4 in its low 14 bits, and every operand of the CTA lies
@@ -142,8 +161,8 @@ __device__ __forceinline__ void mma_issuer(uint32_t base, uint32_t tmem, int q, 
     tc_fence_after();
     for (int j = 0; ok && j <= nt; ++j) {
         if (j < nt) {
-            const int st = j % L::kKV, s = j & 1;
-            if (!mbar_wait(bar(L::BKVF + st), (j / L::kKV) & 1, abort, false)) break;
+            const int st = j % L::kKS, s = j & 1;
+            if (!mbar_wait(bar(L::BKF + st), (j / L::kKS) & 1, abort, false)) break;
             if (j < ntq) {
                 if (j >= 2 && !mbar_wait(bar(L::BSE + 2 * q + s), ((j >> 1) - 1) & 1, abort, false)) break;
                 tc_fence_after();
@@ -156,9 +175,11 @@ __device__ __forceinline__ void mma_issuer(uint32_t base, uint32_t tmem, int q, 
                             kk > 0 ? 1u : 0u);
                 umma_commit(bar(L::BSF + 2 * q + s));
             }
+            umma_commit(bar(L::BKE + st));
         }
         if (j >= 1) {
-            const int jj = j - 1, sp = jj & 1, stp = jj % L::kKV;
+            const int jj = j - 1, sp = jj & 1, stp = jj % L::kVS;
+            if (!mbar_wait(bar(L::BVF + stp), (jj / L::kVS) & 1, abort, false)) break;
             if (jj < ntq) {
                 if (!mbar_wait(bar(L::BPF + 2 * q + sp), (jj >> 1) & 1, abort, false)) break;
                 tc_fence_after();
@@ -171,7 +192,7 @@ __device__ __forceinline__ void mma_issuer(uint32_t base, uint32_t tmem, int q, 
                             id_o, (jj > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(bar(L::BPVD + 2 * q + sp));
             }
-            umma_commit(bar(L::BKVE + stp));
+            umma_commit(bar(L::BVE + stp));
         }
     }
     umma_commit(bar(L::BOF + q));

@@ -38,7 +38,7 @@
 namespace hs {
 namespace tc {
 
-using L = fl::Layout<3, 0>;   // 3-stage K/V ring, nothing beyond the P buffers
+using L = fl::Layout<3, 3, 0>;  // 3-stage K and V rings, nothing beyond the P buffers
 constexpr int kBM = L::kBM, kNQ = L::kNQ, kBN = L::kBN, kD = L::kD;
 constexpr int kList = 16;     // per-row candidate list (>= k/B)
 constexpr int kThreads = L::kThreads;

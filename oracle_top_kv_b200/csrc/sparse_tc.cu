@@ -36,7 +36,7 @@ using namespace tc;
 
 constexpr int kMaxSel = 16;    // selected blocks per row held in registers
 constexpr int kMaxUnion = 1024;
-using L = fl::Layout<2, kMaxUnion * 4>;  // 2-stage K/V ring; the union block list after P
+using L = fl::Layout<3, 2, kMaxUnion * 4>;  // 3 K and 2 V stages; the union block list after P
 constexpr int kBM = L::kBM, kNQ = L::kNQ, kBN = L::kBN, kD = L::kD;
 constexpr int kThreads = L::kThreads;
 constexpr uint32_t kUOff = L::kExtraOff;                  // union block ids, kMaxUnion ints

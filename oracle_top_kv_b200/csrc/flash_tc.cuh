@@ -208,9 +208,10 @@ __device__ __forceinline__ void mma_issuer(uint32_t base, uint32_t tmem, int q, 
 // with packed FMA, row sum into l, and P packed to bf16 pairs.
 // kPolyEvery > 0: every kPolyEvery-th pair of exponentials runs on the FMA
 // pipe (exp2_poly2) instead of the MUFU unit, whose throughput otherwise
-// bounds the tile.  That path never returns an exact 0 (2^-125 for masked
-// keys), so only callers whose rows always keep some key may use it.
-template <int kPolyEvery = 0>
+// bounds the tile.  That path returns 2^-125 rather than 0 below 2^-125, e.g.
+// for masked keys; kZero selects an exact 0 there, for callers whose rows may
+// keep no key at all (whose l must then stay exactly 0).
+template <int kPolyEvery = 0, bool kZero = false>
 __device__ __forceinline__ bool softmax_tile(const uint32_t (&r)[64], int first, int lim, float sl2,
                                              float& m_ref, float& l, float& mt, float& corr,
                                              uint32_t (&pk)[32]) {
@@ -246,8 +247,8 @@ __device__ __forceinline__ bool softmax_tile(const uint32_t (&r)[64], int first,
         const float2 y = ffma2(make_float2(x[2 * c2], x[2 * c2 + 1]), s2, n2);
         if (kPolyEvery > 0 && c2 % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
             const float2 ev = exp2_poly2(y);
-            e[2 * c2] = ev.x;
-            e[2 * c2 + 1] = ev.y;
+            e[2 * c2] = (!kZero || y.x >= -125.f) ? ev.x : 0.f;
+            e[2 * c2 + 1] = (!kZero || y.y >= -125.f) ? ev.y : 0.f;
         } else {
             e[2 * c2] = ex2(y.x);
             e[2 * c2 + 1] = ex2(y.y);

@@ -201,10 +201,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const int lim = (sel && row_valid) ? pos - key0 : -1;  // last kept column
             const int first = kWin ? pos - p.window + 1 - key0 : 0;  // first kept column
-            // a row may see no kept key for a while (m_ref = -inf)
+            // a row may see no kept key for a while (m_ref = -inf), or none at
+            // all: masked keys must give exact zeros
             float mt, corr;
             uint32_t pk[32];
-            const bool resc = fl::softmax_tile(r, first, lim, sl2, m_ref, l, mt, corr, pk);
+            const bool resc =
+                fl::softmax_tile<4, true>(r, first, lim, sl2, m_ref, l, mt, corr, pk);
             // P buffer s is free once the PV of tile j-2 is done
             if (j >= 2 && !fl::warp_wait(bar(L::BPVD + 2 * q + s), ((j >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
             fl::store_p(gbase + L::kPOff + (2 * q + s) * 16384, row, pk);

@@ -230,6 +230,21 @@ def work(w, blk):
     return flops, None, sbytes
 
 
+def sparse_useful_flops(w, blk):
+    """Useful FLOPs of one sparse layer: 4*d per (query head, kept key) -- the
+    selected keys clipped to the row's position plus the window branch's keys."""
+    rows = A.sparse_rows_from_index(blk.idx, blk.cnt, w.mode, w.block_size, w.q_offset)
+    local = A.window_rows(w.batch, w.hkv, w.tq, w.window, w.q_offset) if w.swa_branch else 0
+    return (rows + local) * (w.hq // w.hkv) * 4 * w.head_dim
+
+
+def sparse_on_tensor_cores(w):
+    """Block mode with 64-key blocks at d = 128 in bf16 runs the row-grouped
+    tcgen05 kernel (a CTA streams the union of its rows' selected blocks)."""
+    return (w.mode == "block" and w.dtype == "bf16" and w.head_dim == 128 and
+            w.block_size == 64 and w.ksel <= 16 and 128 % (w.hq // w.hkv) == 0)
+
+
 def traffic_for(kernel, workload):
     """Per-launch DRAM bytes from the committed ncu summary, if the kernel's
     source is unchanged since the capture; else None."""
@@ -350,6 +365,19 @@ def run_ours(args, rank, world, device):
                 "peak_source": full_peak_src,
                 "work_per_launch": flops if flops is not None else full_bytes,
                 "avg_launch_ms": full_s * 1e3}
+    elif not w.decode and sparse_on_tensor_cores(w):
+        uf = sparse_useful_flops(w, blk)
+        rate = uf / sparse_s / 1e12
+        roof = {"kernel": "sparse_attn_reuse", "bound": "tensor", "achieved": rate,
+                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": rate / peaks["bf16_tflops_sustained"],
+                "traffic": traffic_for("sparse_attn_reuse", w.name),
+                "peak_source": f"{peak_kind} bf16_tflops_sustained",
+                "work_per_launch": uf, "avg_launch_ms": sparse_s * 1e3,
+                "note": "block mode runs on the tensor cores over each CTA's union of its rows' "
+                        "selected blocks; work = the useful FLOPs, 4*d per (query head, kept "
+                        "key), while the MMAs issued cover every union block for every row "
+                        "(about 4x); the pages' logical-bytes rate is sparse_kv_gbs"}
     else:
         roof = {"kernel": "decode_sparse" if w.decode else "sparse_attn_reuse", "bound": "hbm",
                 "achieved": sparse_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",

@@ -132,10 +132,16 @@ __device__ __forceinline__ uint64_t warp_kth_largest(const uint64_t* buf, int n,
                                                      uint32_t* hist) {
     const int lane = threadIdx.x & 31;
     uint64_t lo = ~0ull, hi = 0ull;
-    for (int i = lane; i < n; i += 32) {
-        const uint64_t key = buf[i];
-        lo = key < lo ? key : lo;
-        hi = key > hi ? key : hi;
+    for (int base = 0; base < n; base += 8 * 32) {  // 8 loads in flight per lane
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = base + u * 32 + lane;
+            if (i < n) {
+                const uint64_t key = buf[i];
+                lo = key < lo ? key : lo;
+                hi = key > hi ? key : hi;
+            }
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -152,9 +158,17 @@ __device__ __forceinline__ uint64_t warp_kth_largest(const uint64_t* buf, int n,
 #pragma unroll
         for (int x = 0; x < 8; ++x) hist[lane * 8 + x] = 0;
         __syncwarp();
-        for (int i = lane; i < n; i += 32) {
-            const uint64_t key = buf[i];
-            if (key >= lo && key <= hi) atomicAdd(&hist[(uint32_t)((key - lo) >> shift)], 1u);
+        for (int base = 0; base < n; base += 8 * 32) {
+            uint64_t key[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {  // all loads first, then the atomics
+                const int i = base + u * 32 + lane;
+                key[u] = i < n ? buf[i] : 0ull;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (base + u * 32 + lane < n && key[u] >= lo && key[u] <= hi)
+                    atomicAdd(&hist[(uint32_t)((key[u] - lo) >> shift)], 1u);
         }
         __syncwarp();
         // lane L owns buckets 255-8L .. 248-8L (descending).  Count above each.
@@ -194,9 +208,15 @@ __device__ __forceinline__ uint64_t warp_kth_largest(const uint64_t* buf, int n,
         if (in_b == 1) {
             // the K-th key is the only one left in [lo, hi]: fetch it
             uint64_t hit = 0;
-            for (int i = lane; i < n; i += 32) {
-                const uint64_t key = buf[i];
-                if (key >= lo && key <= hi) hit = key;
+            for (int base = 0; base < n; base += 8 * 32) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int i = base + u * 32 + lane;
+                    if (i < n) {
+                        const uint64_t key = buf[i];
+                        if (key >= lo && key <= hi) hit = key;
+                    }
+                }
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
@@ -209,22 +229,47 @@ __device__ __forceinline__ uint64_t warp_kth_largest(const uint64_t* buf, int n,
     return lo;  // not reached for unique keys: each pass shrinks the range 256-fold
 }
 
-// Keep only keys >= kth (in place, order not preserved); returns the new count.
+// Keep only keys >= kth, compacted in place in their original order; returns
+// the new count.  Chunks of 8 x 32 keys: the whole chunk is read into
+// registers before any of it is written back (so the loads overlap instead of
+// each waiting for the previous store), which is safe in place because a kept
+// key's new position is never past its old one.
 __device__ __forceinline__ int warp_keep_at_least(uint64_t* buf, int n, uint64_t kth) {
     const int lane = threadIdx.x & 31;
     int out = 0;
-    for (int base = 0; base < n; base += 32) {
-        const int i = base + lane;
-        uint64_t key = 0;
-        bool keep = false;
-        if (i < n) { key = buf[i]; keep = key >= kth; }
-        const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+    for (int base = 0; base < n; base += 8 * 32) {
+        uint64_t key[8];
+        bool keep[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = base + u * 32 + lane;
+            key[u] = i < n ? buf[i] : 0ull;
+            keep[u] = i < n && key[u] >= kth;
+        }
         __syncwarp();
-        if (keep) buf[out + __popc(bal & ((1u << lane) - 1))] = key;
-        out += __popc(bal);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const uint32_t bal = __ballot_sync(0xffffffffu, keep[u]);
+            if (keep[u]) buf[out + __popc(bal & ((1u << lane) - 1))] = key[u];
+            out += __popc(bal);
+        }
         __syncwarp();
     }
     return out;
+}
+
+// Number of keys >= thr among buf[0 .. n) (warp-wide; 8 loads in flight per lane).
+__device__ __forceinline__ int warp_count_at_least(const uint64_t* buf, int n, uint64_t thr) {
+    const int lane = threadIdx.x & 31;
+    int c = 0;
+    for (int base = 0; base < n; base += 8 * 32) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = base + u * 32 + lane;
+            c += (i < n && buf[i] >= thr) ? 1 : 0;
+        }
+    }
+    return __reduce_add_sync(0xffffffffu, c);
 }
 
 // Cut the buffer to its K best keys; returns the K-th best key (the new
@@ -279,9 +324,7 @@ __device__ __forceinline__ int warp_cut_sampled(uint64_t* buf, int n, int K, int
         const uint64_t thr = __shfl_sync(0xffffffffu, (uint32_t)(e < 32 ? a : b), e & 31) |
                              ((uint64_t)__shfl_sync(0xffffffffu, (uint32_t)((e < 32 ? a : b) >> 32),
                                                     e & 31) << 32);
-        int c = 0;
-        for (int i = lane; i < n; i += 32) c += buf[i] >= thr;
-        c = __reduce_add_sync(0xffffffffu, c);
+        const int c = warp_count_at_least(buf, n, thr);
         if (c < K) continue;            // too high: a top-K key would go
         if (n - c < min_free) break;    // keeps too much: exact cut instead
         const int m = warp_keep_at_least(buf, n, thr);

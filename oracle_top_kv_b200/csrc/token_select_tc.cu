@@ -187,6 +187,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint64_t* bufs = reinterpret_cast<uint64_t*>(gb + kBufOff);
         uint32_t* hist = reinterpret_cast<uint32_t*>(gb + kHistOff + wid * 1024);
         const int bar_id = 1 + set;
+        // Admission compares a key's float score with the float score of the
+        // position's threshold key (thf, in registers): score >= thf admits
+        // every key that beats the 64-bit threshold (and at most the few that
+        // tie its score), and admitting more than necessary is always safe --
+        // the cuts and the finalize select exactly.  Bulk tiles (all four
+        // positions live, none selecting everything, no scores to write, the
+        // tile entirely below the first position's window, hence below every
+        // window of the four and visible to all) need nothing else.
+        bool bulk_ok = Kc > 0 && a.sel == nullptr;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) bulk_ok = bulk_ok && live[i] && !all_sel[i];
+        const int lo_first = tpos[0] - p.window + 1;
+        float thf[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         bool ok = true;
         // Every warp runs every iteration (the set meets at named barriers);
         // after an abort the waits fail at once and the work is skipped.
@@ -205,7 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(BSE + s));
             const int key = j * kKeys + quad * 32 + lane;
-            uint64_t k64[4];
+            const bool bulk = bulk_ok && (j + 1) * kKeys <= lo_first;  // warp-uniform
+            float sc[4];
             uint32_t bal[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -222,10 +236,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     v[hh] = r2.x;
                     v[hh + 1] = r2.y;
                 }
-                const float sc = fmaxf(max3f(max3f(v[0], v[1], v[2]), max3f(v[3], v[4], v[5]),
-                                             max3f(v[6], v[7], v[8])),
-                                       max3f(max3f(v[9], v[10], v[11]),
-                                             max3f(v[12], v[13], v[14]), v[15]));
+                sc[i] = fmaxf(max3f(max3f(v[0], v[1], v[2]), max3f(v[3], v[4], v[5]),
+                                    max3f(v[6], v[7], v[8])),
+                              max3f(max3f(v[9], v[10], v[11]), max3f(v[12], v[13], v[14]), v[15]));
+                if (bulk) {
+                    bal[i] = __ballot_sync(0xffffffffu, sc[i] >= thf[i]);
+                    continue;
+                }
                 const int t = tpos[i];
                 const bool visible = live[i] && key <= t;
                 const int pos = set * 4 + i;
@@ -233,31 +250,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float* srow = a.sel ? a.sel + orow * p.ksel : nullptr;
                 // Every lane reaches the ballot below: no per-lane early exit.
                 const int lo = t - p.window + 1;
-                k64[i] = sel_key(sc, (uint32_t)key);
                 bool cand = false;
                 if (all_sel[i]) {
-                    if (visible && srow) srow[key] = exp2f(sc);
+                    if (visible && srow) srow[key] = exp2f(sc[i]);
                 } else if (visible && key >= lo) {
-                    if (srow) srow[Kc + (key - lo)] = exp2f(sc);
+                    if (srow) srow[Kc + (key - lo)] = exp2f(sc[i]);
                 } else {
-                    cand = visible && Kc > 0 && key < lo && k64[i] > s_th[pos];
+                    cand = visible && Kc > 0 && key < lo && sc[i] >= thf[i];
                 }
                 bal[i] = __ballot_sync(0xffffffffu, cand);
             }
-            // one lane reserves the slots of all four positions (independent atomics)
-            int basei[4] = {0, 0, 0, 0};
-            if (lane == 0) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    if (bal[i]) basei[i] = atomicAdd(&s_cnt[set * 4 + i], __popc(bal[i]));
-            }
+            // lanes 0..3 reserve the slots of the four positions at once
+            const uint32_t my_bal = lane == 0 ? bal[0] : lane == 1 ? bal[1] : lane == 2 ? bal[2] : bal[3];
+            int my_base = 0;
+            if (lane < 4 && my_bal != 0u) my_base = atomicAdd(&s_cnt[set * 4 + lane], __popc(my_bal));
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 if (!bal[i]) continue;  // warp-uniform
-                const int bi = __shfl_sync(0xffffffffu, basei[i], 0);
+                const int bi = __shfl_sync(0xffffffffu, my_base, i);
                 if ((bal[i] >> lane) & 1u)
                     bufs[(size_t)(set * 4 + i) * kCap + bi + __popc(bal[i] & ((1u << lane) - 1))] =
-                        k64[i];
+                        sel_key(sc[i], (uint32_t)key);
             }
             }  // got
             // cut a buffer that could overflow on the next tile
@@ -276,6 +289,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
+            // a cut may have raised the thresholds: refresh their float scores
+            // (-inf while nothing was cut, and never NaN)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint64_t th = s_th[set * 4 + i];
+                const float x = order_float((uint32_t)(th >> 32));
+                thf[i] = (th == 0ull || x != x) ? -INFINITY : x;
+            }
         }
         // ---- finalize: one warp per position (K stages are free: all MMAs done)
         asm volatile("bar.sync 3, 256;" ::: "memory");

@@ -16,10 +16,12 @@
 // shared memory (admission threshold = the k-w-th best key after each cut).
 //
 // Warps: 0 TMA (Q once, K tiles of 128 keys through a 2-stage ring), 1 TMEM +
-// MMA issuer (S^T in 4 TMEM buffers), 2..9 scorers in two sets of four (each
-// set covers the 128 TMEM lanes = keys, and 4 of the 8 positions).  The sets
+// MMA issuer (S^T in 4 TMEM buffers), 2..17 scorers in four sets of four (each
+// set covers the 128 TMEM lanes = keys, and 2 of the 8 positions).  The sets
 // only meet at the TMEM buffers, so one set's buffer cut does not stall the
-// other for up to 3 tiles.
+// others for up to 3 tiles.  The scorers' dependent chains (TMEM load, FMA,
+// max, ballot, shared atomics) are latency-bound, so the work is spread over
+// 16 warps with 2 positions per thread rather than 8 warps with 4.
 #include "hs_common.cuh"
 #include "hs_kernels.cuh"
 #include "tc_ptx.cuh"
@@ -32,10 +34,13 @@ using namespace tc;
 constexpr int kG = 16;          // heads per group handled here
 constexpr int kPos = 8;         // positions per CTA
 constexpr int kKeys = 128;      // keys per K tile (= MMA M)
+constexpr int kPP = 2;          // positions per scorer thread
+constexpr int kSets = kPos / kPP;          // scorer sets of four warps
+constexpr int kScorers = 4 * kSets;        // scorer warps
 constexpr int kHd = 128;
 constexpr int kStages = 2;       // K ring (the MMA is far ahead of the scorers)
 constexpr int kSBufs = 4;        // S^T buffers in TMEM: the two scorer sets may drift 3 tiles
-constexpr int kThreads = 64 + 256;
+constexpr int kThreads = 64 + 32 * kScorers;
 constexpr int kMaxRanked = 1024;            // k - w handled here
 // Per-position buffer entries: the k - w kept, one tile of admissions, and
 // 6 tiles' worth of headroom between cuts (what shared memory holds).
@@ -45,7 +50,7 @@ constexpr int kBitmapKeys = 65536;  // finalize by id bitmap (8 KB per position)
 constexpr uint32_t kQOff = 0;                         // 2 x 16 KB
 constexpr uint32_t kKOff = 32768;                     // kStages x 32 KB (sort scratch later)
 constexpr uint32_t kBufOff = kKOff + kStages * 32768; // kPos x kCap x 8
-constexpr uint32_t kHistOff = kBufOff + kPos * kCap * 8;   // 8 warps x 1 KB
+constexpr uint32_t kHistOff = kBufOff + kPos * kCap * 8;   // kPos positions x 1 KB
 constexpr uint32_t kBarOff = kHistOff + 8 * 1024;
 enum { BQ = 0, BKF = 1, BKE = BKF + kStages, BSF = BKE + kStages, BSE = BSF + kSBufs,
        BDRAIN = BSE + kSBufs, BCOUNT = BDRAIN + 1 };
@@ -101,7 +106,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         mbar_init(bar(BQ), 1);
         for (int i = 0; i < kStages; ++i) { mbar_init(bar(BKF + i), 1); mbar_init(bar(BKE + i), 1); }
-        for (int i = 0; i < kSBufs; ++i) { mbar_init(bar(BSF + i), 1); mbar_init(bar(BSE + i), 8); }
+        for (int i = 0; i < kSBufs; ++i) { mbar_init(bar(BSF + i), 1); mbar_init(bar(BSE + i), kScorers); }
         mbar_init(bar(BDRAIN), 1);
         *abort_flag = 0;
         for (int i = 0; i < kPos; ++i) { s_cnt[i] = 0; s_th[i] = 0ull; }
@@ -164,18 +169,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ scorers
-        const int set = (warp - 2) >> 2;  // positions 4*set .. 4*set+3
+        const int set = (warp - 2) >> 2;  // positions kPP*set ..
         const int quad = warp & 3;        // TMEM lane quadrant = keys 32*quad ..
-        const int wid = warp - 2;         // 0..7
-        const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16) + set * 64;
+        const int wid = warp - 2;         // 0 .. kScorers-1
+        const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16) + set * (kPP * kG);
         const float sl2 = p.scale_log2;
-        // this thread's 4 positions: lse (log2 domain) of their 16 heads
-        float nlse2[4][kG];  // -lse2
-        int tpos[4];
-        bool live[4], all_sel[4];
+        // this thread's kPP positions: lse (log2 domain) of their 16 heads
+        float nlse2[kPP][kG];  // -lse2
+        int tpos[kPP];
+        bool live[kPP], all_sel[kPP];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int r = row0 + set * 4 + i;
+        for (int i = 0; i < kPP; ++i) {
+            const int r = row0 + set * kPP + i;
             live[i] = r < p.t_q;
             tpos[i] = p.q_offset + r;
             all_sel[i] = tpos[i] + 1 <= p.k;
@@ -185,21 +190,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                                        : 0.f;
         }
         uint64_t* bufs = reinterpret_cast<uint64_t*>(gb + kBufOff);
-        uint32_t* hist = reinterpret_cast<uint32_t*>(gb + kHistOff + wid * 1024);
+        // scratch of the position this warp cuts (quads 0..kPP-1 of a set cut)
+        uint32_t* hist = reinterpret_cast<uint32_t*>(
+            gb + kHistOff + (set * kPP + (quad < kPP ? quad : 0)) * 1024);
         const int bar_id = 1 + set;
         // Admission compares a key's float score with the float score of the
         // position's threshold key (thf, in registers): score >= thf admits
         // every key that beats the 64-bit threshold (and at most the few that
         // tie its score), and admitting more than necessary is always safe --
-        // the cuts and the finalize select exactly.  Bulk tiles (all four
+        // the cuts and the finalize select exactly.  Bulk tiles (the thread's
         // positions live, none selecting everything, no scores to write, the
         // tile entirely below the first position's window, hence below every
-        // window of the four and visible to all) need nothing else.
+        // window of the set and visible to all) need nothing else.
         bool bulk_ok = Kc > 0 && a.sel == nullptr;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) bulk_ok = bulk_ok && live[i] && !all_sel[i];
+        for (int i = 0; i < kPP; ++i) bulk_ok = bulk_ok && live[i] && !all_sel[i];
         const int lo_first = tpos[0] - p.window + 1;
-        float thf[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float thf[kPP];
+#pragma unroll
+        for (int i = 0; i < kPP; ++i) thf[i] = -INFINITY;
         bool ok = true;
         // Every warp runs every iteration (the set meets at named barriers);
         // after an abort the waits fail at once and the work is skipped.
@@ -210,21 +219,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!got) ok = false;
             if (got) {
             tc_fence_after();
-            uint32_t r0[32], r1[32];
+            uint32_t r0[32];
             tmem_ld32(tq + 128 * s, r0);
-            tmem_ld32(tq + 128 * s + 32, r1);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(BSE + s));
             const int key = j * kKeys + quad * 32 + lane;
             const bool bulk = bulk_ok && (j + 1) * kKeys <= lo_first;  // warp-uniform
-            float sc[4];
-            uint32_t bal[4];
+            float sc[kPP];
+            uint32_t bal[kPP];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint32_t* rr = i < 2 ? r0 : r1;
-                const int c0 = (i & 1) * 16;
+            for (int i = 0; i < kPP; ++i) {
+                const uint32_t* rr = r0;
+                const int c0 = i * kG;
                 // a2 - lse2 of the 16 heads (packed FMA), then their max (3-input max)
                 float v[kG];
 #pragma unroll
@@ -245,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const int t = tpos[i];
                 const bool visible = live[i] && key <= t;
-                const int pos = set * 4 + i;
+                const int pos = set * kPP + i;
                 const size_t orow = ((size_t)b * p.hkv + u) * p.t_q + row0 + pos;
                 float* srow = a.sel ? a.sel + orow * p.ksel : nullptr;
                 // Every lane reaches the ballot below: no per-lane early exit.
@@ -260,23 +268,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 bal[i] = __ballot_sync(0xffffffffu, cand);
             }
-            // lanes 0..3 reserve the slots of the four positions at once
-            const uint32_t my_bal = lane == 0 ? bal[0] : lane == 1 ? bal[1] : lane == 2 ? bal[2] : bal[3];
-            int my_base = 0;
-            if (lane < 4 && my_bal != 0u) my_base = atomicAdd(&s_cnt[set * 4 + lane], __popc(my_bal));
+            // lanes 0..kPP-1 reserve the slots of the thread's positions at once
+            uint32_t my_bal = bal[0];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 1; i < kPP; ++i) my_bal = lane == i ? bal[i] : my_bal;
+            int my_base = 0;
+            if (lane < kPP && my_bal != 0u) my_base = atomicAdd(&s_cnt[set * kPP + lane], __popc(my_bal));
+#pragma unroll
+            for (int i = 0; i < kPP; ++i) {
                 if (!bal[i]) continue;  // warp-uniform
                 const int bi = __shfl_sync(0xffffffffu, my_base, i);
                 if ((bal[i] >> lane) & 1u)
-                    bufs[(size_t)(set * 4 + i) * kCap + bi + __popc(bal[i] & ((1u << lane) - 1))] =
+                    bufs[(size_t)(set * kPP + i) * kCap + bi + __popc(bal[i] & ((1u << lane) - 1))] =
                         sel_key(sc[i], (uint32_t)key);
             }
             }  // got
             // cut a buffer that could overflow on the next tile
             asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
-            if (ok) {
-                const int pos = set * 4 + quad;
+            if (ok && quad < kPP) {
+                const int pos = set * kPP + quad;
                 const int n = s_cnt[pos];
                 if (n > kCap - kKeys) {
                     uint64_t th;
@@ -292,17 +302,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             // a cut may have raised the thresholds: refresh their float scores
             // (-inf while nothing was cut, and never NaN)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint64_t th = s_th[set * 4 + i];
+            for (int i = 0; i < kPP; ++i) {
+                const uint64_t th = s_th[set * kPP + i];
                 const float x = order_float((uint32_t)(th >> 32));
                 thf[i] = (th == 0ull || x != x) ? -INFINITY : x;
             }
         }
         // ---- finalize: one warp per position (K stages are free: all MMAs done)
-        asm volatile("bar.sync 3, 256;" ::: "memory");
+        asm volatile("bar.sync %0, %1;" ::"r"(1 + kSets), "r"(32 * kScorers) : "memory");
         const int pos = wid;
         const int r = row0 + pos;
-        if (ok && r < p.t_q) {
+        if (ok && wid < kPos && r < p.t_q) {
             const int t = p.q_offset + r;
             const size_t orow = ((size_t)b * p.hkv + u) * p.t_q + r;
             int32_t* irow = a.idx + orow * p.ksel;
@@ -314,7 +324,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
                 uint64_t* buf = bufs + (size_t)pos * kCap;
                 int n = Kc > 0 ? s_cnt[pos] : 0;
-                if (n > Kc) { warp_cut_to_k(buf, n, Kc, hist); n = Kc; }
+                uint32_t* fhist = reinterpret_cast<uint32_t*>(gb + kHistOff + pos * 1024);
+                if (n > Kc) { warp_cut_to_k(buf, n, Kc, fhist); n = Kc; }
                 __syncwarp();
                 if (!srow && t < kBitmapKeys) {
                     // ascending ids without sorting: mark the winners in a bitmap

@@ -565,12 +565,17 @@ def cpu_value(w, t_step):
 
 def run_reference(args, w, world):
     inputs = oracle_inputs(w)
+    # Each oracle call converts the K/V prefix of every (batch, group) it
+    # touches to float64 once, a cost the whole step pays once per unit: the
+    # sample must hold many rows per unit for the extrapolation by row count
+    # to stay fair (decode samples whole units, whose conversion is their work).
+    budget = 12 if w.decode else 8192
     for s in range(args.warmup):
-        oracle_sample_time(w, inputs, budget_rows=12, seed=1000 + s)
+        oracle_sample_time(w, inputs, budget_rows=budget, seed=1000 + s)
     times = []
     sample = cores = None
     for s in range(max(1, args.steps)):
-        t, sample, cores = oracle_sample_time(w, inputs, budget_rows=12, seed=s)
+        t, sample, cores = oracle_sample_time(w, inputs, budget_rows=budget, seed=s)
         times.append(t)
     t_step = statistics.mean(times)
     v = cpu_value(w, t_step)

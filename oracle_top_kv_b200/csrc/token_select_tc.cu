@@ -42,10 +42,12 @@ constexpr int kStages = 2;       // K ring (the MMA is far ahead of the scorers)
 constexpr int kSBufs = 4;        // S^T buffers in TMEM: the two scorer sets may drift 3 tiles
 constexpr int kThreads = 64 + 32 * kScorers;
 constexpr int kMaxRanked = 1024;            // k - w handled here
-// Per-position buffer entries: the k - w kept, one tile of admissions, and
-// 6 tiles' worth of headroom between cuts (what shared memory holds).
+// Per-position buffer entries: the k - w kept, two tiles of admissions
+// between cut checks, and 5 tiles' worth of headroom (what shared memory holds).
 constexpr int kCap = kMaxRanked + 7 * kKeys;
 constexpr int kBitmapKeys = 65536;  // finalize by id bitmap (8 KB per position) below this
+// a cut at n > kCap - 2 kKeys must leave room for two more tiles
+static_assert((kCap - 2 * kKeys - kMaxRanked) / 2 >= 2 * kKeys, "cut headroom");
 
 constexpr uint32_t kQOff = 0;                         // 2 x 16 KB
 constexpr uint32_t kKOff = 32768;                     // kStages x 32 KB (sort scratch later)
@@ -283,29 +285,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                         sel_key(sc[i], (uint32_t)key);
             }
             }  // got
-            // cut a buffer that could overflow on the next tile
-            asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
-            if (ok && quad < kPP) {
-                const int pos = set * kPP + quad;
-                const int n = s_cnt[pos];
-                if (n > kCap - kKeys) {
-                    uint64_t th;
-                    const int m = warp_cut_sampled(bufs + (size_t)pos * kCap, n, Kc,
-                                                   (kCap - kKeys - Kc) / 2, hist, &th);
-                    if (lane == 0) {
-                        s_th[pos] = th > s_th[pos] ? th : s_th[pos];
-                        s_cnt[pos] = m;
+            // Every second tile the set meets to cut the buffers that could
+            // overflow within the next two tiles (a tile appends at most kKeys
+            // keys per position; a cut frees at least kCutFree slots or leaves
+            // Kc), then refreshes its thresholds.
+            if (j & 1) {
+                asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
+                if (ok && quad < kPP) {
+                    const int pos = set * kPP + quad;
+                    const int n = s_cnt[pos];
+                    if (n > kCap - 2 * kKeys) {
+                        uint64_t th;
+                        const int m = warp_cut_sampled(bufs + (size_t)pos * kCap, n, Kc,
+                                                       (kCap - 2 * kKeys - Kc) / 2, hist, &th);
+                        if (lane == 0) {
+                            s_th[pos] = th > s_th[pos] ? th : s_th[pos];
+                            s_cnt[pos] = m;
+                        }
                     }
                 }
-            }
-            asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
-            // a cut may have raised the thresholds: refresh their float scores
-            // (-inf while nothing was cut, and never NaN)
+                asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
+                // a cut may have raised the thresholds: refresh their float scores
+                // (-inf while nothing was cut, and never NaN)
 #pragma unroll
-            for (int i = 0; i < kPP; ++i) {
-                const uint64_t th = s_th[set * kPP + i];
-                const float x = order_float((uint32_t)(th >> 32));
-                thf[i] = (th == 0ull || x != x) ? -INFINITY : x;
+                for (int i = 0; i < kPP; ++i) {
+                    const uint64_t th = s_th[set * kPP + i];
+                    const float x = order_float((uint32_t)(th >> 32));
+                    thf[i] = (th == 0ull || x != x) ? -INFINITY : x;
+                }
             }
         }
         // ---- finalize: one warp per position (K stages are free: all MMAs done)

@@ -58,3 +58,45 @@ def test_sparse_rows_from_index_block_clipping():
     # row t=4: block0 (4 keys) + block1 keys 4..4 (1); t=5: 4 + 2; t=6: 4
     assert A.sparse_rows_from_index(idx, cnt, "block", 4, q_offset=4) == 5 + 6 + 4
     assert A.window_rows(1, 1, 3, 2, q_offset=0) == 1 + 2 + 2
+
+
+def test_sparse_useful_flops_brute_force():
+    """The block-sparse roofline's work: 4*d per (query head, kept key), where a
+    row keeps the keys <= t of its selected blocks and, with the window branch,
+    the keys t-w+1..t of its own K'/V'; counted here by enumerating pairs."""
+    torch = pytest.importorskip("torch")
+    import importlib
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    bench = importlib.import_module("bench")
+    from oracle_top_kv_b200 import workloads as wl
+    w = wl.scaled(wl.WORKLOADS["hysparse_7b_block"], name="tiny", batch=2, hq=6, hkv=2, t=40,
+                  block_size=8, k=24, window=5)
+    g = torch.Generator().manual_seed(7)
+    b, hkv, tq, ks = w.batch, w.hkv, w.tq, w.ksel
+    idx = torch.full((b, hkv, tq, ks), -1, dtype=torch.int32)
+    cnt = torch.zeros(b, hkv, tq, dtype=torch.int32)
+    for bb in range(b):
+        for u in range(hkv):
+            for t in range(tq):
+                nb = t // w.block_size + 1
+                c = int(torch.randint(0, min(ks, nb) + 1, (1,), generator=g))
+                sel = torch.randperm(nb, generator=g)[:c].sort().values
+                idx[bb, u, t, :c] = sel.to(torch.int32)
+                cnt[bb, u, t] = c
+
+    class Blk:
+        pass
+    blk = Blk()
+    blk.idx, blk.cnt = idx, cnt
+    pairs = 0
+    for bb in range(b):
+        for u in range(hkv):
+            for t in range(tq):
+                keys = set()
+                for x in range(int(cnt[bb, u, t])):
+                    r = int(idx[bb, u, t, x])
+                    keys |= {i for i in range(r * w.block_size, (r + 1) * w.block_size) if i <= t}
+                window = {i for i in range(max(0, t - w.window + 1), t + 1)} if w.swa_branch else set()
+                pairs += (len(keys) + len(window)) * (w.hq // w.hkv)
+    assert bench.sparse_useful_flops(w, blk) == pairs * 4 * w.head_dim

@@ -14,6 +14,9 @@ Function map (titles of the pages the method is described on):
                       "HySparse2 ..." 4.2 (token-level top-k, forced window).
   sparse_attn      -- "HySparse 混合稀疏注意力（一）" sections on cross-layer KV
                       reuse and the two memories of one query; "HySparse ..." 3.3.
+  gate_sink        -- "HySparse 混合稀疏注意力（一）" section on the two sigmoid
+                      gates; "HySparse ..." 3.3 (branch fusion) and its
+                      configuration note on per-head sink biases.
 """
 from __future__ import annotations
 
@@ -68,6 +71,8 @@ def _bind(lib):
                                     P, P, P, P, P, P, P, P]
     lib.orc_sparse_attn.restype = ctypes.c_int
     lib.orc_num_threads.restype = ctypes.c_int
+    lib.orc_gate_sink.argtypes = [ctypes.c_int, ctypes.c_int] + [P] * 11
+    lib.orc_gate_sink.restype = ctypes.c_int
     return lib
 
 
@@ -312,3 +317,35 @@ def sparse_attn_rows(q, kf, vf, idx_rows, cnt_rows, rows, pos, mode, block_size,
             out["o_l"][ns] = r["o_l"]
             out["lse_l"][ns] = r["lse_l"]
     return out
+
+
+def gate_sink(o_g, lse_g, o_l=None, lse_l=None, sink_g=None, sink_l=None, z_g=None, z_l=None):
+    """Sparse-layer output with per-head sinks and sigmoid gates (orc_gate_sink).
+
+    o_* [b, hq, t, d], lse_* and z_* [b, hq, t], sink_* [hq].  Returns
+    (o, lse_g', lse_l') with lse_l' None for one branch."""
+    o_g = _f64(o_g)
+    b, hq, t, d = o_g.shape
+    n = b * hq * t
+    lse_g = _f64(lse_g).reshape(n)
+
+    def per_entry(s):
+        if s is None:
+            return None
+        return _f64(np.broadcast_to(np.asarray(s, np.float64).reshape(1, hq, 1), (b, hq, t))).reshape(n)
+
+    def opt(a, shape):
+        return None if a is None else _f64(a).reshape(shape)
+
+    o_l_, lse_l_ = opt(o_l, (n, d)), opt(lse_l, n)
+    s_g_, s_l_ = per_entry(sink_g), per_entry(sink_l)
+    z_g_, z_l_ = opt(z_g, n), opt(z_l, n)
+    o = np.zeros((n, d))
+    lg = np.zeros(n)
+    ll = np.zeros(n) if o_l is not None else None
+    rc = _load().orc_gate_sink(n, d, _ptr(o_g), _ptr(lse_g), _ptr(s_g_), _ptr(z_g_), _ptr(o_l_),
+                               _ptr(lse_l_), _ptr(s_l_), _ptr(z_l_), _ptr(o), _ptr(lg), _ptr(ll))
+    if rc != 0:
+        raise ValueError(f"orc_gate_sink failed ({rc})")
+    return (o.reshape(b, hq, t, d), lg.reshape(b, hq, t),
+            None if ll is None else ll.reshape(b, hq, t))

@@ -319,6 +319,57 @@ int orc_sparse_attn(const orc_params* p, const double* q, const double* kf,
     return bad ? ORC_BAD_ARG : ORC_OK;
 }
 
+/*
+ * Output of a sparse layer: a sink per branch, then the sigmoid-gate fusion of
+ * the two branches.
+ *   [HS-1] "两个 sigmoid gate，而不是二选一": o_t = g^G (.) o^global + g^L (.) o^local,
+ *          g^G, g^L = sigma(W_g x_t), two independent sigmoids (no softmax
+ *          between the branches);
+ *   [HS-P] 3.3, branch fusion (sigmoid gates on both outputs, then the sum), and
+ *          the configuration note: sparse and SWA branches carry a learnable
+ *          per-head sink bias (the gpt-oss construction).
+ * Readings: a gate acts per head (one value per row and head); the caller
+ * supplies its pre-activation z (the projection W_g x_t belongs to the model).
+ * A sink is one more logit s_h in the branch's softmax whose value vector is
+ * zero, so the branch output and log-sum-exp become
+ *     o' = o e^lse / (e^lse + e^s),     lse' = log(e^lse + e^s).
+ * n entries (row, head) of d channels each; o_l, lse_l, s_l, z_l may be NULL
+ * (one branch); s_* NULL: no sink; z_* NULL: gate 1.  Writes o [n][d] and the
+ * branches' lse' (lse_g_out always, lse_l_out when o_l is given).
+ */
+static double log_add_exp(double a, double b) {
+    const double m = a > b ? a : b;
+    if (m == -INFINITY) return -INFINITY;
+    return m + log(exp(a - m) + exp(b - m));
+}
+
+int orc_gate_sink(int n, int d, const double* o_g, const double* lse_g, const double* s_g,
+                  const double* z_g, const double* o_l, const double* lse_l, const double* s_l,
+                  const double* z_l, double* o, double* lse_g_out, double* lse_l_out) {
+    if (n < 0 || d <= 0 || !o_g || !lse_g || !o || !lse_g_out) return ORC_BAD_ARG;
+    if (o_l && (!lse_l || !lse_l_out)) return ORC_BAD_ARG;
+    for (int e = 0; e < n; ++e) {
+        /* global branch: share of its softmax mass on real keys, and its gate */
+        const double lg = s_g ? log_add_exp(lse_g[e], s_g[e]) : lse_g[e];
+        const double fg = s_g ? exp(lse_g[e] - lg) : 1.0;
+        const double gg = z_g ? 1.0 / (1.0 + exp(-z_g[e])) : 1.0;
+        lse_g_out[e] = lg;
+        double fl = 0.0, gl = 0.0;
+        if (o_l) {
+            const double ll = s_l ? log_add_exp(lse_l[e], s_l[e]) : lse_l[e];
+            fl = s_l ? exp(lse_l[e] - ll) : 1.0;
+            gl = z_l ? 1.0 / (1.0 + exp(-z_l[e])) : 1.0;
+            lse_l_out[e] = ll;
+        }
+        for (int x = 0; x < d; ++x) {
+            double v = gg * fg * o_g[(size_t)e * d + x];
+            if (o_l) v += gl * fl * o_l[(size_t)e * d + x];
+            o[(size_t)e * d + x] = v;
+        }
+    }
+    return ORC_OK;
+}
+
 int orc_num_threads(void) {
 #ifdef _OPENMP
     extern int omp_get_max_threads(void);

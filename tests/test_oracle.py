@@ -312,3 +312,63 @@ def test_needles_are_selected_for_their_query():
                                rows=rows)
     for n, (b, u, i, h, j) in enumerate(plants):
         assert i // w.block_size in set(r["idx"][n, :r["cnt"][n]].tolist())
+
+
+# ------------------------------------------------------------- gate and sink
+def test_sink_is_an_extra_key_with_zero_value():
+    """A per-head sink bias s_h is one more logit in the softmax whose value
+    vector is zero: attention over the keys plus such a key (built so that
+    tau q_h . k_s = s_h for both heads of the group) must give gate_sink's o'
+    and lse' applied to attention over the keys alone."""
+    d, L = 8, 11
+    q = _rand((1, 2, 1, d), 31)
+    k = _rand((1, 1, L, d), 32)
+    v = _rand((1, 1, L, d), 33)
+    s = np.array([0.7, -1.3])
+    tau = 1.0 / math.sqrt(d)
+    Q = q[0, :, 0, :]                                     # [2, d]
+    k_s = Q.T @ np.linalg.solve(Q @ Q.T, s / tau)         # tau * Q k_s = s
+    np.testing.assert_allclose(tau * Q @ k_s, s, atol=1e-12)
+    k_aug = np.concatenate([k_s.reshape(1, 1, 1, d), k], axis=2)
+    v_aug = np.concatenate([np.zeros((1, 1, 1, d)), v], axis=2)
+    pa = oracle.Params(1, 2, 1, d, 1, L + 1, mode="token", block_size=1, k=L + 1, window=1,
+                       q_offset=L)
+    ra = oracle.full_attn_index(pa, q, k_aug, v_aug)
+    pr = oracle.Params(1, 2, 1, d, 1, L, mode="token", block_size=1, k=L, window=1,
+                       q_offset=L - 1)
+    rr = oracle.full_attn_index(pr, q, k, v)
+    o_g = rr["o"][0][None, :, None, :]                     # [1, 2, 1, d]
+    lse_g = rr["lse"][0][None, :, None]
+    o, lse, _ = oracle.gate_sink(o_g, lse_g, sink_g=s)
+    np.testing.assert_allclose(o[0, :, 0], ra["o"][0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse[0, :, 0], ra["lse"][0], rtol=0, atol=1e-12)
+
+
+def test_gate_identities():
+    """sigma(0) = 1/2 on both branches; sigma(z) + sigma(-z) = 1, so equal
+    branch outputs with opposite gate logits give that output back; a very
+    negative gate logit removes its branch."""
+    o_g = _rand((2, 3, 5, 4), 41)
+    o_l = _rand((2, 3, 5, 4), 42)
+    lse_g = _rand((2, 3, 5), 43)
+    lse_l = _rand((2, 3, 5), 44)
+    z = _rand((2, 3, 5), 45, std=3.0)
+    zero = np.zeros((2, 3, 5))
+    o, lg, ll = oracle.gate_sink(o_g, lse_g, o_l, lse_l, z_g=zero, z_l=zero)
+    np.testing.assert_allclose(o, 0.5 * (o_g + o_l), rtol=0, atol=1e-14)
+    np.testing.assert_array_equal(lg, lse_g)
+    np.testing.assert_array_equal(ll, lse_l)
+    o, _, _ = oracle.gate_sink(o_g, lse_g, o_g, lse_g, z_g=z, z_l=-z)
+    np.testing.assert_allclose(o, o_g, rtol=0, atol=1e-14)
+    o, _, _ = oracle.gate_sink(o_g, lse_g, o_l, lse_l, z_g=z, z_l=np.full_like(z, -800.0))
+    np.testing.assert_allclose(o, o_g / (1.0 + np.exp(-z))[..., None], rtol=0, atol=1e-14)
+
+
+def test_sink_on_an_empty_branch():
+    """A branch that kept no key (o = 0, lse = -inf) keeps o' = 0 and gets
+    lse' = s: the sink is then the whole softmax mass."""
+    o_g = np.zeros((1, 2, 3, 4))
+    lse_g = np.full((1, 2, 3), -np.inf)
+    o, lse, _ = oracle.gate_sink(o_g, lse_g, sink_g=[0.25, -2.0])
+    assert np.all(o == 0.0)
+    np.testing.assert_array_equal(lse[0, :, 0], [0.25, -2.0])

@@ -36,6 +36,14 @@ MUTANTS = {
                           "const int lo = t - p->window > 0 ? t - p->window : 0;"),
     "query_row_transposed": ("((size_t)b * p->hq + h) * p->t_q + j)",
                              "((size_t)h * p->batch + b) * p->t_q + j)"),
+    "sink_share_inverted": ("const double fg = s_g ? exp(lse_g[e] - lg) : 1.0;",
+                            "const double fg = s_g ? exp(lg - lse_g[e]) : 1.0;"),
+    "sink_lse_not_updated": ("const double lg = s_g ? log_add_exp(lse_g[e], s_g[e]) : lse_g[e];",
+                             "const double lg = lse_g[e];"),
+    "gate_sign_flipped": ("const double gg = z_g ? 1.0 / (1.0 + exp(-z_g[e])) : 1.0;",
+                          "const double gg = z_g ? 1.0 / (1.0 + exp(z_g[e])) : 1.0;"),
+    "local_gate_reads_global": ("gl = z_l ? 1.0 / (1.0 + exp(-z_l[e])) : 1.0;",
+                                "gl = z_l ? 1.0 / (1.0 + exp(-z_g[e])) : 1.0;"),
 }
 
 PINS = [
@@ -51,6 +59,9 @@ PINS = [
     lambda: pins.test_block_sparse_masks_future_keys_inside_a_selected_block(),
     lambda: pins.test_local_window_branch_matches_banded_library_attention(),
     lambda: pins.test_retained_mass_decomposition_and_bound(),
+    lambda: pins.test_sink_is_an_extra_key_with_zero_value(),
+    lambda: pins.test_gate_identities(),
+    lambda: pins.test_sink_on_an_empty_branch(),
 ]
 
 

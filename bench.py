@@ -393,6 +393,7 @@ def run_ours(args, rank, world, device):
     full_key = "full_index_gbs" if flops is None else "full_index_tflops"
 
     e2e = run_e2e(args, blk, w, stream, ideal, world, device) if not args.no_e2e else None
+    gate_sink = None if w.decode else time_gate_sink(blk, w, stream, peaks)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
@@ -415,8 +416,47 @@ def run_ours(args, rank, world, device):
                   "hbm_gbs": peaks["hbm_gbs"], "source": peak_kind},
         "roofline": roof, "gpu_launches": launches, "clocks": clocks.summary(),
         "e2e": e2e,
+        "gate_sink": gate_sink,
     }
     return line
+
+
+def time_gate_sink(blk, w, stream, peaks, reps=10):
+    """The sparse-layer output epilogue (per-head sinks, sigmoid-gate fusion of
+    the branches: hs_sparse_gate_sink) on layer 0's branch outputs, timed on its
+    own after the step (it is not part of the step).  Algorithmic bytes: the
+    branch outputs and lse read, gate pre-activations read, the fused output and
+    the updated lse written."""
+    hs = blk.hs
+    g = torch.Generator(device="cpu").manual_seed(5)
+    two = blk.ol[0] is not None
+    nb = 2 if two else 1
+    sink = [torch.randn(w.hq, generator=g).to(blk.dev) for _ in range(nb)]
+    gate = [torch.randn(w.batch, w.hq, w.tq, generator=g).to(blk.dev) for _ in range(nb)]
+    lse = [blk.lg[0].clone()] + ([blk.ll[0].clone()] if two else [])
+    o = torch.empty_like(blk.og[0])
+
+    def call():
+        hs.hs_sparse_gate_sink(blk.p, blk.og[0], lse[0], o, blk.ol[0], lse[1] if two else None,
+                               sink[0], sink[1] if two else None, gate[0],
+                               gate[1] if two else None, stream)
+    for _ in range(3):
+        call()
+    e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    rows = w.batch * w.hq * w.tq
+    elt = 2 if w.dtype == "bf16" else 4
+    nbytes = rows * (w.head_dim * elt * (nb + 1) + 4 * 3 * nb)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"kernel": "gate_sink_kernel", "ms": ms, "bytes": nbytes, "gbs": gbs,
+            "frac_of_hbm": gbs / peaks["hbm_gbs"], "branches": nb,
+            "note": "sparse-layer output epilogue, timed alone after the step"}
 
 
 def capture_step(blk, w, device):

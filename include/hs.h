@@ -128,6 +128,31 @@ hs_status hs_sparse_attn_reuse(const hs_params* p, const void* q_sparse, const v
                                void* o_local, float* lse_local, void* workspace,
                                size_t ws_bytes, void* stream);
 
+/*
+ * Output of a sparse layer: a per-head sink in each branch, then the sigmoid
+ * gates that fuse the branches ("HySparse 混合稀疏注意力（一）", the section on
+ * the two sigmoid gates; "HySparse: ..." 3.3, branch fusion, and the papers'
+ * configuration notes on per-head sink biases in the sparse and window
+ * branches).  For every row (b, h, t), in fp32:
+ *     f_x = e^lse_x / (e^lse_x + e^sink_x[h])   (1 without a sink)
+ *     o   = sigmoid(gate_global) f_g o_global + sigmoid(gate_local) f_l o_local
+ * and lse_x is replaced IN PLACE by log(e^lse_x + e^sink_x[h]): the sink is
+ * one more logit with a zero value vector in the branch's softmax.
+ * o_global, o_local, o: [batch][hq][t_q][head_dim], p->dtype (bf16 or fp32);
+ *           o may be o_global or o_local.
+ * lse_global, lse_local: float [batch][hq][t_q] (as hs_sparse_attn_reuse writes them).
+ * o_local / lse_local: both or neither (neither: one branch, e.g. HySparse2).
+ * sink_global, sink_local: float [hq] or NULL (no sink); gate_global,
+ *           gate_local: float [batch][hq][t_q] pre-activations or NULL (gate 1);
+ *           the local ones only with a local branch.
+ * p: batch, hq, hkv, head_dim (64 or 128), t_q and dtype as for the layer.
+ * One elementwise kernel; asynchronous on `stream`; pointers 16-byte aligned.
+ */
+hs_status hs_sparse_gate_sink(const hs_params* p, const void* o_global, float* lse_global,
+                              const void* o_local, float* lse_local, const float* sink_global,
+                              const float* sink_local, const float* gate_global,
+                              const float* gate_local, void* o, void* stream);
+
 typedef enum { HS_DECODE_FULL_INDEX = 0, HS_DECODE_SPARSE = 1 } hs_decode_kind;
 
 /*

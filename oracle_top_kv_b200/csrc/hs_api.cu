@@ -20,6 +20,7 @@
 #include "token_select_tc.cu"
 #include "noalloc.cu"
 #include "sparse.cu"
+#include "gate_sink.cu"
 
 namespace hs {
 static std::atomic<uint64_t> g_launches{0};
@@ -240,6 +241,28 @@ hs_status hs_decode_sparse_noalloc(const hs_params* p, const void* q, const void
     return launched(2, [&] {
         return hs::launch_decode_sparse_noalloc(kp, q, k_cache, v_cache, seq_len, idx, idx_count,
                                                 o, lse, st);
+    });
+}
+
+hs_status hs_sparse_gate_sink(const hs_params* p, const void* o_global, float* lse_global,
+                              const void* o_local, float* lse_local, const float* sink_global,
+                              const float* sink_local, const float* gate_global,
+                              const float* gate_local, void* o, void* stream) {
+    KParams kp;
+    hs_status s = resolve(p, false, &kp);
+    if (s != HS_OK) return s;
+    if (!ok_ptr(o_global) || !ok_ptr(lse_global) || !ok_ptr(o) || !ok_opt(o_local) ||
+        !ok_opt(lse_local) || !ok_opt(sink_global) || !ok_opt(sink_local) ||
+        !ok_opt(gate_global) || !ok_opt(gate_local))
+        return HS_ERR_INVALID_ARG;
+    // the local branch comes with its lse; its sink and gate only with it
+    if ((o_local == nullptr) != (lse_local == nullptr)) return HS_ERR_INVALID_ARG;
+    if (!o_local && (sink_local || gate_local)) return HS_ERR_INVALID_ARG;
+    if (kp.t_q == 0) return HS_OK;
+    return launched(1, [&] {
+        return hs::launch_gate_sink(kp, p->dtype, o_global, lse_global, o_local, lse_local,
+                                    sink_global, sink_local, gate_global, gate_local, o,
+                                    static_cast<cudaStream_t>(stream));
     });
 }
 

@@ -72,6 +72,12 @@ cudaError_t launch_decode_sparse_split(const KParams& p, const void* q, const vo
 // Token-mode selection on the tensor cores (bf16, d = 128, 16 heads per group,
 // k - w <= 1024); reads lse from the attention pass.
 bool token_select_tc_supported(const KParams& p, int dtype);
+// Sparse-layer output: per-head sinks and sigmoid-gate fusion of the branches
+// (gate_sink.cu).  o_l / lse_l null: one branch; sink / gate null: none.
+cudaError_t launch_gate_sink(const KParams& p, int dtype, const void* o_g, float* lse_g,
+                             const void* o_l, float* lse_l, const float* sink_g,
+                             const float* sink_l, const float* z_g, const float* z_l, void* o,
+                             cudaStream_t st);
 cudaError_t launch_token_select_tc(const KParams& p, const void* q, const void* k,
                                    const float* lse, int32_t* idx, int32_t* cnt, float* sel,
                                    cudaStream_t st);

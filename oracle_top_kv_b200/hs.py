@@ -72,6 +72,7 @@ def load(path: str = LIB_PATH):
     lib.hs_sparse_attn_reuse.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, P, P, S, P]
     lib.hs_decode_step.argtypes = [PP, I32, P, P, P, P, P, P, P, P, P, P, S, P]
     lib.hs_decode_sparse_noalloc.argtypes = [PP, P, P, P, P, P, P, P, P, P]
+    lib.hs_sparse_gate_sink.argtypes = [PP, P, P, P, P, P, P, P, P, P, P]
     lib.hs_workspace_size.argtypes = [PP, I32]
     lib.hs_workspace_size.restype = S
     lib.hs_device_status.argtypes = [P, ctypes.POINTER(I32)]
@@ -80,7 +81,7 @@ def load(path: str = LIB_PATH):
     lib.hs_launch_count.argtypes = []
     lib.hs_launch_count.restype = ctypes.c_uint64
     for name in ("hs_full_attn_index", "hs_sparse_attn_reuse", "hs_decode_step",
-                 "hs_device_status", "hs_decode_sparse_noalloc"):
+                 "hs_device_status", "hs_decode_sparse_noalloc", "hs_sparse_gate_sink"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -137,6 +138,19 @@ def hs_sparse_attn_reuse(p, q_sparse, k_f, v_f, idx, idx_count, k_local, v_local
                                     _ptr(o_global), _ptr(lse_global), _ptr(o_local),
                                     _ptr(lse_local), wp, wb, _stream(stream)),
            "hs_sparse_attn_reuse")
+
+
+def hs_sparse_gate_sink(p, o_global, lse_global, o, o_local=None, lse_local=None,
+                        sink_global=None, sink_local=None, gate_global=None, gate_local=None,
+                        stream=None):
+    """Per-head sinks and sigmoid-gate fusion of a sparse layer's branches
+    (include/hs.h); updates lse_global / lse_local in place."""
+    lib = load()
+    _check(lib.hs_sparse_gate_sink(ctypes.byref(p), _ptr(o_global), _ptr(lse_global),
+                                   _ptr(o_local), _ptr(lse_local), _ptr(sink_global),
+                                   _ptr(sink_local), _ptr(gate_global), _ptr(gate_local), _ptr(o),
+                                   _stream(stream)),
+           "hs_sparse_gate_sink")
 
 
 def hs_decode_step(p, kind, q, k_cache, v_cache, seq_len, idx, idx_count, o, lse=None,

@@ -118,3 +118,23 @@ def test_workspace_sizes(lib):
     assert hs.hs_workspace_size(p, hs.HS_WS_DECODE_FULL) > 0
     with pytest.raises(hs.HsError):
         hs.hs_workspace_size(_p(hq=30), hs.HS_WS_FULL)
+
+
+def _gate_sink(p, o_g=FAKE, lse_g=FAKE, o_l=None, lse_l=None, s_g=None, s_l=None, z_g=None,
+               z_l=None, o=FAKE):
+    return hs.load().hs_sparse_gate_sink(ctypes.byref(p), o_g, lse_g, o_l, lse_l, s_g, s_l, z_g,
+                                         z_l, o, None)
+
+
+def test_gate_sink_argument_checks(lib):
+    p = _p()
+    bad = hs.HS_ERR_INVALID_ARG
+    assert _gate_sink(p, o_l=FAKE) == bad                  # local output without its lse
+    assert _gate_sink(p, lse_l=FAKE) == bad                # local lse without its output
+    assert _gate_sink(p, s_l=FAKE) == bad                  # local sink without a local branch
+    assert _gate_sink(p, z_l=FAKE) == bad                  # local gate without a local branch
+    assert _gate_sink(p, o=None) == bad                    # no output
+    assert _gate_sink(p, o_g=FAKE + 8) == bad              # misaligned
+    assert _gate_sink(p, z_g=FAKE + 4) == bad
+    assert _gate_sink(_p(head_dim=96)) == hs.HS_ERR_UNSUPPORTED
+    assert _gate_sink(_p(t_q=0, t_kv=4)) == hs.HS_OK       # nothing to do, nothing launched

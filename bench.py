@@ -245,19 +245,29 @@ def sparse_on_tensor_cores(w):
             w.block_size == 64 and w.ksel <= 16 and 128 % (w.hq // w.hkv) == 0)
 
 
+def code_hash(paths):
+    """sha256 of the sources' code: comments and whitespace removed, so that a
+    comment edit does not mark a capture as stale while any code change does."""
+    import re
+    h = hashlib.sha256()
+    for f in paths:
+        text = open(os.path.join(ROOT, f), encoding="utf-8").read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
+    return h.hexdigest()
+
+
 def traffic_for(kernel, workload):
     """Per-launch DRAM bytes from the committed ncu summary, if the kernel's
-    source is unchanged since the capture; else None."""
+    source code is unchanged since the capture; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     d = json.load(open(path)).get(f"{kernel}@{workload}")
     if not d:
         return None
-    h = hashlib.sha256()
-    for f in d.get("sources", []):
-        h.update(open(os.path.join(ROOT, f), "rb").read())
-    return d["bytes_per_launch"] if h.hexdigest() == d.get("sha256") else None
+    return d["bytes_per_launch"] if code_hash(d.get("sources", [])) == d.get("sha256") else None
 
 
 def workload_of(args):

@@ -2,7 +2,8 @@
 // layer (full_tc.cu) and the row-grouped sparse layer (sparse_tc.cu).
 //
 // A CTA runs two 128-row Q tiles over a list of 64-key tiles that both share.
-// Warp 0 is the TMA producer, warp 1 owns TMEM, warps 2..9 are two softmax
+// Warp 0 is the TMA producer (K and V through rings of their own), warp 1
+// owns TMEM, warps 2..9 are two softmax
 // warpgroups with one thread per row, and one thread per Q tile (warp 1 for
 // tile 0, warp 10 for tile 1) issues that tile's MMAs:
 //   S = Q K^T  (M = 128, N = 64, K = 16 x 8) into one of two TMEM buffers,

@@ -19,7 +19,8 @@
 // loaded once for the whole group.  A CTA runs two consecutive Q tiles that
 // share every K/V tile; their softmax warpgroups alternate on the tensor core.
 // Warp roles:
-//   warp 0       TMA producer (both Q tiles once; K and V tiles, 3-stage ring)
+//   warp 0       TMA producer (both Q tiles once; K and V tiles through
+//                rings of 3 stages each)
 //   warp 1       TMEM owner and MMA issuer of Q tile 0; warp 10 issues for
 //                Q tile 1: S = Q K^T into one of two TMEM buffers, then
 //                O += P V (P from shared memory, V MN-major).  One issuing
@@ -27,8 +28,8 @@
 //                both tiles as fast as the tensor core runs them.
 //   warps 2..9   two softmax warpgroups, one thread per row (TMEM lane):
 //                online softmax with lazy rescaling of O (only when the max
-//                grows by > 2^8), P to shared memory, block-score capture,
-//                epilogue.
+//                grows by > 2^8), a third of the exponentials on the FMA
+//                pipe, P to shared memory, block-score capture, epilogue.
 // All waits are bounded (tc_ptx.cuh); a timeout aborts the CTA cleanly.
 #include "flash_tc.cuh"
 #include "hs_common.cuh"

@@ -15,10 +15,11 @@
 // not select (masked to -inf), but each K/V block is read once per CTA
 // instead of once per row, and both contractions run on the tensor cores.
 //
-// Warp roles as in full_tc.cu: warp 0 TMA producer (Q once, union blocks
-// through a 2-stage K/V ring), warp 1 TMEM owner and MMA issuer of Q tile 0,
-// warp 10 MMA issuer of Q tile 1, warps 2..9
-// two softmax warpgroups (one thread per row).  Supported: bf16, d = 128,
+// Warp roles as in full_tc.cu: warp 0 TMA producer (Q once, the union blocks'
+// K and V through 3- and 2-stage rings), warp 1 TMEM owner and MMA issuer of
+// Q tile 0, warp 10 MMA issuer of Q tile 1, warps 2..9 two softmax warpgroups
+// (one thread per row; a quarter of the exponentials on the FMA pipe, exact
+// zeros for masked keys).  Supported: bf16, d = 128,
 // block mode with B = 64 (= the key tile), 128 % g == 0, and a union of at
 // most kMaxUnion blocks (2 * (128/g) positions x k/B ids).  The window branch
 // over the layer's own K'/V' (keys t-w+1..t) is a second launch of the same

@@ -100,3 +100,20 @@ def test_sparse_useful_flops_brute_force():
                 window = {i for i in range(max(0, t - w.window + 1), t + 1)} if w.swa_branch else set()
                 pairs += (len(keys) + len(window)) * (w.hq // w.hkv)
     assert bench.sparse_useful_flops(w, blk) == pairs * 4 * w.head_dim
+
+
+def test_code_hash_ignores_comments_not_code(tmp_path, monkeypatch):
+    """The DRAM-traffic table is tied to a kernel's code: a comment or spacing
+    edit keeps its hash, any code edit changes it."""
+    import importlib
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    bench = importlib.import_module("bench")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    f = tmp_path / "k.cu"
+    f.write_text("// header\nint f(int x) { /* twice */ return 2 * x; }\n")
+    h0 = bench.code_hash(["k.cu"])
+    f.write_text("// a longer header\n\nint f(int x) {\n    // doubled\n    return 2 * x;\n}\n")
+    assert bench.code_hash(["k.cu"]) == h0
+    f.write_text("// header\nint f(int x) { /* twice */ return 3 * x; }\n")
+    assert bench.code_hash(["k.cu"]) != h0

@@ -39,7 +39,7 @@ constexpr int kSets = kPos / kPP;          // scorer sets of four warps
 constexpr int kScorers = 4 * kSets;        // scorer warps
 constexpr int kHd = 128;
 constexpr int kStages = 2;       // K ring (the MMA is far ahead of the scorers)
-constexpr int kSBufs = 4;        // S^T buffers in TMEM: the two scorer sets may drift 3 tiles
+constexpr int kSBufs = 4;        // S^T buffers in TMEM: the scorer sets may drift 3 tiles apart
 constexpr int kThreads = 64 + 32 * kScorers;
 constexpr int kMaxRanked = 1024;            // k - w handled here
 // Per-position buffer entries: the k - w kept, two tiles of admissions

@@ -3,15 +3,23 @@
 
 A step is one pass of the hot path over one batch of synthetic input: the
 full-attention layer with its oracle indexer, then the block's sparse layers
-reusing its K^F/V^F and index set (HySparse 7B-dense-shaped block-level
-prefill by default: b=2, T=16384, 32/8 heads, d=128, bf16, B=64, k=1024,
-1 full : 3 sparse, each sparse layer with its own 128-token window K'/V').
+reusing its K^F/V^F and index set.  Default workload: the 1M-token HySparse2
+prefill chunk (8192 queries at the end of a 2^20-token causal prefix, 64/4
+heads, d=128, bf16, token top-k with k=1024 including the last w=128, then
+11 sparse layers); --workload picks another one.
 
-Printed value (rank 0, one JSON line): the step's peak-normalised throughput,
-    (F_full / P_tensor + B_sparse / P_hbm) / t_step, summed over ranks,
-i.e. the fraction of one B200's roofline the step achieves (N x that for N
-replicas).  The line also carries the two halves of the metric separately:
-full+index TFLOP/s and sparse-reuse K/V GB/s, each with its fraction of peak.
+Printed value (rank 0, one JSON line): the fraction of one B200's roofline
+the step reaches, summed over ranks (N x that for N replicas):
+    value = (F_full / P_tensor + n_sparse * t_sparse_min) / t_step
+with t_sparse_min the sparse layer's own physical bound,
+    max(useful FLOPs / P_tensor, least bytes / P_hbm),
+useful FLOPs = 4 d per (query head, kept key) and least bytes = every
+distinct K/V row the layer's queries keep read once, plus q', outputs, lse
+and index rows.  Decode steps are HBM-bound: (cache bytes + n_sparse *
+selected-row bytes) / P_hbm.  P_tensor is the measured burst bf16 peak when
+the SM clock stayed at its maximum with no power cap in the timed region,
+else the sustained one (the line says which).  The pages' logical gather
+rate ("reads k+w tokens" per query) is reported beside it as sparse_kv_gbs.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -282,6 +290,70 @@ def workload_of(args):
     return w
 
 
+def tensor_peak(peaks, clk):
+    """The bf16 tensor peak that applies to the timed region: the burst figure
+    while the median SM clock stayed within 3% of its maximum with no power
+    cap, the sustained (power-capped) one otherwise."""
+    sm, mx, reasons = clk.get("sm_mhz"), clk.get("sm_max_mhz"), clk.get("reasons") or []
+    if sm and mx and sm >= 0.97 * mx and "sw_power_cap" not in reasons:
+        return peaks["bf16_tflops"], "bf16_tflops"
+    return peaks["bf16_tflops_sustained"], "bf16_tflops_sustained"
+
+
+def sparse_bound(w, blk, p_tensor, p_hbm):
+    """A sparse layer's physical roofline: max(useful FLOPs / P_tensor, least
+    bytes / P_hbm).  Prefill only (decode steps are counted in bytes)."""
+    if w.decode:
+        return {"bound": "hbm", "t_min": 0.0}
+    uf = sparse_useful_flops(w, blk)
+    urows = A.sparse_unique_rows_from_index(blk.idx, blk.cnt, w.mode, w.block_size, w.q_offset)
+    ulocal = (w.batch * w.hkv * min(w.t, w.q_offset + w.tq)) if w.swa_branch else 0
+    elt = 2 if w.dtype == "bf16" else 4
+    ub = A.sparse_layer_unique_bytes(urows, w.batch, w.hq, w.tq, w.head_dim, elt, w.ksel,
+                                     w.hkv, ulocal, local=w.swa_branch)
+    t_c, t_m = uf / p_tensor, ub / p_hbm
+    return {"bound": "tensor" if t_c >= t_m else "hbm", "useful_flops": uf, "least_bytes": ub,
+            "distinct_kv_rows": urows + ulocal, "t_min": max(t_c, t_m)}
+
+
+def config_of(w, world, launch):
+    return {"workload": w.name, "batch": w.batch, "seq_len": w.t, "hq": w.hq,
+            "hkv": w.hkv, "head_dim": w.head_dim, "mode": w.mode,
+            "block_size": w.block_size, "k": w.k, "window": w.window,
+            "decode": w.decode, "t_q": w.tq, "q_offset": w.q_offset,
+            "sparse_layers": w.n_sparse, "parallelism": f"replicas{world}",
+            "l2": "inputs larger than L2 (K^F+V^F alone exceed 126 MB)",
+            "launch": launch}
+
+
+def kernel_breakdown(blk, w, sh):
+    """Device time of each of the library's kernels in one untimed step (CUPTI
+    kernel records through torch.profiler): which kernel dominates."""
+    try:
+        from torch.profiler import ProfilerActivity, profile
+        torch.cuda.synchronize()
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            blk.full(sh)
+            for layer in range(w.n_sparse):
+                blk.sparse(layer, sh)
+            torch.cuda.synchronize()
+        agg = {}
+        for e in prof.events():
+            if e.device_type.name != "CUDA":
+                continue
+            name = e.name.split("(")[0].replace("void ", "")
+            t = getattr(e, "device_time_total", None)
+            if t is None:
+                t = e.cuda_time_total
+            n, tot = agg.get(name, (0, 0.0))
+            agg[name] = (n + 1, tot + t / 1e3)
+        total = sum(v[1] for v in agg.values()) or 1.0
+        return [{"kernel": k, "launches": n, "ms": ms, "share": ms / total}
+                for k, (n, ms) in sorted(agg.items(), key=lambda kv: -kv[1][1])]
+    except Exception as e:  # the breakdown is a diagnostic; never fail the bench for it
+        return {"error": repr(e)[:200]}
+
+
 def run_ours(args, rank, world, device):
     from oracle_top_kv_b200 import hs
     hs.load()
@@ -319,19 +391,31 @@ def run_ours(args, rank, world, device):
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
+    nvtx = torch.cuda.nvtx
     for s in range(args.steps):
+        nvtx.range_push(f"step {s}")
         evs[s][0].record(stream)
         if graphs:
+            nvtx.range_push("full layer + index")
             graphs[0].replay()
+            nvtx.range_pop()
             evs[s][1].record(stream)
+            nvtx.range_push(f"{w.n_sparse} sparse layers")
             graphs[1].replay()
+            nvtx.range_pop()
             evs[s][2].record(stream)
+            nvtx.range_pop()
             continue
+        nvtx.range_push("full layer + index")
         blk.full(sh)
+        nvtx.range_pop()
         evs[s][1].record(stream)
         for layer in range(w.n_sparse):
+            nvtx.range_push(f"sparse layer {layer}")
             blk.sparse(layer, sh)
+            nvtx.range_pop()
             evs[s][2 + layer].record(stream)
+        nvtx.range_pop()
     t1.record(stream)
     torch.cuda.synchronize(device)
     launches = hs.hs_launch_count() - launches0
@@ -349,17 +433,19 @@ def run_ours(args, rank, world, device):
         sparse_ms = [evs[s][1 + l].elapsed_time(evs[s][2 + l]) for s in range(args.steps)
                      for l in range(w.n_sparse)]
     ms_step = total_ms / args.steps
-
-    p_tensor = peaks["bf16_tflops_sustained"] * 1e12
+    clk = clocks.summary()
+    p_tensor_tf, tensor_kind = tensor_peak(peaks, clk)
+    p_tensor = p_tensor_tf * 1e12
     p_hbm = peaks["hbm_gbs"] * 1e9
     full_s = statistics.mean(full_ms) / 1e3
     sparse_s = statistics.mean(sparse_ms) / 1e3
     sparse_gbs = sbytes / sparse_s / 1e9
     tokens = w.batch * w.tq
+    sp_bound = sparse_bound(w, blk, p_tensor, p_hbm)
     if flops is not None:
-        ideal = flops / p_tensor + w.n_sparse * sbytes / p_hbm
-        full_rate, full_unit, full_peak = flops / full_s / 1e12, "TFLOP/s", peaks["bf16_tflops_sustained"]
-        full_bound, full_peak_src = "tensor", f"{peak_kind} bf16_tflops_sustained"
+        ideal = flops / p_tensor + w.n_sparse * sp_bound["t_min"]
+        full_rate, full_unit, full_peak = flops / full_s / 1e12, "TFLOP/s", p_tensor_tf
+        full_bound, full_peak_src = "tensor", f"{peak_kind} {tensor_kind}"
     else:
         ideal = (full_bytes + w.n_sparse * sbytes) / p_hbm
         full_rate, full_unit, full_peak = full_bytes / full_s / 1e9, "GB/s", peaks["hbm_gbs"]
@@ -367,64 +453,69 @@ def run_ours(args, rank, world, device):
     value = world * ideal / (ms_step / 1e3)
     # dominant kernel: the one with the larger share of the step
     if sum(full_ms) >= sum(sparse_ms):
-        roof = {"kernel": "decode_full_index" if w.decode else "full_attn_index",
-                "bound": full_bound, "achieved": full_rate, "peak": full_peak,
+        name = "decode_full_index" if w.decode else "full_attn_index"
+        roof = {"kernel": name, "bound": full_bound, "achieved": full_rate, "peak": full_peak,
                 "unit": full_unit, "frac": full_rate / full_peak,
-                "traffic": traffic_for("decode_full_index" if w.decode else "full_attn_index",
-                                       w.name),
-                "peak_source": full_peak_src,
+                "traffic": traffic_for(name, w.name), "peak_source": full_peak_src,
                 "work_per_launch": flops if flops is not None else full_bytes,
                 "avg_launch_ms": full_s * 1e3}
-    elif not w.decode and sparse_on_tensor_cores(w):
-        uf = sparse_useful_flops(w, blk)
-        rate = uf / sparse_s / 1e12
-        roof = {"kernel": "sparse_attn_reuse", "bound": "tensor", "achieved": rate,
-                "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                "frac": rate / peaks["bf16_tflops_sustained"],
-                "traffic": traffic_for("sparse_attn_reuse", w.name),
-                "peak_source": f"{peak_kind} bf16_tflops_sustained",
-                "work_per_launch": uf, "avg_launch_ms": sparse_s * 1e3,
-                "note": "block mode runs on the tensor cores over each CTA's union of its rows' "
-                        "selected blocks; work = the useful FLOPs, 4*d per (query head, kept "
-                        "key), while the MMAs issued cover every union block for every row "
-                        "(about 4x); the pages' logical-bytes rate is sparse_kv_gbs"}
+        if flops is not None and w.mode == "token":
+            roof["note"] = ("one C-ABI call = the tensor-core attention pass, then the token "
+                            "selection pass (which recomputes QK^T: +50% tensor work); work = "
+                            "the algorithmic FLOPs 4*d*hq per causal pair")
+    elif w.decode:
+        roof = {"kernel": "decode_sparse", "bound": "hbm", "achieved": sparse_gbs,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": sparse_gbs / peaks["hbm_gbs"],
+                "traffic": traffic_for("decode_sparse", w.name),
+                "peak_source": f"{peak_kind} hbm_gbs", "work_per_launch": sbytes,
+                "avg_launch_ms": sparse_s * 1e3}
     else:
-        roof = {"kernel": "decode_sparse" if w.decode else "sparse_attn_reuse", "bound": "hbm",
-                "achieved": sparse_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": sparse_gbs / peaks["hbm_gbs"],
-                "traffic": traffic_for("decode_sparse" if w.decode else "sparse_attn_reuse",
-                                       w.name),
-                "peak_source": f"{peak_kind} hbm_gbs",
-                "work_per_launch": sbytes, "avg_launch_ms": sparse_s * 1e3,
-                "note": "work = the logical K/V rows the index sets make the queries read "
-                        "(the pages' accounting); the kernels read far fewer bytes from DRAM "
-                        "(L2-resident rows; block mode reads each CTA's union of selected "
-                        "blocks once), so achieved exceeds the HBM peak: see traffic"}
+        sb = sp_bound
+        if sb["bound"] == "tensor":
+            ach, pk, unit, wk = sb["useful_flops"] / sparse_s / 1e12, p_tensor_tf, "TFLOP/s", \
+                sb["useful_flops"]
+        else:
+            ach, pk, unit, wk = sb["least_bytes"] / sparse_s / 1e9, peaks["hbm_gbs"], "GB/s", \
+                sb["least_bytes"]
+        roof = {"kernel": "sparse_attn_reuse", "bound": sb["bound"], "achieved": ach,
+                "peak": pk, "unit": unit, "frac": ach / pk,
+                "traffic": traffic_for("sparse_attn_reuse", w.name),
+                "peak_source": f"{peak_kind} " + (tensor_kind if sb["bound"] == "tensor"
+                                                  else "hbm_gbs"),
+                "work_per_launch": wk, "avg_launch_ms": sparse_s * 1e3,
+                "note": "the sparse layer's physical bound: max(useful FLOPs / P_tensor, least "
+                        "bytes / P_hbm), useful FLOPs = 4*d per (query head, kept key), least "
+                        "bytes = distinct K/V rows kept + q' + outputs + index; the pages' "
+                        "logical-bytes rate is sparse_kv_gbs"}
     full_key = "full_index_gbs" if flops is None else "full_index_tflops"
 
+    kernels = kernel_breakdown(blk, w, sh) if not args.no_breakdown else None
     e2e = run_e2e(args, blk, w, stream, ideal, world, device) if not args.no_e2e else None
     gate_sink = None if w.decode else time_gate_sink(blk, w, stream, peaks)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": {"workload": w.name, "batch": w.batch, "seq_len": w.t, "hq": w.hq,
-                   "hkv": w.hkv, "head_dim": w.head_dim, "mode": w.mode,
-                   "block_size": w.block_size, "k": w.k, "window": w.window,
-                   "decode": w.decode, "t_q": w.tq, "q_offset": w.q_offset,
-                   "sparse_layers": w.n_sparse, "parallelism": f"replicas{world}",
-                   "l2": "inputs larger than L2 (step reads > 1 GB; K^F+V^F alone 134 MB)",
-                   "launch": "cuda graph replays (full-layer graph, sparse-layers graph)"
-                   if graphs else "per-call launches"},
+        "config": config_of(w, world, "cuda graph replays (full-layer graph, sparse-layers graph)"
+                            if graphs else "per-call launches"),
         full_key: full_rate * world,
         "full_index_frac_of_peak": full_rate / full_peak,
         "sparse_kv_gbs": sparse_gbs * world,
-        "sparse_frac_of_hbm_peak": sparse_gbs / peaks["hbm_gbs"],
+        "sparse_kv_gbs_note": "the pages' logical accounting: every K/V row each query's "
+                              "index set reads; rows shared between queries count once per "
+                              "query, so this rate can exceed the HBM peak",
+        "sparse_bound": {k: v for k, v in sp_bound.items() if k != "t_min"},
+        "sparse_frac_of_bound": sp_bound["t_min"] / sparse_s,
         "full_ms": full_s * 1e3, "sparse_ms_per_layer": sparse_s * 1e3,
         "tokens_per_s": world * tokens / (ms_step / 1e3),
-        "peaks": {"bf16_tflops_sustained": peaks["bf16_tflops_sustained"],
-                  "hbm_gbs": peaks["hbm_gbs"], "source": peak_kind},
-        "roofline": roof, "gpu_launches": launches, "clocks": clocks.summary(),
+        "peaks": {"bf16_tflops": peaks["bf16_tflops"],
+                  "bf16_tflops_sustained": peaks["bf16_tflops_sustained"],
+                  "hbm_gbs": peaks["hbm_gbs"], "source": peak_kind,
+                  "tensor_peak_used": tensor_kind,
+                  "rule": "burst while the median SM clock stays within 3% of its maximum "
+                          "with no power cap; sustained otherwise"},
+        "roofline": roof, "gpu_launches": launches, "clocks": clk,
+        "kernels": kernels,
         "e2e": e2e,
         "gate_sink": gate_sink,
     }
@@ -545,7 +636,14 @@ def run_e2e(args, blk, w, stream, ideal, world, device):
 
 # --------------------------------------------------------------- oracle arm
 def oracle_inputs(w):
+    """The step's inputs on the host.  K^F/V^F are held in float64 (the oracle's
+    arithmetic type) when that fits in 10 GB, so that a sample's time is the
+    oracle's work on resident inputs -- as the GPU's is -- rather than a
+    conversion of the whole cache; otherwise each sample converts the units it
+    touches."""
     q, k, v, _ = wl.full_layer_inputs(w, device="cpu")
+    if 2 * k.numel() * 8 <= 10 << 30:
+        k, v = k.double().numpy(), v.double().numpy()
     layers = []
     for layer in range(w.n_sparse):
         qs = wl.sparse_layer_query(w, layer, device="cpu")
@@ -598,28 +696,51 @@ def oracle_sample_time(w, inputs, budget_rows=48, seed=0):
     return est_full + est_sparse, sample, oracle.num_threads()
 
 
-def cpu_value(w, t_step):
+def cpu_ideal(w):
+    """The roofline time of one step (the numerator of value) for the CPU arms,
+    which have no GPU index set: the sparse layer's distinct rows are taken as
+    min(rows its queries read, visible keys) per unit, and the tensor peak is
+    the sustained one (the CPU arms have no GPU clock record)."""
     peaks, _ = load_peaks()
     p_hbm = peaks["hbm_gbs"] * 1e9
+    p_t = peaks["bf16_tflops_sustained"] * 1e12
     if w.decode:
         full_b = A.decode_full_bytes(w.batch, w.hkv, w.head_dim, [w.t] * w.batch, 2)
         sp = w.batch * w.hkv * min(w.k, w.t) * 2 * w.head_dim * 2
-        return (full_b + w.n_sparse * sp) / p_hbm / t_step
+        return (full_b + w.n_sparse * sp) / p_hbm
     flops = A.full_layer_flops(w.batch, w.hq, w.head_dim, w.tq, w.q_offset)
-    rows = w.batch * w.hkv * sum(min(w.k, w.q_offset + j + 1) for j in range(w.tq))
+    per_unit = sum(min(w.k, w.q_offset + j + 1) for j in range(w.tq))  # keys read per unit
+    visible = min(w.t, w.q_offset + w.tq)
     local = A.window_rows(w.batch, w.hkv, w.tq, w.window, w.q_offset) if w.swa_branch else 0
-    sbytes = A.sparse_layer_bytes(rows, w.batch, w.hq, w.tq, w.head_dim, 2, w.ksel, w.hkv, local)
-    ideal = (flops / (peaks["bf16_tflops_sustained"] * 1e12) + w.n_sparse * sbytes / p_hbm)
-    return ideal / t_step
+    uf = (w.batch * w.hkv * per_unit + local) * w.group * 4 * w.head_dim
+    urows = w.batch * w.hkv * min(per_unit, visible)
+    ulocal = w.batch * w.hkv * visible if w.swa_branch else 0
+    ub = A.sparse_layer_unique_bytes(urows, w.batch, w.hq, w.tq, w.head_dim, 2, w.ksel, w.hkv,
+                                     ulocal, local=w.swa_branch)
+    return flops / p_t + w.n_sparse * max(uf / p_t, ub / p_hbm)
+
+
+def cpu_value(w, t_step):
+    return cpu_ideal(w) / t_step
+
+
+def calibrate_rows(w, inputs, target_s, lo, hi):
+    """Rows per oracle sample so that one sample takes about target_s seconds."""
+    rows, took = lo, 0.0
+    for _ in range(4):
+        t0 = time.perf_counter()
+        oracle_sample_time(w, inputs, budget_rows=rows, seed=7)
+        took = time.perf_counter() - t0
+        if took >= 0.5 * target_s or rows >= hi:
+            break
+        rows = max(rows + 1, min(hi, int(rows * target_s / max(took, 1e-3))))
+    return rows
 
 
 def run_reference(args, w, world):
     inputs = oracle_inputs(w)
-    # Each oracle call converts the K/V prefix of every (batch, group) it
-    # touches to float64 once, a cost the whole step pays once per unit: the
-    # sample must hold many rows per unit for the extrapolation by row count
-    # to stay fair (decode samples whole units, whose conversion is their work).
-    budget = 12 if w.decode else 8192
+    hi = w.batch * w.hkv * 8 if w.decode else w.batch * w.hkv * w.tq
+    budget = calibrate_rows(w, inputs, 5.0, 4 if w.decode else 16, hi)
     for s in range(args.warmup):
         oracle_sample_time(w, inputs, budget_rows=budget, seed=1000 + s)
     times = []
@@ -630,10 +751,13 @@ def run_reference(args, w, world):
     t_step = statistics.mean(times)
     v = cpu_value(w, t_step)
     return {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": t_step * 1e3,
+            "ms_per_step_is": "extrapolated: each step times a bounded sample of the "
+                              "workload's rows and scales it to the whole step",
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": w.name, "batch": w.batch, "seq_len": w.t},
+            "config": config_of(w, world, "fp64 CPU oracle, OpenMP over the host cores"),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": "per step: " + sample},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -645,13 +769,15 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="hysparse_7b_block", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--workload", default="long_1m_chunk", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--batch", type=int, default=0, help="override the batch (reduced replica)")
     ap.add_argument("--seq", type=int, default=0, help="override the sequence length")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="time per-call launches instead of CUDA graph replays")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-breakdown", action="store_true",
+                    help="skip the per-kernel device-time breakdown (one untimed step)")
     args = ap.parse_args()
 
     rank, world, local = hdist.world()
@@ -668,18 +794,11 @@ def main():
         hdist.init("nccl", device)
     line = run_ours(args, rank, world, device)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        # grow the sample until it is about 10 s of oracle work (the first,
-        # small one also pays one-off set-up, so the scaling is repeated)
+        # a sample of about 10 s of oracle work (calibrated on smaller ones)
         inputs = oracle_inputs(w)
         max_rows = w.batch * w.hkv * 8 if w.decode else w.batch * w.hkv * w.tq
-        rows, took = 48, 0.0
-        for _ in range(4):
-            t0 = time.perf_counter()
-            t, sample, cores = oracle_sample_time(w, inputs, budget_rows=rows, seed=7)
-            took = time.perf_counter() - t0
-            if took >= 5.0 or rows >= max_rows:
-                break
-            rows = min(max_rows, int(rows * 10.0 / max(took, 1e-3)))
+        rows = calibrate_rows(w, inputs, 10.0, 4 if w.decode else 16, max_rows)
+        t, sample, cores = oracle_sample_time(w, inputs, budget_rows=rows, seed=7)
         line["cpu_baseline"] = {"value": cpu_value(w, t), "unit": UNIT, "cores": cores,
                                 "kind": "oracle", "sample": sample,
                                 "ms_per_step_extrapolated": t * 1e3}

@@ -91,3 +91,46 @@ def sparse_layer_bytes(kv_rows, batch, hq, t_q, d, elt, ksel, hkv, local_rows=0)
     outs = (2 if local_rows else 1) * batch * hq * t_q * (d * elt + 4)
     index = batch * hkv * t_q * (ksel + 1) * 4
     return kv + q + outs + index
+
+
+def sparse_unique_rows_from_index(idx, cnt, mode, block_size, q_offset=0):
+    """Distinct K/V rows the sparse layer's queries keep, summed over (batch,
+    group) units: the least it must read from memory, however its queries
+    share them.
+
+    idx [b, hkv, t_q, ksel] and cnt [b, hkv, t_q] (torch tensors).  Token
+    mode: the distinct token ids.  Block mode: the union of the kept keys, a
+    selected block kept up to the latest position among the rows selecting it.
+    """
+    import torch
+    b, hkv, tq, ksel = idx.shape
+    valid = torch.arange(ksel, device=idx.device).view(1, 1, 1, ksel) < cnt.unsqueeze(-1)
+    pos = (torch.arange(tq, device=idx.device) + q_offset).view(tq, 1).expand(tq, ksel)
+    total = 0
+    for bb in range(b):
+        for u in range(hkv):
+            m = valid[bb, u]
+            ids = idx[bb, u][m].long()
+            if ids.numel() == 0:
+                continue
+            if mode == "token":
+                total += int(torch.unique(ids).numel())
+                continue
+            # latest position selecting each block, then its keys up to there
+            last = torch.full((int(ids.max()) + 1,), -1, dtype=torch.long, device=idx.device)
+            last.scatter_reduce_(0, ids, pos[m].long(), reduce="amax")
+            blk = torch.arange(last.numel(), device=idx.device)
+            keep = (last - blk * block_size + 1).clamp(min=0, max=block_size)
+            total += int(keep[last >= 0].sum().item())
+    return total
+
+
+def sparse_layer_unique_bytes(unique_rows, batch, hq, t_q, d, elt, ksel, hkv, local_unique=0,
+                              local=False):
+    """Least memory traffic of a sparse layer: every distinct K/V row touched
+    once, q' read, o (and o_local) and lse written, the index rows read."""
+    kv = (unique_rows + local_unique) * 2 * d * elt
+    q = batch * hq * t_q * d * elt
+    outs = (2 if local else 1) * batch * hq * t_q * (d * elt + 4)
+    index = batch * hkv * t_q * (ksel + 1) * 4
+    return kv + q + outs + index

@@ -117,3 +117,32 @@ def test_code_hash_ignores_comments_not_code(tmp_path, monkeypatch):
     assert bench.code_hash(["k.cu"]) == h0
     f.write_text("// header\nint f(int x) { /* twice */ return 3 * x; }\n")
     assert bench.code_hash(["k.cu"]) != h0
+
+
+def test_sparse_unique_rows_brute_force():
+    """Distinct K/V rows a sparse layer touches (its least memory traffic),
+    counted by enumerating every row's kept keys into one set per unit."""
+    torch = pytest.importorskip("torch")
+    g = torch.Generator().manual_seed(11)
+    b, hkv, tq, off = 2, 3, 30, 9
+    for mode, B, ks in (("token", 1, 7), ("block", 4, 3)):
+        idx = torch.full((b, hkv, tq, ks), -1, dtype=torch.int32)
+        cnt = torch.zeros(b, hkv, tq, dtype=torch.int32)
+        want = 0
+        for bb in range(b):
+            for u in range(hkv):
+                keys = set()
+                for j in range(tq):
+                    t = off + j
+                    nc = t // B + 1
+                    c = int(torch.randint(0, min(ks, nc) + 1, (1,), generator=g))
+                    sel = torch.randperm(nc, generator=g)[:c].sort().values
+                    idx[bb, u, j, :c] = sel.to(torch.int32)
+                    cnt[bb, u, j] = c
+                    for r in sel.tolist():
+                        keys |= {i for i in range(r * B, (r + 1) * B) if i <= t}
+                want += len(keys)
+        assert A.sparse_unique_rows_from_index(idx, cnt, mode, B, q_offset=off) == want
+        got = A.sparse_layer_unique_bytes(want, b, 6, tq, 8, 2, ks, hkv)
+        assert got == want * 2 * 8 * 2 + b * 6 * tq * 8 * 2 + b * 6 * tq * (8 * 2 + 4) + \
+            b * hkv * tq * (ks + 1) * 4

@@ -137,6 +137,7 @@ class HybridBlock:
         self.p = hs.make_params(w.batch, w.hq, w.hkv, w.head_dim, w.tq, w.t, w.q_offset, w.dtype,
                                 w.mode, w.block_size, w.k, w.window)
         self.o, self.lse, self.idx, self.cnt, _ = hs.full_outputs(self.p, device)
+        self.ws_full = hs.workspace(self.p, hs.HS_WS_FULL, device)
         self.qs, self.kl, self.vl, self.og, self.lg, self.ol, self.ll = [], [], [], [], [], [], []
         for layer in range(w.n_sparse):
             qs = wl.sparse_layer_query(w, layer, device=device)
@@ -154,7 +155,7 @@ class HybridBlock:
 
     def full(self, stream):
         self.hs.hs_full_attn_index(self.p, self.q, self.k, self.v, self.o, self.lse, self.idx,
-                                   self.cnt, None, None, stream)
+                                   self.cnt, None, self.ws_full, stream)
 
     def sparse(self, layer, stream):
         self.hs.hs_sparse_attn_reuse(self.p, self.qs[layer], self.k, self.v, self.idx, self.cnt,

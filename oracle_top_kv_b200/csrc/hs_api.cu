@@ -18,6 +18,7 @@
 #include "full_tc.cu"
 #include "sparse_tc.cu"
 #include "token_select_tc.cu"
+#include "token_select_wide.cu"
 #include "noalloc.cu"
 #include "sparse.cu"
 #include "gate_sink.cu"
@@ -108,8 +109,6 @@ extern "C" {
 hs_status hs_full_attn_index(const hs_params* p, const void* q, const void* k, const void* v,
                              void* o, float* lse, int32_t* idx, int32_t* idx_count,
                              float* sel_scores, void* workspace, size_t ws_bytes, void* stream) {
-    (void)workspace;
-    (void)ws_bytes;
     KParams kp;
     hs_status s = resolve(p, false, &kp);
     if (s != HS_OK) return s;
@@ -128,6 +127,11 @@ hs_status hs_full_attn_index(const hs_params* p, const void* q, const void* k, c
             cudaError_t e =
                 hs::launch_full_tc(kp, q, k, v, o, lse, idx, idx_count, sel_scores, 0, st);
             if (e != cudaSuccess) return e;
+            // long scans: the wide selector, when the caller gave its workspace
+            if (hs::token_select_wide_applies(kp, p->dtype) && workspace != nullptr &&
+                aligned16(workspace) && ws_bytes >= hs::token_select_wide_workspace(kp))
+                return hs::launch_token_select_wide(kp, q, k, lse, idx, idx_count, sel_scores,
+                                                    workspace, ws_bytes, st);
             if (hs::token_select_tc_supported(kp, p->dtype))
                 return hs::launch_token_select_tc(kp, q, k, lse, idx, idx_count, sel_scores, st);
             return hs::launch_full_simt(kp, p->dtype, q, k, v, o, lse, idx, idx_count,
@@ -188,6 +192,10 @@ size_t hs_workspace_size(const hs_params* p, int32_t which) {
     if (which < HS_WS_FULL || which > HS_WS_DECODE_SPARSE) return (size_t)-1;
     if (resolve(p, decode, &kp) != HS_OK) return (size_t)-1;
     switch (which) {
+        case HS_WS_FULL:
+            return hs::full_tc_supported(kp, p->dtype) && hs::token_select_wide_applies(kp, p->dtype)
+                       ? hs::token_select_wide_workspace(kp)
+                       : 0;
         case HS_WS_DECODE_FULL: return hs::decode_full_workspace(kp);
         case HS_WS_DECODE_SPARSE: return hs::decode_sparse_workspace(kp);
         default: return 0;

@@ -82,6 +82,14 @@ cudaError_t launch_token_select_tc(const KParams& p, const void* q, const void* 
                                    const float* lse, int32_t* idx, int32_t* cnt, float* sel,
                                    cudaStream_t st);
 
+// Token-mode selection for long scans (>= 2^18 keys): 16 positions per work
+// item, N = 256, candidate buffers in the workspace (persistent grid).
+bool token_select_wide_applies(const KParams& p, int dtype);
+size_t token_select_wide_workspace(const KParams& p);
+cudaError_t launch_token_select_wide(const KParams& p, const void* q, const void* k,
+                                     const float* lse, int32_t* idx, int32_t* cnt, float* sel,
+                                     void* ws, size_t ws_bytes, cudaStream_t st);
+
 // Sparse decode step with its scratch in a file-scope device array.
 size_t noalloc_scratch_bytes();
 cudaError_t launch_decode_sparse_noalloc(const KParams& p, const void* q, const void* kc,

@@ -11,17 +11,28 @@
 //
 // with Q's rows position-major (one 4-D TMA box with the head and position
 // strides swapped), so a thread owns one key and holds all 16 heads of each
-// of its positions in registers: the group max is in-thread FFMA + FMNMX with
-// the fp32 lse.  Each position keeps an exact streaming top-(k-w) buffer in
-// shared memory (admission threshold = the k-w-th best key after each cut).
+// of its positions in registers: the group max is in-thread packed FMA plus
+// three-input max with the fp32 lse.  Each position keeps an exact streaming
+// top-(k-w) buffer in shared memory (admission threshold = a key at or below
+// the (k-w)-th best seen so far, raised by each cut of the buffer).
 //
-// Warps: 0 TMA (Q once, K tiles of 128 keys through a 2-stage ring), 1 TMEM +
-// MMA issuer (S^T in 4 TMEM buffers), 2..17 scorers in four sets of four (each
-// set covers the 128 TMEM lanes = keys, and 2 of the 8 positions).  The sets
-// only meet at the TMEM buffers, so one set's buffer cut does not stall the
-// others for up to 3 tiles.  The scorers' dependent chains (TMEM load, FMA,
-// max, ballot, shared atomics) are latency-bound, so the work is spread over
-// 16 warps with 2 positions per thread rather than 8 warps with 4.
+// What bounds it: per 128-key tile the tensor core reads its operands from
+// shared memory (K 32 KB + Q^T 32 KB over the 8 MMAs) while TMA writes the
+// next K tile (32 KB): 96 KB of shared-memory traffic per 512 MMA cycles,
+// and the K tiles stream from L2 (every CTA of a group scans the same keys).
+// So the K ring is as deep as shared memory allows next to the candidate
+// buffers (two instantiations: a 3-stage ring for long scans, a 2-stage ring
+// with larger buffers, hence fewer cuts, for shorter ones), and the scorers
+// keep a short fast path: a tile in which no key of the thread's four
+// positions reaches its threshold costs two TMEM loads, the packed group max
+// and one warp vote.
+//
+// Warps: 0 TMA (Q once, K tiles through the ring), 1 TMEM + MMA issuer (S^T
+// into 4 TMEM buffers), 2..9 scorers in two sets of four (a set covers the
+// 128 TMEM lanes = keys, and 4 of the 8 positions).  A set meets every second
+// tile at a named barrier; each of its warps then cuts its own position's
+// buffer if two more tiles could overflow it.  The sets only meet at the TMEM
+// buffers, so one set's cut does not stall the other for up to 3 tiles.
 #include "hs_common.cuh"
 #include "hs_kernels.cuh"
 #include "tc_ptx.cuh"
@@ -34,34 +45,49 @@ using namespace tc;
 constexpr int kG = 16;          // heads per group handled here
 constexpr int kPos = 8;         // positions per CTA
 constexpr int kKeys = 128;      // keys per K tile (= MMA M)
-constexpr int kPP = 2;          // positions per scorer thread
-constexpr int kSets = kPos / kPP;          // scorer sets of four warps
-constexpr int kScorers = 4 * kSets;        // scorer warps
 constexpr int kHd = 128;
-constexpr int kStages = 2;       // K ring (the MMA is far ahead of the scorers)
 constexpr int kSBufs = 4;        // S^T buffers in TMEM: the scorer sets may drift 3 tiles apart
-constexpr int kThreads = 64 + 32 * kScorers;
-constexpr int kMaxRanked = 1024;            // k - w handled here
-// Per-position buffer entries: the k - w kept, two tiles of admissions
-// between cut checks, and 5 tiles' worth of headroom (what shared memory holds).
-constexpr int kCap = kMaxRanked + 7 * kKeys;
+constexpr int kCheck = 2;        // tiles between a set's cut checks
 constexpr int kBitmapKeys = 65536;  // finalize by id bitmap (8 KB per position) below this
-// a cut at n > kCap - 2 kKeys must leave room for two more tiles
-static_assert((kCap - 2 * kKeys - kMaxRanked) / 2 >= 2 * kKeys, "cut headroom");
-
-constexpr uint32_t kQOff = 0;                         // 2 x 16 KB
-constexpr uint32_t kKOff = 32768;                     // kStages x 32 KB (sort scratch later)
-constexpr uint32_t kBufOff = kKOff + kStages * 32768; // kPos x kCap x 8
-constexpr uint32_t kHistOff = kBufOff + kPos * kCap * 8;   // kPos positions x 1 KB
-constexpr uint32_t kBarOff = kHistOff + 8 * 1024;
-enum { BQ = 0, BKF = 1, BKE = BKF + kStages, BSF = BKE + kStages, BSE = BSF + kSBufs,
-       BDRAIN = BSE + kSBufs, BCOUNT = BDRAIN + 1 };
-constexpr uint32_t kMiscOff = kBarOff + BCOUNT * 8;  // tmem(4) abort(4) cnt[8](32) thresh[8](64)
-constexpr uint32_t kSmemBytes = kMiscOff + 8 + 32 + 64 + 1024;
 constexpr uint32_t kTmemCols = 128 * kSBufs;
-static_assert(kStages * 32768 >= 8 * kMaxRanked * 8, "sort scratch fits in the K ring");
-static_assert(kStages * 32768 >= 8 * (kBitmapKeys / 8), "id bitmaps fit in the K ring");
-static_assert(kSmemBytes <= 232448, "shared memory");
+
+// Shared-memory map of an instantiation with a kStages-deep K ring,
+// candidate buffers of kCap entries per position and kPP positions per
+// scorer thread (sets of four warps, one per TMEM lane quadrant).
+template <int kStages, int kCap, int kPP_>
+struct Cfg {
+    static constexpr int kStagesN = kStages, kCapN = kCap, kPP = kPP_;
+    static constexpr int kSets = kPos / kPP;      // scorer sets of four warps
+    static constexpr int kScorers = 4 * kSets;    // scorer warps
+    static constexpr int kThreads = 64 + 32 * kScorers;
+    static_assert(kScorers >= kPos, "the finalize runs one scorer warp per position");
+    // largest k - w handled: an exact cut leaves k - w entries, which must
+    // leave room for the kCheck tiles of appends before the next check
+    static constexpr int kMaxRanked = kCap - (kCheck + 1) * kKeys < 1024
+                                          ? kCap - (kCheck + 1) * kKeys
+                                          : 1024;
+    static constexpr uint32_t kQOff = 0;                          // 2 x 16 KB
+    static constexpr uint32_t kKOff = 32768;                      // kStages x 32 KB (finalize scratch later)
+    static constexpr uint32_t kBufOff = kKOff + kStages * 32768;  // kPos x kCap x 8
+    static constexpr uint32_t kHistOff = kBufOff + kPos * kCap * 8;  // kPos x 1 KB
+    static constexpr uint32_t kBarOff = kHistOff + kPos * 1024;
+    enum { BQ = 0, BKF = 1, BKE = BKF + kStages, BSF = BKE + kStages, BSE = BSF + kSBufs,
+           BDRAIN = BSE + kSBufs, BCOUNT = BDRAIN + 1 };
+    // tmem slot (4) | abort (4) | count[kPos] (32) | threshold key[kPos] (64)
+    static constexpr uint32_t kMiscOff = kBarOff + BCOUNT * 8;
+    static constexpr uint32_t kSmemBytes = kMiscOff + 8 + 4 * kPos + 8 * kPos + 1024;
+    static_assert(kSmemBytes <= 232448, "shared memory");
+    static_assert(kStages * 32768 >= kPos * kMaxRanked * 8, "sort scratch fits in the K ring");
+    static_assert(kStages * 32768 >= kPos * (kBitmapKeys / 8), "id bitmaps fit in the K ring");
+    static_assert(kMaxRanked >= kKeys, "buffers hold at least one cut's worth");
+};
+
+// long scans: deeper ring; shorter scans: larger buffers (fewer cuts)
+#ifndef TSEL_PP
+#define TSEL_PP 4
+#endif
+using CfgLong = Cfg<3, 1408, TSEL_PP>;
+using CfgShort = Cfg<2, 1920, TSEL_PP>;
 
 struct Args {
     KParams p;
@@ -79,9 +105,27 @@ __device__ __forceinline__ void drain(uint32_t bar, uint32_t parity) {
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+// max over 16 heads of a2 - lse2 for one key and position: raw logits r[0..16)
+// (TMEM words), scale sl2, -lse2 of the heads in nl[0..16).
+__device__ __forceinline__ float group_max16(const uint32_t* r, float sl2, const float* nl) {
+    float v[kG];
+#pragma unroll
+    for (int hh = 0; hh < kG; hh += 2) {
+        const float2 r2 = ffma2(make_float2(__uint_as_float(r[hh]), __uint_as_float(r[hh + 1])),
+                                make_float2(sl2, sl2), make_float2(nl[hh], nl[hh + 1]));
+        v[hh] = r2.x;
+        v[hh + 1] = r2.y;
+    }
+    return fmaxf(max3f(max3f(v[0], v[1], v[2]), max3f(v[3], v[4], v[5]), max3f(v[6], v[7], v[8])),
+                 max3f(max3f(v[9], v[10], v[11]), max3f(v[12], v[13], v[14]), v[15]));
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::kThreads, 1)
     token_select_kernel(const __grid_constant__ CUtensorMap tmap_q,
                         const __grid_constant__ CUtensorMap tmap_k, Args a) {
+    constexpr int kStages = C::kStagesN, kCap = C::kCapN, kPP = C::kPP;
+    constexpr int kSets = C::kSets, kScorers = C::kScorers;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -99,23 +143,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nt = min((p.t_kv + kKeys - 1) / kKeys, pos_max / kKeys + 1);
     const int Kc = p.k - p.window;
 
-    auto bar = [&](int i) { return base + kBarOff + 8u * i; };
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gb + kMiscOff);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + kMiscOff + 4);
-    int* s_cnt = reinterpret_cast<int*>(gb + kMiscOff + 8);
-    unsigned long long* s_th = reinterpret_cast<unsigned long long*>(gb + kMiscOff + 40);
+    auto bar = [&](int i) { return base + C::kBarOff + 8u * i; };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gb + C::kMiscOff);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + C::kMiscOff + 4);
+    int* s_cnt = reinterpret_cast<int*>(gb + C::kMiscOff + 8);
+    unsigned long long* s_th = reinterpret_cast<unsigned long long*>(gb + C::kMiscOff + 8 + 4 * kPos);
 
     if (threadIdx.x == 0) {
-        mbar_init(bar(BQ), 1);
-        for (int i = 0; i < kStages; ++i) { mbar_init(bar(BKF + i), 1); mbar_init(bar(BKE + i), 1); }
-        for (int i = 0; i < kSBufs; ++i) { mbar_init(bar(BSF + i), 1); mbar_init(bar(BSE + i), kScorers); }
-        mbar_init(bar(BDRAIN), 1);
+        mbar_init(bar(C::BQ), 1);
+        for (int i = 0; i < kStages; ++i) { mbar_init(bar(C::BKF + i), 1); mbar_init(bar(C::BKE + i), 1); }
+        for (int i = 0; i < kSBufs; ++i) { mbar_init(bar(C::BSF + i), 1); mbar_init(bar(C::BSE + i), kScorers); }
+        mbar_init(bar(C::BDRAIN), 1);
         *abort_flag = 0;
         for (int i = 0; i < kPos; ++i) { s_cnt[i] = 0; s_th[i] = 0ull; }
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(base + kMiscOff, kTmemCols);
+        tmem_alloc(base + C::kMiscOff, kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -127,47 +171,55 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             prefetch_tmap(&tmap_q);
             prefetch_tmap(&tmap_k);
-            mbar_arrive_expect_tx(bar(BQ), 32768);
-            tma_load_4d(base + kQOff, &tmap_q, bar(BQ), 0, u * kG, row0, b);
-            tma_load_4d(base + kQOff + 16384, &tmap_q, bar(BQ), 64, u * kG, row0, b);
+            mbar_arrive_expect_tx(bar(C::BQ), 32768);
+            tma_load_4d(base + C::kQOff, &tmap_q, bar(C::BQ), 0, u * kG, row0, b);
+            tma_load_4d(base + C::kQOff + 16384, &tmap_q, bar(C::BQ), 64, u * kG, row0, b);
             int issued = 0;
             for (int j = 0; j < nt; ++j) {
                 const int st = j % kStages;
-                if (j >= kStages && !mbar_wait(bar(BKE + st), ((j / kStages) - 1) & 1, abort_flag)) break;
-                const uint32_t f = bar(BKF + st);
+                if (j >= kStages &&
+                    !mbar_wait(bar(C::BKE + st), ((j / kStages) - 1) & 1, abort_flag, false))
+                    break;
+                const uint32_t f = bar(C::BKF + st);
                 mbar_arrive_expect_tx(f, 32768);
-                const uint32_t kd = base + kKOff + st * 32768;
+                const uint32_t kd = base + C::kKOff + st * 32768;
                 tma_load_3d(kd, &tmap_k, f, 0, j * kKeys, bu);
                 tma_load_3d(kd + 16384, &tmap_k, f, 64, j * kKeys, bu);
                 issued = j + 1;
             }
-            drain(bar(BQ), 0);
+            drain(bar(C::BQ), 0);
             for (int j = max(0, issued - kStages); j < issued; ++j)
-                drain(bar(BKF + j % kStages), (j / kStages) & 1);
+                drain(bar(C::BKF + j % kStages), (j / kStages) & 1);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t id = idesc_bf16(kKeys, kPos * kG, false, false);
-            bool ok = mbar_wait(bar(BQ), 0, abort_flag);
+            // descriptors built once; an operand `off` bytes further is the
+            // descriptor plus off >> 4 (every operand lies below 256 KB)
+            const uint64_t dk0 = sw128_desc(base + C::kKOff, 16, 1024);
+            const uint64_t dq = sw128_desc(base + C::kQOff, 16, 1024);
+            bool ok = mbar_wait(bar(C::BQ), 0, abort_flag, false);
             tc_fence_after();
             for (int j = 0; ok && j < nt; ++j) {
                 const int st = j % kStages, s = j % kSBufs;
-                if (!mbar_wait(bar(BKF + st), (j / kStages) & 1, abort_flag)) break;
-                if (j >= kSBufs && !mbar_wait(bar(BSE + s), ((j / kSBufs) - 1) & 1, abort_flag))
+                if (!mbar_wait(bar(C::BKF + st), (j / kStages) & 1, abort_flag, false)) break;
+                if (j >= kSBufs &&
+                    !mbar_wait(bar(C::BSE + s), ((j / kSBufs) - 1) & 1, abort_flag, false))
                     break;
                 tc_fence_after();
-                const uint32_t kb = base + kKOff + st * 32768;
+                const uint64_t dk = dk0 + (uint64_t)(st * (32768 >> 4));
+                // K step kk: d columns 16kk.. = 32-byte column group kk&3 of d half kk>>2
 #pragma unroll
                 for (int kk = 0; kk < kHd / 16; ++kk) {
-                    const uint64_t ad = sw128_desc(kb + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                    const uint64_t bd = sw128_desc(base + kQOff + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                    umma_ss(tmem + 128 * s, ad, bd, id, kk > 0 ? 1u : 0u);
+                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    umma_ss(tmem + 128 * s, dk + (uint64_t)(off >> 4), dq + (uint64_t)(off >> 4),
+                            id, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(bar(BSF + s));
-                umma_commit(bar(BKE + st));
+                umma_commit(bar(C::BSF + s));
+                umma_commit(bar(C::BKE + st));
             }
-            umma_commit(bar(BDRAIN));
-            drain(bar(BDRAIN), 0);
+            umma_commit(bar(C::BDRAIN));
+            drain(bar(C::BDRAIN), 0);
         }
     } else {
         // ------------------------------------------------------------ scorers
@@ -176,9 +228,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int wid = warp - 2;         // 0 .. kScorers-1
         const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16) + set * (kPP * kG);
         const float sl2 = p.scale_log2;
-        // this thread's kPP positions: lse (log2 domain) of their 16 heads
-        float nlse2[kPP][kG];  // -lse2
-        int tpos[kPP];
+        // this thread's kPP positions: -lse2 of their 16 heads, the last key
+        // each may rank (t - w; -1 when it ranks nothing), and thresholds
+        float nlse2[kPP][kG];
+        int tpos[kPP], lim[kPP];
         bool live[kPP], all_sel[kPP];
 #pragma unroll
         for (int i = 0; i < kPP; ++i) {
@@ -186,127 +239,102 @@ __global__ void __launch_bounds__(kThreads, 1)
             live[i] = r < p.t_q;
             tpos[i] = p.q_offset + r;
             all_sel[i] = tpos[i] + 1 <= p.k;
+            lim[i] = (live[i] && !all_sel[i] && Kc > 0) ? tpos[i] - p.window : -1;
 #pragma unroll
             for (int hh = 0; hh < kG; ++hh)
                 nlse2[i][hh] = live[i] ? -a.lse[((size_t)b * p.hq + u * kG + hh) * p.t_q + r] * kLog2e
                                        : 0.f;
         }
-        uint64_t* bufs = reinterpret_cast<uint64_t*>(gb + kBufOff);
-        // scratch of the position this warp cuts (quads 0..kPP-1 of a set cut)
-        uint32_t* hist = reinterpret_cast<uint32_t*>(
-            gb + kHistOff + (set * kPP + (quad < kPP ? quad : 0)) * 1024);
+        uint64_t* bufs = reinterpret_cast<uint64_t*>(gb + C::kBufOff);
+        // the position this warp cuts (quads 0..kPP-1 of a set cut)
+        const bool cutter = quad < kPP;
+        const int my_pos = set * kPP + (cutter ? quad : 0);
+        uint32_t* hist = reinterpret_cast<uint32_t*>(gb + C::kHistOff + my_pos * 1024);
         const int bar_id = 1 + set;
         // Admission compares a key's float score with the float score of the
-        // position's threshold key (thf, in registers): score >= thf admits
-        // every key that beats the 64-bit threshold (and at most the few that
-        // tie its score), and admitting more than necessary is always safe --
-        // the cuts and the finalize select exactly.  Bulk tiles (the thread's
-        // positions live, none selecting everything, no scores to write, the
-        // tile entirely below the first position's window, hence below every
-        // window of the set and visible to all) need nothing else.
-        bool bulk_ok = Kc > 0 && a.sel == nullptr;
-#pragma unroll
-        for (int i = 0; i < kPP; ++i) bulk_ok = bulk_ok && live[i] && !all_sel[i];
-        const int lo_first = tpos[0] - p.window + 1;
+        // position's threshold key (thf): score >= thf admits every key that
+        // beats the 64-bit threshold (and at most the few tying its score);
+        // admitting more than necessary is always safe -- the cuts and the
+        // finalize select exactly.
         float thf[kPP];
 #pragma unroll
         for (int i = 0; i < kPP; ++i) thf[i] = -INFINITY;
+        const uint32_t lt_mask = (1u << lane) - 1u;
         bool ok = true;
         // Every warp runs every iteration (the set meets at named barriers);
         // after an abort the waits fail at once and the work is skipped.
         for (int j = 0; j < nt; ++j) {
             const int s = j % kSBufs;
-            bool got = ok && mbar_wait(bar(BSF + s), (j / kSBufs) & 1, abort_flag);
+            bool got = ok && mbar_wait(bar(C::BSF + s), (j / kSBufs) & 1, abort_flag);
             got = __all_sync(0xffffffffu, got);
             if (!got) ok = false;
             if (got) {
-            tc_fence_after();
-            uint32_t r0[32];
-            tmem_ld32(tq + 128 * s, r0);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(BSE + s));
-            const int key = j * kKeys + quad * 32 + lane;
-            const bool bulk = bulk_ok && (j + 1) * kKeys <= lo_first;  // warp-uniform
-            float sc[kPP];
-            uint32_t bal[kPP];
+                tc_fence_after();
+                uint32_t r[kPP * kG];
 #pragma unroll
-            for (int i = 0; i < kPP; ++i) {
-                const uint32_t* rr = r0;
-                const int c0 = i * kG;
-                // a2 - lse2 of the 16 heads (packed FMA), then their max (3-input max)
-                float v[kG];
+                for (int c = 0; c < kPP * kG; c += 32)
+                    tmem_ld32(tq + 128 * s + c, *reinterpret_cast<uint32_t(*)[32]>(&r[c]));
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(C::BSE + s));
+                const int key = j * kKeys + quad * 32 + lane;
+                float sc[kPP];
+                bool any = false;
 #pragma unroll
-                for (int hh = 0; hh < kG; hh += 2) {
-                    const float2 r2 = ffma2(make_float2(__uint_as_float(rr[c0 + hh]),
-                                                        __uint_as_float(rr[c0 + hh + 1])),
-                                            make_float2(sl2, sl2),
-                                            make_float2(nlse2[i][hh], nlse2[i][hh + 1]));
-                    v[hh] = r2.x;
-                    v[hh + 1] = r2.y;
+                for (int i = 0; i < kPP; ++i) {
+                    sc[i] = group_max16(&r[i * kG], sl2, nlse2[i]);
+                    any |= (sc[i] >= thf[i]) & (key <= lim[i]);
                 }
-                sc[i] = fmaxf(max3f(max3f(v[0], v[1], v[2]), max3f(v[3], v[4], v[5]),
-                                    max3f(v[6], v[7], v[8])),
-                              max3f(max3f(v[9], v[10], v[11]), max3f(v[12], v[13], v[14]), v[15]));
-                if (bulk) {
-                    bal[i] = __ballot_sync(0xffffffffu, sc[i] >= thf[i]);
-                    continue;
-                }
-                const int t = tpos[i];
-                const bool visible = live[i] && key <= t;
-                const int pos = set * kPP + i;
-                const size_t orow = ((size_t)b * p.hkv + u) * p.t_q + row0 + pos;
-                float* srow = a.sel ? a.sel + orow * p.ksel : nullptr;
-                // Every lane reaches the ballot below: no per-lane early exit.
-                const int lo = t - p.window + 1;
-                bool cand = false;
-                if (all_sel[i]) {
-                    if (visible && srow) srow[key] = exp2f(sc[i]);
-                } else if (visible && key >= lo) {
-                    if (srow) srow[Kc + (key - lo)] = exp2f(sc[i]);
-                } else {
-                    cand = visible && Kc > 0 && key < lo && sc[i] >= thf[i];
-                }
-                bal[i] = __ballot_sync(0xffffffffu, cand);
-            }
-            // lanes 0..kPP-1 reserve the slots of the thread's positions at once
-            uint32_t my_bal = bal[0];
+                if (__any_sync(0xffffffffu, any)) {
+                    // appends: per position, one slot reservation for the warp
 #pragma unroll
-            for (int i = 1; i < kPP; ++i) my_bal = lane == i ? bal[i] : my_bal;
-            int my_base = 0;
-            if (lane < kPP && my_bal != 0u) my_base = atomicAdd(&s_cnt[set * kPP + lane], __popc(my_bal));
-#pragma unroll
-            for (int i = 0; i < kPP; ++i) {
-                if (!bal[i]) continue;  // warp-uniform
-                const int bi = __shfl_sync(0xffffffffu, my_base, i);
-                if ((bal[i] >> lane) & 1u)
-                    bufs[(size_t)(set * kPP + i) * kCap + bi + __popc(bal[i] & ((1u << lane) - 1))] =
-                        sel_key(sc[i], (uint32_t)key);
-            }
-            }  // got
-            // Every second tile the set meets to cut the buffers that could
-            // overflow within the next two tiles (a tile appends at most kKeys
-            // keys per position; a cut frees at least kCutFree slots or leaves
-            // Kc), then refreshes its thresholds.
-            if (j & 1) {
-                asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
-                if (ok && quad < kPP) {
-                    const int pos = set * kPP + quad;
-                    const int n = s_cnt[pos];
-                    if (n > kCap - 2 * kKeys) {
-                        uint64_t th;
-                        const int m = warp_cut_sampled(bufs + (size_t)pos * kCap, n, Kc,
-                                                       (kCap - 2 * kKeys - Kc) / 2, hist, &th);
-                        if (lane == 0) {
-                            s_th[pos] = th > s_th[pos] ? th : s_th[pos];
-                            s_cnt[pos] = m;
+                    for (int i = 0; i < kPP; ++i) {
+                        const bool cand = (sc[i] >= thf[i]) & (key <= lim[i]);
+                        const uint32_t bal = __ballot_sync(0xffffffffu, cand);
+                        if (bal == 0u) continue;  // warp-uniform
+                        const int pos = set * kPP + i;
+                        int at = 0;
+                        if (lane == 0) at = atomicAdd(&s_cnt[pos], __popc(bal));
+                        at = __shfl_sync(0xffffffffu, at, 0) + __popc(bal & lt_mask);
+                        if (cand) {
+                            if (at < kCap) bufs[(size_t)pos * kCap + at] = sel_key(sc[i], (uint32_t)key);
+                            else set_status(HS_ERR_BOUNDS);  // not reached: the cuts keep room
                         }
                     }
                 }
+                if (a.sel) {
+                    // scores of the keys selected without ranking (tests ask for them)
+#pragma unroll
+                    for (int i = 0; i < kPP; ++i) {
+                        const int t = tpos[i];
+                        if (!live[i] || key > t) continue;
+                        float* srow = a.sel + (((size_t)b * p.hkv + u) * p.t_q + row0 + set * kPP + i) * p.ksel;
+                        if (all_sel[i]) srow[key] = exp2f(sc[i]);
+                        else if (key >= t - p.window + 1) srow[Kc + (key - (t - p.window + 1))] = exp2f(sc[i]);
+                    }
+                }
+            }  // got
+            // Every kCheck-th tile the set meets to cut the buffers that could
+            // overflow within the next kCheck tiles (a tile appends at most
+            // kKeys keys per position), then refreshes its thresholds.
+            if (j % kCheck == kCheck - 1) {
                 asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
-                // a cut may have raised the thresholds: refresh their float scores
-                // (-inf while nothing was cut, and never NaN)
+                const int n = s_cnt[my_pos];
+                if (ok && cutter && n > kCap - kCheck * kKeys) {
+                    // keep at most halfway between k - w and the trigger
+                    const int target = Kc + (kCap - kCheck * kKeys - Kc) / 2;
+                    uint64_t th;
+                    const int m = warp_cut_sampled(bufs + (size_t)my_pos * kCap, n, Kc, n - target,
+                                                   hist, &th);
+                    if (lane == 0) {
+                        s_th[my_pos] = th > s_th[my_pos] ? th : s_th[my_pos];
+                        s_cnt[my_pos] = m;
+                    }
+                }
+                asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
+                // a cut may have raised the thresholds: refresh their float
+                // scores (-inf while nothing was cut, and never NaN)
 #pragma unroll
                 for (int i = 0; i < kPP; ++i) {
                     const uint64_t th = s_th[set * kPP + i];
@@ -330,14 +358,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int x = lane; x < n_out; x += 32) irow[x] = x;
             } else {
                 uint64_t* buf = bufs + (size_t)pos * kCap;
-                int n = Kc > 0 ? s_cnt[pos] : 0;
-                uint32_t* fhist = reinterpret_cast<uint32_t*>(gb + kHistOff + pos * 1024);
+                int n = Kc > 0 ? min(s_cnt[pos], kCap) : 0;
+                uint32_t* fhist = reinterpret_cast<uint32_t*>(gb + C::kHistOff + pos * 1024);
                 if (n > Kc) { warp_cut_to_k(buf, n, Kc, fhist); n = Kc; }
                 __syncwarp();
                 if (!srow && t < kBitmapKeys) {
                     // ascending ids without sorting: mark the winners in a bitmap
                     // over 0..t, then read the set bits out in word order
-                    uint32_t* bm = reinterpret_cast<uint32_t*>(gb + kKOff) + (size_t)wid * (kBitmapKeys / 32);
+                    uint32_t* bm = reinterpret_cast<uint32_t*>(gb + C::kKOff) + (size_t)wid * (kBitmapKeys / 32);
                     const int words = (t >> 5) + 1;
                     const int per = (words + 31) >> 5;  // words per lane, consecutive
                     for (int x = lane; x < per * 32; x += 32) bm[x] = 0u;
@@ -367,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 } else {
                     const int sort_n = next_pow2(Kc > 0 ? Kc : 1);
-                    uint64_t* sb = reinterpret_cast<uint64_t*>(gb + kKOff) + (size_t)wid * kMaxRanked;
+                    uint64_t* sb = reinterpret_cast<uint64_t*>(gb + C::kKOff) + (size_t)wid * C::kMaxRanked;
                     for (int x = lane; x < sort_n; x += 32)
                         sb[x] = x < n ? (((uint64_t)sel_key_id(buf[x]) << 32) | (buf[x] >> 32)) : ~0ull;
                     __syncwarp();
@@ -398,11 +426,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// Key tiles one CTA scans for the latest of its positions, and the scan
+// length from which the deeper K ring pays off over fewer buffer cuts.
+constexpr int kLongScanTiles = 2048;  // 262144 keys
+
 }  // namespace tsel
 
 bool token_select_tc_supported(const KParams& p, int dtype) {
     return dtype == HS_BF16 && p.head_dim == 128 && p.mode == 1 && p.group == tsel::kG &&
-           p.k - p.window <= tsel::kMaxRanked;
+           p.k - p.window <= tsel::CfgShort::kMaxRanked;
+}
+
+template <class C>
+static cudaError_t launch_tsel(const CUtensorMap& mq, const CUtensorMap& mk, const tsel::Args& a,
+                               long long grid, cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(tsel::token_select_kernel<C>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    tsel::token_select_kernel<C><<<(unsigned)grid, C::kThreads, C::kSmemBytes, st>>>(mq, mk, a);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_token_select_tc(const KParams& p, const void* q, const void* k,
@@ -428,12 +471,12 @@ cudaError_t launch_token_select_tc(const KParams& p, const void* q, const void* 
     a.cnt = cnt;
     a.sel = sel;
     a.n_ptiles = (p.t_q + kPos - 1) / kPos;
-    cudaError_t e = cudaFuncSetAttribute(
-        token_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, tsel::kSmemBytes);
-    if (e != cudaSuccess) return e;
     const long long grid = (long long)a.n_ptiles * p.batch * p.hkv;
-    token_select_kernel<<<(unsigned)grid, tsel::kThreads, tsel::kSmemBytes, st>>>(mq, mk, a);
-    return cudaGetLastError();
+    const long long scan = ((long long)p.q_offset + p.t_q + kKeys - 1) / kKeys;
+    // the deeper ring's smaller buffers need headroom above k - w for their cuts
+    if (scan >= kLongScanTiles && p.k - p.window <= CfgLong::kCapN - 4 * kKeys)
+        return launch_tsel<CfgLong>(mq, mk, a, grid, st);
+    return launch_tsel<CfgShort>(mq, mk, a, grid, st);
 }
 
 }  // namespace hs

@@ -46,7 +46,8 @@ def run_full(w, gen_device="cpu", rows=None, check_scores=True):
     q, k, v = _cuda(q, k, v)
     p = P.abi_params(w)
     o, lse, idx, cnt, sel = hs.full_outputs(p, with_scores=True)
-    hs.hs_full_attn_index(p, q, k, v, o, lse, idx, cnt, sel)
+    ws = hs.workspace(p, hs.HS_WS_FULL)
+    hs.hs_full_attn_index(p, q, k, v, o, lse, idx, cnt, sel, ws)
     torch.cuda.synchronize()
     assert hs.hs_device_status() == 0
     rws = P.all_rows(w) if rows is None else rows
@@ -59,6 +60,26 @@ def run_full(w, gen_device="cpu", rows=None, check_scores=True):
     g_idx = P.gpu_rows(idx.cpu().numpy(), rws, False)
     g_cnt = P.gpu_rows(cnt.cpu().numpy(), rws, False)
     P.check_index(g_idx, g_cnt, orc, w.mode, w.window, w.k, f"{w.name} index")
+    if w.mode == "token":
+        # Without score output the selectors take their other finalize paths
+        # (id bitmap): same kernel, same arithmetic, so identical index sets.
+        # Without the workspace a long scan takes the shared-memory selector
+        # instead of the wide one, whose scores round differently (the wide
+        # one folds lse into the contraction): that set must pass the oracle
+        # check on its own.
+        for wsx in ([ws, None] if ws is not None else [None]):
+            idx2, cnt2 = torch.full_like(idx, -7), torch.full_like(cnt, -7)
+            hs.hs_full_attn_index(p, q, k, v, torch.empty_like(o), torch.empty_like(lse), idx2,
+                                  cnt2, None, wsx)
+            torch.cuda.synchronize()
+            assert hs.hs_device_status() == 0
+            if wsx is ws:
+                assert torch.equal(idx2, idx) and torch.equal(cnt2, cnt), \
+                    f"{w.name}: index without scores"
+            else:
+                P.check_index(P.gpu_rows(idx2.cpu().numpy(), rws, False),
+                              P.gpu_rows(cnt2.cpu().numpy(), rws, False), orc, w.mode, w.window,
+                              w.k, f"{w.name} index without workspace")
     if check_scores:
         g_sel = P.gpu_rows(sel.cpu().double().numpy(), rws, False)
         for n in range(len(g_cnt)):
@@ -119,6 +140,10 @@ SMALL = {
                                    hq=4, hkv=1, t=150, k=24, window=24),
     "bf16_token_chunk": wl.scaled(wl.WORKLOADS["long_1m_chunk"], name="bf16_token_chunk",
                                   hq=16, hkv=1, t=1500, t_q=300, q_offset=1200, k=256, window=32),
+    # a scan of >= 2048 key tiles: the selector's deep-ring instantiation
+    "bf16_token_long_scan": wl.scaled(wl.WORKLOADS["long_1m_chunk"], name="bf16_token_long_scan",
+                                      hq=16, hkv=1, t=266240, t_q=40, q_offset=266200, k=1024,
+                                      window=128, needles="loguniform:16"),
     "bf16_select_all": wl.scaled(wl.WORKLOADS["hysparse2_prefill"], name="bf16_select_all",
                                  hq=4, hkv=2, t=100, k=128, window=16),
     "bf16_single_token": wl.scaled(wl.WORKLOADS["hysparse2_prefill"], name="bf16_single_token",

@@ -7,7 +7,14 @@
 // warpgroups with one thread per row, and one thread per Q tile (warp 1 for
 // tile 0, warp 10 for tile 1) issues that tile's MMAs:
 //   S = Q K^T  (M = 128, N = 64, K = 16 x 8) into one of two TMEM buffers,
-//   O += P V   (N = 128, V as the MN-major operand; P from shared memory).
+//   O += P V   (N = 128, V as the MN-major operand; P from TMEM).
+// The softmax writes P (bf16 pairs) back over the first 32 columns of the S
+// buffer it read, and the PV MMA takes its A operand from there: P never
+// touches shared memory, whose bandwidth the operand reads of the S MMAs
+// (Q 4 KB + K 2 KB per 32-cycle MMA) and the TMA writes already saturate.
+// An S buffer needs no release of its own: the MMAs of one issuer execute in
+// issue order, so S of tile j + 2 (same buffer) follows PV of tile j, which
+// waited for that tile's P.
 // The kernels differ in which key tiles they visit, which keys a row keeps,
 // and what they do besides attention (block-score capture, union building).
 #pragma once
@@ -155,7 +162,6 @@ __device__ __forceinline__ void mma_issuer(uint32_t base, uint32_t tmem, int q, 
     const uint32_t id_o = idesc_bf16(L::kBM, L::kD, false, true);
     const uint64_t dq = sw128_desc(base + L::kQOff + q * 32768, 16, 1024);
     const uint64_t dk0 = sw128_desc(base + L::kKOff, 16, 1024);
-    const uint64_t dp0 = sw128_desc(base + L::kPOff + q * 32768, 16, 1024);
     const uint64_t dv0 = sw128_desc(base + L::kVOff, 8192, 1024);  // V: MN-major, d halves 8 KB apart
     const uint32_t ts = tmem + q * 256, to = tmem + q * 256 + 128;
     bool ok = mbar_wait(bar(L::BQ), 0, abort, false);
@@ -165,7 +171,6 @@ __device__ __forceinline__ void mma_issuer(uint32_t base, uint32_t tmem, int q, 
             const int st = j % L::kKS, s = j & 1;
             if (!mbar_wait(bar(L::BKF + st), (j / L::kKS) & 1, abort, false)) break;
             if (j < ntq) {
-                if (j >= 2 && !mbar_wait(bar(L::BSE + 2 * q + s), ((j >> 1) - 1) & 1, abort, false)) break;
                 tc_fence_after();
                 const uint64_t dk = dk0 + (uint64_t)(st * (16384 >> 4));
                 // K step kk: d columns 16kk.. = 32-byte column group kk&3 of d half kk>>2
@@ -184,13 +189,14 @@ __device__ __forceinline__ void mma_issuer(uint32_t base, uint32_t tmem, int q, 
             if (jj < ntq) {
                 if (!mbar_wait(bar(L::BPF + 2 * q + sp), (jj >> 1) & 1, abort, false)) break;
                 tc_fence_after();
-                const uint64_t dp = dp0 + (uint64_t)(sp * (16384 >> 4));
+                const uint32_t tp = ts + 64 * sp;  // P: columns 0..31 of S buffer sp
                 const uint64_t dv = dv0 + (uint64_t)(stp * (16384 >> 4));
-                // K step kk: keys 16kk.. = P column group kk, V rows 16kk..
+                // K step kk: keys 16kk.. = P columns 8kk.. (two keys per column),
+                // V rows 16kk..
 #pragma unroll
                 for (int kk = 0; kk < L::kBN / 16; ++kk)
-                    umma_ss(to, dp + (uint64_t)((kk * 32) >> 4), dv + (uint64_t)((kk * 2048) >> 4),
-                            id_o, (jj > 0 || kk > 0) ? 1u : 0u);
+                    umma_ts(to, tp + 8 * kk, dv + (uint64_t)((kk * 2048) >> 4), id_o,
+                            (jj > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(bar(L::BPVD + 2 * q + sp));
             }
             umma_commit(bar(L::BVE + stp));
@@ -265,6 +271,91 @@ __device__ __forceinline__ bool softmax_tile(const uint32_t (&r)[64], int first,
 #pragma unroll
     for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(e[2 * c], e[2 * c + 1]);
     return resc;
+}
+
+// The same tile without the tile maximum, for callers that do not need it
+// (no block-score capture): p = 2^(x*scale_log2 - m_ref) against the current
+// reference directly.  The reference lags by design, so p may exceed 1; when
+// the tile's sum stays below 2^8 every p of the tile is below 2^8 (the lazy
+// rescale's own bound) and nothing else is needed.  Otherwise (a logit far
+// above the reference, or inf/nan from one far enough above it) the tile
+// takes its maximum, rescales l (and asks the caller to rescale O) and
+// recomputes.  The first tile of a row (m_ref = -inf) starts from its
+// maximum; it must keep at least one key (key 0 is in every row's first tile
+// of the full layer).  Saves the 31 three-input max instructions of the
+// maximum on all but the rare tiles that move the reference.
+template <int kPolyEvery = 0>
+__device__ __forceinline__ void exp_tile(const float (&x)[64], float sl2, float m_ref,
+                                         float (&e)[64], float& sum) {
+    const float2 s2 = make_float2(sl2, sl2), n2 = make_float2(-m_ref, -m_ref);
+    float2 acc[8];
+#pragma unroll
+    for (int c2 = 0; c2 < 32; ++c2) {
+        const float2 y = ffma2(make_float2(x[2 * c2], x[2 * c2 + 1]), s2, n2);
+        if (kPolyEvery > 0 && c2 % (kPolyEvery > 0 ? kPolyEvery : 1) == kPolyEvery - 1) {
+            const float2 ev = exp2_poly2(y);
+            e[2 * c2] = ev.x;
+            e[2 * c2 + 1] = ev.y;
+        } else {
+            e[2 * c2] = ex2(y.x);
+            e[2 * c2 + 1] = ex2(y.y);
+        }
+        const float2 ev = make_float2(e[2 * c2], e[2 * c2 + 1]);
+        acc[c2 & 7] = c2 < 8 ? ev : fadd2(acc[c2 & 7], ev);
+    }
+#pragma unroll
+    for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+        for (int c = 0; c < w; ++c) acc[c] = fadd2(acc[c], acc[c + w]);
+    sum = acc[0].x + acc[0].y;
+}
+
+__device__ __forceinline__ float tile_max64(const float (&x)[64]) {
+    float m3[22];
+#pragma unroll
+    for (int c = 0; c < 21; ++c) m3[c] = max3f(x[3 * c], x[3 * c + 1], x[3 * c + 2]);
+    m3[21] = x[63];
+#pragma unroll
+    for (int c = 0; c < 7; ++c) m3[c] = max3f(m3[3 * c], m3[3 * c + 1], m3[3 * c + 2]);
+    return max3f(max3f(m3[0], m3[1], m3[2]), max3f(m3[3], m3[4], m3[5]), fmaxf(m3[6], m3[21]));
+}
+
+template <int kPolyEvery = 0>
+__device__ __forceinline__ bool softmax_tile_lazy(const uint32_t (&r)[64], int lim, float sl2,
+                                                  float& m_ref, float& l, float& corr,
+                                                  uint32_t (&pk)[32]) {
+    float x[64];
+#pragma unroll
+    for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(r[c]);
+    if (lim < 63) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) x[c] = c <= lim ? x[c] : -INFINITY;
+    }
+    corr = 1.f;
+    bool resc = false;
+    if (m_ref == -INFINITY) m_ref = tile_max64(x) * sl2;  // first tile: O is still empty
+    float e[64], lt;
+    exp_tile<kPolyEvery>(x, sl2, m_ref, e, lt);
+    if (!(lt < 256.f)) {
+        const float mt = tile_max64(x) * sl2;  // > m_ref + 2: some p >= 4
+        corr = ex2(m_ref - mt);
+        resc = true;
+        m_ref = mt;
+        l *= corr;
+        exp_tile<kPolyEvery>(x, sl2, m_ref, e, lt);
+    }
+    l += lt;
+#pragma unroll
+    for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(e[2 * c], e[2 * c + 1]);
+    return resc;
+}
+
+// P row (64 keys as 32 bf16 pairs) over the first 32 columns of the TMEM S
+// buffer at trow_s (every lane of the warp calls this; the caller then
+// fences and signals the MMA issuer).
+__device__ __forceinline__ void store_p_tmem(uint32_t trow_s, const uint32_t (&pk)[32]) {
+    tmem_st32(trow_s, pk);
+    tmem_wait_st();
 }
 
 // P row (64 keys, bf16) into the 128B-swizzled P buffer, made visible to the

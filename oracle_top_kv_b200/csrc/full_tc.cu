@@ -23,13 +23,15 @@
 //                rings of 3 stages each)
 //   warp 1       TMEM owner and MMA issuer of Q tile 0; warp 10 issues for
 //                Q tile 1: S = Q K^T into one of two TMEM buffers, then
-//                O += P V (P from shared memory, V MN-major).  One issuing
+//                O += P V (P from TMEM, V MN-major).  One issuing
 //                thread per tile: a single thread cannot issue the MMAs of
 //                both tiles as fast as the tensor core runs them.
 //   warps 2..9   two softmax warpgroups, one thread per row (TMEM lane):
 //                online softmax with lazy rescaling of O (only when the max
-//                grows by > 2^8), a third of the exponentials on the FMA
-//                pipe, P to shared memory, block-score capture, epilogue.
+//                grows by > 2^8), P back into TMEM, epilogue.  Block mode
+//                takes every tile's maximum (the block score, captured into
+//                the row's list) and runs a third of the exponentials on the
+//                FMA pipe; token mode needs no maximum (lazy softmax).
 // All waits are bounded (tc_ptx.cuh); a timeout aborts the CTA cleanly.
 #include "flash_tc.cuh"
 #include "hs_common.cuh"
@@ -81,6 +83,12 @@ __device__ __forceinline__ int tiles_for(const KParams& p, int first_row, int P)
     return min((p.t_kv + kBN - 1) / kBN, (p.q_offset + last_row) / kBN + 1);
 }
 
+// kCapture: block-mode index (needs every tile's maximum); otherwise o and lse
+// only, with the lazy softmax that skips the tile maximum and runs every
+// exponential on the MUFU unit (measured: offloading a share to the FMA pipe,
+// which the block path needs, no longer pays once the maximum is gone).
+constexpr int kLazyPolyEvery = 0;
+template <bool kCapture>
 __global__ void __launch_bounds__(kThreads, 1)
     full_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                    const __grid_constant__ CUtensorMap tmap_k,
@@ -158,21 +166,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld32(trow + 64 * s, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
             tmem_ld32(trow + 64 * s + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
             tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(L::BSE + 2 * q + s));
 
             // causal: keys <= pos (only the diagonal tile masks anything).  Key 0
             // is in every row's first tile, so every row keeps a key and a third
             // of the exponentials can run on the FMA pipe.
-            float mt, corr;
+            float corr;
             uint32_t pk[32];
-            const bool resc =
-                fl::softmax_tile<3>(r, 0, pos - j * kBN, sl2, m_ref, l, mt, corr, pk);
-            if (a.capture && mt > -INFINITY) list_insert(lv, li, mt, j);
-            // P buffer s of this tile is free once the PV of tile j-2 is done
-            if (j >= 2 && !fl::warp_wait(bar(L::BPVD + 2 * q + s), ((j >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
-            fl::store_p(gbase + L::kPOff + (2 * q + s) * 16384, row, pk);
+            bool resc;
+            if (kCapture) {
+                float mt;
+                resc = fl::softmax_tile<3>(r, 0, pos - j * kBN, sl2, m_ref, l, mt, corr, pk);
+                if (mt > -INFINITY) list_insert(lv, li, mt, j);
+            } else {
+                resc = fl::softmax_tile_lazy<kLazyPolyEvery>(r, pos - j * kBN, sl2, m_ref, l, corr, pk);
+            }
+            // P over the S buffer just read: its previous P (tile j-2) was consumed
+            // by a PV that executed before this tile's S MMA
+            fl::store_p_tmem(trow + 64 * s, pk);
             if (__any_sync(0xffffffffu, resc)) {
                 // O may only be touched once the PV of tile j-1 has finished
                 if (!fl::warp_wait(bar(L::BPVD + 2 * q + (s ^ 1)), ((j - 1) >> 1) & 1, abort_flag)) { ok = false; break; }
@@ -193,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             fl::store_o(trow + 128, true, 1.f / l, row_ok, a.o + orow * kD);
             if (row_ok) a.lse[orow] = lse2 * kLn2;
         }
-        if (a.capture) {
+        if (kCapture) {
             // ---- group merge.  Rows hh*P + pr of the g heads share position
             // pr; each row's list is sorted by (score desc, id asc).  The g
             // lists of a position are k-way merged in that order, skipping ids
@@ -324,11 +334,12 @@ cudaError_t launch_full_tc(const KParams& p, const void* q, const void* k, const
     a.P = P;
     a.n_ctas_q = (p.t_q + kNQ * P - 1) / (kNQ * P);
     a.capture = capture;
-    cudaError_t e = cudaFuncSetAttribute(full_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    auto kern = capture ? full_tc_kernel<true> : full_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemBytes);
     if (e != cudaSuccess) return e;
     const long long grid = (long long)a.n_ctas_q * p.batch * p.hkv;
-    full_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, a);
+    kern<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, a);
     return cudaGetLastError();
 }
 

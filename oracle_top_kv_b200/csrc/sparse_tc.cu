@@ -187,9 +187,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld32(trow + 64 * s, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
             tmem_ld32(trow + 64 * s + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
             tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(L::BSE + 2 * q + s));
 
             // global: this row keeps the block only if it selected it, and keys
             // <= t; window: keys t-w+1..t
@@ -208,9 +205,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t pk[32];
             const bool resc =
                 fl::softmax_tile<4, true>(r, first, lim, sl2, m_ref, l, mt, corr, pk);
-            // P buffer s is free once the PV of tile j-2 is done
-            if (j >= 2 && !fl::warp_wait(bar(L::BPVD + 2 * q + s), ((j >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
-            fl::store_p(gbase + L::kPOff + (2 * q + s) * 16384, row, pk);
+            // P over the S buffer just read: its previous P (tile j-2) was consumed
+            // by a PV that executed before this tile's S MMA
+            fl::store_p_tmem(trow + 64 * s, pk);
             if (__any_sync(0xffffffffu, resc)) {
                 // O may only be touched once the PV of tile j-1 has finished
                 if (!fl::warp_wait(bar(L::BPVD + 2 * q + (s ^ 1)), ((j - 1) >> 1) & 1, abort_flag)) { ok = false; break; }

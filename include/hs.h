@@ -102,7 +102,12 @@ typedef struct {
  * idx, idx_count: outputs (ascending, -1 padded).
  * sel_scores: optional output [batch][hkv][t_q][ksel] fp32, the S_bar of each
  *             selected entry (0 in the padding); NULL to skip.
- * workspace:  hs_workspace_size(p, HS_WS_FULL) bytes (may be 0 / NULL).
+ * workspace:  hs_workspace_size(p, HS_WS_FULL) bytes.  Non-zero only in token
+ *             mode for long scans (q_offset + t_q >= 2^18 keys, bf16, d = 128,
+ *             16 heads per group, k - w <= 1024): the candidate buffers of the
+ *             wide selector (about 38 MB on a 148-SM GPU).  With a smaller
+ *             workspace, or NULL, such a call takes the shared-memory selector
+ *             instead: same result rule, slower on long scans.
  */
 hs_status hs_full_attn_index(const hs_params* p, const void* q, const void* k,
                              const void* v, void* o, float* lse, int32_t* idx,
@@ -227,6 +232,18 @@ const char* hs_status_string(int32_t status);
  * devices, all streams).  A diagnostic for callers that account for launches;
  * it counts successful launch calls, not completed kernels. */
 uint64_t hs_launch_count(void);
+
+/* Failure-detection diagnostic (the pages have no counterpart).  Every wait
+ * of a kernel on another role of its CTA (a TMA copy, an MMA, a stage of the
+ * pipeline) is bounded: after `cycles` SM clock cycles it gives up, records
+ * HS_ERR_TIMEOUT in the device status word (read with hs_device_status),
+ * and the CTA drains the copies and MMAs it has in flight, frees its tensor
+ * memory and returns, leaving its outputs unspecified and the context usable.
+ * This sets that bound for kernels launched afterwards on the current device;
+ * cycles <= 0 restores the default of 2e9 (about a second).  Synchronous:
+ * call it while no kernel of this library runs on the device.  Tests use a
+ * bound of a few hundred cycles to make waits run out on purpose. */
+hs_status hs_set_wait_limit(int64_t cycles);
 
 #ifdef __cplusplus
 }

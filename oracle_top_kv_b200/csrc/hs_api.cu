@@ -288,6 +288,12 @@ hs_status hs_device_status(void* stream, int32_t* out) {
 
 uint64_t hs_launch_count(void) { return hs::g_launches.load(std::memory_order_relaxed); }
 
+hs_status hs_set_wait_limit(int64_t cycles) {
+    const long long v = cycles > 0 ? (long long)cycles : hs::tc::kWaitCycles;
+    return cudaMemcpyToSymbol(hs::g_wait_limit, &v, sizeof(v)) == cudaSuccess ? HS_OK
+                                                                               : HS_ERR_CUDA;
+}
+
 const char* hs_status_string(int32_t status) {
     switch (status) {
         case HS_OK: return "HS_OK";

@@ -21,6 +21,10 @@ __device__ int g_status = 0;
 
 __device__ __forceinline__ void set_status(int code) { atomicCAS(&g_status, 0, code); }
 
+// SM clock cycles a bounded wait may take before it gives up (per device; the
+// host sets it through hs_set_wait_limit, a failure-detection diagnostic).
+__device__ long long g_wait_limit = 2000000000ll;
+
 // ---------------------------------------------------------------- element I/O
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }

@@ -51,20 +51,22 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
     return ok != 0;
 }
 
-// Bounded wait: gives up after ~kWaitCycles SM cycles (about a second), or
-// as soon as another role of the CTA has given up.  A timeout records
-// HS_ERR_TIMEOUT in the device status word and raises the CTA's abort flag.
+// Bounded wait: gives up after g_wait_limit SM cycles (by default 2e9, about
+// a second), or as soon as another role of the CTA has given up.  A timeout
+// records HS_ERR_TIMEOUT in the device status word and raises the CTA's abort
+// flag.  Drains of work already in flight (copies, MMAs) wait up to the fixed
+// kWaitCycles instead: that work completes on its own.
 constexpr long long kWaitCycles = 2000000000ll;
 // sleep = false: poll without suspending (for single-thread roles on the
 // critical path, whose wake-up latency would delay the whole pipeline).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           bool sleep = true) {
     if (mbar_try_wait(bar, parity)) return true;
-    const long long t0 = clock64();
+    const long long t0 = clock64(), limit = g_wait_limit;
     for (;;) {
         if (sleep ? mbar_try_wait_sleep(bar, parity) : mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (clock64() - t0 > kWaitCycles) {
+        if (clock64() - t0 > limit) {
             *abort = 1;
             set_status(HS_ERR_TIMEOUT);
             return false;

@@ -25,7 +25,8 @@ HS_DECODE_FULL_INDEX, HS_DECODE_SPARSE = 0, 1
 HS_WS_FULL, HS_WS_SPARSE, HS_WS_DECODE_FULL, HS_WS_DECODE_SPARSE = 0, 1, 2, 3
 
 EXPORTS = ("hs_full_attn_index", "hs_sparse_attn_reuse", "hs_decode_step", "hs_workspace_size",
-           "hs_device_status", "hs_status_string", "hs_launch_count", "hs_decode_sparse_noalloc")
+           "hs_device_status", "hs_status_string", "hs_launch_count", "hs_decode_sparse_noalloc",
+           "hs_set_wait_limit")
 
 
 class HsError(RuntimeError):
@@ -76,6 +77,7 @@ def load(path: str = LIB_PATH):
     lib.hs_workspace_size.argtypes = [PP, I32]
     lib.hs_workspace_size.restype = S
     lib.hs_device_status.argtypes = [P, ctypes.POINTER(I32)]
+    lib.hs_set_wait_limit.argtypes = [ctypes.c_int64]
     lib.hs_status_string.argtypes = [I32]
     lib.hs_status_string.restype = ctypes.c_char_p
     lib.hs_launch_count.argtypes = []
@@ -182,6 +184,11 @@ def hs_device_status(stream=None) -> int:
     out = ctypes.c_int32(0)
     _check(load().hs_device_status(_stream(stream), ctypes.byref(out)), "hs_device_status")
     return int(out.value)
+
+
+def hs_set_wait_limit(cycles: int) -> None:
+    """Bound, in SM cycles, of the kernels' waits (<= 0: the default)."""
+    _check(load().hs_set_wait_limit(int(cycles)), "hs_set_wait_limit")
 
 
 def hs_status_string(code) -> str:

@@ -38,7 +38,12 @@
  *    launch returns HS_ERR_CUDA.  Errors found on the device (an index or
  *    sequence length out of range) skip the offending row and set a sticky
  *    per-device status word that hs_device_status reads.  No kernel traps.
- *  - Supported: head_dim in {64, 128}; hq % hkv == 0 with hq/hkv <= 16;
+ *  - Supported: head_dim in {64, 128, 256}; hq % hkv == 0 with hq/hkv <= 64
+ *    (HySparse2 is MQA 64/1 at head dim 256: "HySparse2 ...", 6.4, and its
+ *    reading notes' KV-cache table).  Groups of up to 16 heads at head_dim
+ *    <= 128 run on the tensor cores; wider groups and head_dim 256 run on
+ *    CUDA-core kernels (same results, lower throughput).  The paged and the
+ *    allocation-free entry points take groups of <= 16 heads, head_dim <= 128.
  *    block mode: block_size in {16, 32, 64, 128}, k % block_size == 0,
  *    k/block_size <= 64; token mode: 0 <= window <= k <= 4096;
  *    dtype fp32 or bf16 (decode: bf16 only).
@@ -232,6 +237,50 @@ const char* hs_status_string(int32_t status);
  * devices, all streams).  A diagnostic for callers that account for launches;
  * it counts successful launch calls, not completed kernels. */
 uint64_t hs_launch_count(void);
+
+/*
+ * Paged K^F/V^F ("HySparse 混合稀疏注意力（一）", 工程实现中的关键约束 items 2 and
+ * 3: the sparse index keeps logical token ids, a block table translates them
+ * into physical pages, and the kernel resolves the addresses while it loads
+ * each K/V row instead of first copying the selected rows to a contiguous
+ * buffer).  The cache is a pool of pages, k_pool and v_pool both
+ * [n_pages][hkv][page_size][head_dim] bf16; logical key i of sequence b lives
+ * in page block_table[b * max_pages + i / page_size] at row i % page_size.
+ * Index sets (idx) hold logical ids, exactly as the contiguous entry points
+ * write and read them.
+ */
+typedef struct {
+    const int32_t* block_table; /* DEVICE int32 [batch][max_pages]               */
+    int32_t page_size;          /* rows (tokens) per page, >= 1                  */
+    int32_t max_pages;          /* logical pages per sequence (table row stride) */
+    int32_t n_pages;            /* pages in the pool                             */
+} hs_pages;
+
+/*
+ * hs_sparse_attn_reuse over a paged K^F/V^F: the global branch only (no
+ * local window branch), bf16, token or block mode, any page size.
+ * p->t_kv must equal pages->max_pages * pages->page_size (the logical
+ * capacity), and n_pages * hkv * page_size must stay below 2^31.  A block
+ * table entry outside [0, n_pages) for a row that is read masks that row and
+ * sets HS_ERR_BOUNDS on the device.
+ */
+hs_status hs_sparse_attn_reuse_paged(const hs_params* p, const hs_pages* pages,
+                                     const void* q_sparse, const void* k_pool,
+                                     const void* v_pool, const int32_t* idx,
+                                     const int32_t* idx_count, void* o_global,
+                                     float* lse_global, void* stream);
+
+/*
+ * hs_decode_step over a paged cache: both kinds, same arguments and results
+ * as hs_decode_step with k_cache/v_cache replaced by the pools; p->t_kv as
+ * for hs_sparse_attn_reuse_paged; the workspace of HS_DECODE_FULL_INDEX is
+ * hs_workspace_size(p, HS_WS_DECODE_FULL) bytes.
+ */
+hs_status hs_decode_step_paged(const hs_params* p, const hs_pages* pages, int32_t kind,
+                               const void* q, const void* k_pool, const void* v_pool,
+                               const int32_t* seq_len, int32_t* idx, int32_t* idx_count,
+                               void* o, float* lse, float* sel_scores, void* workspace,
+                               size_t ws_bytes, void* stream);
 
 /* Failure-detection diagnostic (the pages have no counterpart).  Every wait
  * of a kernel on another role of its CTA (a TMA copy, an MMA, a stage of the

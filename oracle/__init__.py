@@ -14,6 +14,8 @@ Function map (titles of the pages the method is described on):
                       "HySparse2 ..." 4.2 (token-level top-k, forced window).
   sparse_attn      -- "HySparse 混合稀疏注意力（一）" sections on cross-layer KV
                       reuse and the two memories of one query; "HySparse ..." 3.3.
+  gather_pages     -- "HySparse 混合稀疏注意力（一）", 工程实现中的关键约束 item 2
+                      (logical ids, block table to physical pages).
   gate_sink        -- "HySparse 混合稀疏注意力（一）" section on the two sigmoid
                       gates; "HySparse ..." 3.3 (branch fusion) and its
                       configuration note on per-head sink biases.
@@ -316,6 +318,28 @@ def sparse_attn_rows(q, kf, vf, idx_rows, cnt_rows, rows, pos, mode, block_size,
         if k_loc is not None:
             out["o_l"][ns] = r["o_l"]
             out["lse_l"][ns] = r["lse_l"]
+    return out
+
+
+def gather_pages(pool, block_table, page_size):
+    """The logical K^F (or V^F) of a paged cache, [b, hkv, max_pages * page_size, d].
+
+    pool [n_pages, hkv, page_size, d] (numpy or torch), block_table [b, max_pages]:
+    logical key i of sequence b is row i % page_size of page
+    block_table[b, i // page_size] ("HySparse 混合稀疏注意力（一）", 工程实现中的关键约束
+    item 2: the index keeps logical token ids, the block table maps them to
+    physical pages).  The oracle then runs on this contiguous view.
+    """
+    pool = _f64_any(pool)
+    bt = np.asarray(block_table.cpu() if hasattr(block_table, "cpu") else block_table,
+                    dtype=np.int64)
+    b, mp = bt.shape
+    n_pages, hkv, ps, d = pool.shape
+    assert ps == page_size
+    out = np.zeros((b, hkv, mp * ps, d))
+    for bb in range(b):
+        for lp in range(mp):
+            out[bb, :, lp * ps:(lp + 1) * ps] = pool[bt[bb, lp]]
     return out
 
 

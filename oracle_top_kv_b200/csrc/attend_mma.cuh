@@ -13,6 +13,7 @@
 #pragma once
 
 #include "hs_common.cuh"
+#include "hs_kernels.cuh"
 #include "tc_ptx.cuh"
 
 namespace hs {
@@ -620,6 +621,50 @@ __device__ __forceinline__ void store_rows_t(const AttnStateT<D>& st, __nv_bfloa
 }
 
 // Keys first..last (inclusive) as contiguous chunks.
+// Logical key -> row of a paged pool for one (sequence, kv group): the
+// index sets keep logical token ids and the block table turns each into its
+// page and row as the gather loads it ("HySparse 混合稀疏注意力（一）",
+// 工程实现中的关键约束 item 2: the sparse index keeps logical token ranges,
+// a block table translates them into physical page pieces, the kernel reads
+// them directly).  A page id outside the pool marks the row masked and sets
+// HS_ERR_BOUNDS.
+struct PageMap {
+    const int32_t* bt;  // this sequence's row of the block table
+    int page_size, max_pages, n_pages, hkv, u;
+    __device__ __forceinline__ int row(int key) const {
+        const int lp = key / page_size;
+        const int pg = lp < max_pages ? bt[lp] : -1;
+        if (pg < 0 || pg >= n_pages) { set_status(HS_ERR_BOUNDS); return -1; }
+        return (pg * hkv + u) * page_size + (key - lp * page_size);
+    }
+};
+
+// A gathered-row source whose keys are translated through a PageMap; the
+// gather then reads from the pool's base.
+template <class Src>
+struct PagedSrc {
+    static constexpr bool kContig = false;
+    Src src;
+    PageMap pm;
+    __device__ __forceinline__ int key(int r) const {
+        const int k = src.key(r);
+        return k < 0 ? -1 : pm.row(k);
+    }
+};
+
+// Consecutive keys first..last as a gathered-row source (for pools, whose
+// rows are not consecutive across pages).
+struct KeyRange {
+    static constexpr bool kContig = false;
+    int first, last;
+    __device__ __forceinline__ int n_chunks() const { return (last - first + kChunk) / kChunk; }
+    __device__ __forceinline__ int key(int r) const { return first + r <= last ? first + r : -1; }
+};
+
+__device__ __forceinline__ PageMap page_map(const KParams& p, int b, int u) {
+    return PageMap{p.bt + (size_t)b * p.max_pages, p.page_size, p.max_pages, p.n_pages, p.hkv, u};
+}
+
 struct ContiguousKeys {
     static constexpr bool kContig = true;
     int first, last;

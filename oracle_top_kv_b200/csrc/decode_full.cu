@@ -128,6 +128,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
     decode_full_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, KParams p,
                              const __nv_bfloat16* __restrict__ q,
+                             const __nv_bfloat16* __restrict__ kc,
+                             const __nv_bfloat16* __restrict__ vc,
                              const int32_t* __restrict__ seq_len, DecodeWs ws) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -155,9 +157,18 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
         uint32_t qf[D / 16][4];
         load_q_frags<D>(qf, q + ((size_t)b * p.hq + u * g) * D, D, g);
         LogitExport<D> hook{ws.logits + (size_t)unit * p.t_kv * 16, last, g, p.scale_log2};
-        const ContiguousKeys src{first, last};
-        attend_rows_tma<D>(st, qf, &tm_k, &tm_v, unit, src.n_chunks(), src, sbase, ring,
-                           p.scale_log2, hook);
+        if (p.bt) {
+            // paged cache: consecutive logical keys, gathered row by row through
+            // the block table (a chunk may straddle pages); the hook gets each
+            // chunk's first logical key
+            const PagedSrc<KeyRange> src{KeyRange{first, last}, page_map(p, b, u)};
+            attend_rows<D>(st, qf, kc, vc, src.src.n_chunks(), src, sbase, p.scale_log2,
+                           [&](int c, float (&s)[4][4], int) { hook(c, s, first + c * kChunk); });
+        } else {
+            const ContiguousKeys src{first, last};
+            attend_rows_tma<D>(st, qf, &tm_k, &tm_v, unit, src.n_chunks(), src, sbase, ring,
+                               p.scale_log2, hook);
+        }
     }
     store_partial<D>(st, ws.part + (size_t)task * 16 * (D + 2), g);
 }
@@ -502,8 +513,11 @@ static cudaError_t launch_decode_full_t(const KParams& p, const void* q, const v
     const size_t smem = (size_t)kDecodeWarps * (WarpSmem<D>::kBytes + 16) + 1024;
     CUtensorMap mk, mv;
     const long long units = (long long)p.batch * p.hkv;
-    if (!tc::encode_rows(&mk, kc, D, p.t_kv, units, kChunk) ||
-        !tc::encode_rows(&mv, vc, D, p.t_kv, units, kChunk))
+    // a paged pool is read by gathers only: its maps (unused) span the pool
+    const long long rows = p.bt ? (long long)p.n_pages * p.hkv * p.page_size : p.t_kv;
+    const long long mu = p.bt ? 1 : units;
+    if (!tc::encode_rows(&mk, kc, D, rows, mu, kChunk) ||
+        !tc::encode_rows(&mv, vc, D, rows, mu, kChunk))
         return cudaErrorInvalidValue;
     auto kern = decode_full_split_kernel<D>;
     cudaError_t e =
@@ -511,7 +525,8 @@ static cudaError_t launch_decode_full_t(const KParams& p, const void* q, const v
     if (e != cudaSuccess) return e;
     const int n_tasks = p.batch * p.hkv * w.n_split;
     kern<<<(n_tasks + kDecodeWarps - 1) / kDecodeWarps, kDecodeWarps * 32, smem, st>>>(
-        mk, mv, p, (const __nv_bfloat16*)q, seq_len, w);
+        mk, mv, p, (const __nv_bfloat16*)q, (const __nv_bfloat16*)kc, (const __nv_bfloat16*)vc,
+        seq_len, w);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = launch_decode_combine(p, w.part, w.n_split, seq_len, o, lse, w.lse2, st)) !=
         cudaSuccess)

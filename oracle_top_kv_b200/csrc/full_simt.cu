@@ -2,8 +2,11 @@
 // version.  Exact fp32 arithmetic for any supported shape; this is the path
 // of the fp32 configurations and the general fallback of the bf16 ones.
 //
-// One CTA per (batch, kv group u, query row j), one warp per head of the group
-// for the attention, then all warps for the selection:
+// One CTA per (batch, kv group u, query row j) -- or, in decode, per (sequence,
+// kv group) at the sequence's newest position -- with up to 16 warps that
+// take the group's heads in turn for the attention (groups of up to 64
+// heads, head_dim 64, 128 or 256: the MQA 64/1 d = 256 shape of "HySparse2
+// ...", 6.4), then all warps for the selection:
 //
 //  phase A (per head h):  online softmax over keys 0..t in chunks of 32
 //      ("HySparse 混合稀疏注意力（一）", exact attention and the online-softmax
@@ -31,6 +34,8 @@ __device__ __forceinline__ float dot_row(const float* __restrict__ qs, const T* 
     return s;
 }
 
+constexpr int kSimtMaxGroup = 64;
+
 template <typename T, int D>
 __global__ void __launch_bounds__(512) full_simt_kernel(KParams p, const T* __restrict__ q,
                                                         const T* __restrict__ k,
@@ -38,21 +43,32 @@ __global__ void __launch_bounds__(512) full_simt_kernel(KParams p, const T* __re
                                                         float* __restrict__ lse,
                                                         int32_t* __restrict__ idx,
                                                         int32_t* __restrict__ cnt,
-                                                        float* __restrict__ sel, int do_attn) {
+                                                        float* __restrict__ sel, int do_attn,
+                                                        const int32_t* __restrict__ seq_len) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const int j = blockIdx.x, u = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nw = blockDim.x >> 5;
     const int g = p.group;
-    const int t = p.q_offset + j;
+    // decode (seq_len given): the one query is the sequence's newest token
+    const int t = seq_len ? seq_len[b] - 1 : p.q_offset + j;
+    if (t < 0 || t >= p.t_kv) {  // uniform over the CTA
+        if (threadIdx.x == 0) {
+            set_status(HS_ERR_BOUNDS);
+            cnt[((size_t)b * p.hkv + u) * p.t_q + j] = 0;
+        }
+        return;
+    }
 
     const int Kc = p.mode == 0 ? p.ksel : p.k - p.window;  // ranked slots
 
     float* qs = reinterpret_cast<float*>(smem_raw);   // [g][D]
-    float* lse2 = qs + g * D;                          // [16]
+    float* lse2 = qs + g * D;                          // [kSimtMaxGroup]
     __shared__ int s_count;
     __shared__ unsigned long long s_thresh;
     BlockTopK topk;
-    topk.setup(reinterpret_cast<unsigned char*>(lse2 + 16), Kc, blockDim.x, &s_count, &s_thresh);
+    topk.setup(reinterpret_cast<unsigned char*>(lse2 + kSimtMaxGroup), Kc, blockDim.x, &s_count,
+               &s_thresh);
 
     const T* kbase = k + ((size_t)b * p.hkv + u) * p.t_kv * D;
     const T* vbase = v + ((size_t)b * p.hkv + u) * p.t_kv * D;
@@ -64,15 +80,15 @@ __global__ void __launch_bounds__(512) full_simt_kernel(KParams p, const T* __re
     }
     __syncthreads();
 
-    // ---------------- phase A: exact attention, one warp per head
+    // ---------------- phase A: exact attention, the warps take the heads in turn
     constexpr int E = D / 32;
     if (!do_attn) {
         // selection only: the attention (and lse) came from another kernel
-        if (threadIdx.x < g)
-            lse2[threadIdx.x] = lse[((size_t)b * p.hq + u * g + threadIdx.x) * p.t_q + j] * kLog2e;
-    } else if (warp < g) {
-        const int h = u * g + warp;
-        const float* qh = qs + warp * D;
+        for (int hh = threadIdx.x; hh < g; hh += blockDim.x)
+            lse2[hh] = lse[((size_t)b * p.hq + u * g + hh) * p.t_q + j] * kLog2e;
+    } else for (int hw = warp; hw < g; hw += nw) {
+        const int h = u * g + hw;
+        const float* qh = qs + hw * D;
         float m = -INFINITY, l = 0.f, acc[E];
 #pragma unroll
         for (int e = 0; e < E; ++e) acc[e] = 0.f;
@@ -101,7 +117,7 @@ __global__ void __launch_bounds__(512) full_simt_kernel(KParams p, const T* __re
         for (int e = 0; e < E; ++e) orow[e] = from_f<T>(acc[e] * inv);
         const float l2 = m + log2f(l);
         if (lane == 0) {
-            lse2[warp] = l2;
+            lse2[hw] = l2;
             lse[((size_t)b * p.hq + h) * p.t_q + j] = l2 * kLn2;
         }
     }
@@ -165,10 +181,11 @@ __global__ void __launch_bounds__(512) full_simt_kernel(KParams p, const T* __re
 template <typename T, int D>
 static cudaError_t launch_full_simt_t(const KParams& p, const void* q, const void* k,
                                       const void* v, void* o, float* lse, int32_t* idx,
-                                      int32_t* cnt, float* sel, int do_attn, cudaStream_t st) {
-    const int nwarps = p.group < 4 ? 4 : p.group;
+                                      int32_t* cnt, float* sel, int do_attn,
+                                      const int32_t* seq_len, cudaStream_t st) {
+    const int nwarps = p.group < 4 ? 4 : (p.group > 16 ? 16 : p.group);
     const int Kc = p.mode == 0 ? p.ksel : p.k - p.window;
-    const size_t smem = sizeof(float) * (p.group * D + 16) +
+    const size_t smem = sizeof(float) * (p.group * D + kSimtMaxGroup) +
                         BlockTopK::smem_bytes(Kc, nwarps * 32);
     auto kern = full_simt_kernel<T, D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -176,21 +193,29 @@ static cudaError_t launch_full_simt_t(const KParams& p, const void* q, const voi
     if (e != cudaSuccess) return e;
     dim3 grid(p.t_q, p.hkv, p.batch);
     kern<<<grid, nwarps * 32, smem, st>>>(p, (const T*)q, (const T*)k, (const T*)v, (T*)o, lse,
-                                           idx, cnt, sel, do_attn);
+                                           idx, cnt, sel, do_attn, seq_len);
     return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_full_simt_d(const KParams& p, const void* q, const void* k,
+                                      const void* v, void* o, float* lse, int32_t* idx,
+                                      int32_t* cnt, float* sel, int do_attn,
+                                      const int32_t* seq_len, cudaStream_t st) {
+    if (p.head_dim == 64)
+        return launch_full_simt_t<T, 64>(p, q, k, v, o, lse, idx, cnt, sel, do_attn, seq_len, st);
+    if (p.head_dim == 128)
+        return launch_full_simt_t<T, 128>(p, q, k, v, o, lse, idx, cnt, sel, do_attn, seq_len, st);
+    return launch_full_simt_t<T, 256>(p, q, k, v, o, lse, idx, cnt, sel, do_attn, seq_len, st);
 }
 
 cudaError_t launch_full_simt(const KParams& p, int dtype, const void* q, const void* k,
                              const void* v, void* o, float* lse, int32_t* idx, int32_t* cnt,
-                             float* sel, int do_attn, cudaStream_t st) {
-    if (dtype == HS_FP32) {
-        if (p.head_dim == 64)
-            return launch_full_simt_t<float, 64>(p, q, k, v, o, lse, idx, cnt, sel, do_attn, st);
-        return launch_full_simt_t<float, 128>(p, q, k, v, o, lse, idx, cnt, sel, do_attn, st);
-    }
-    if (p.head_dim == 64)
-        return launch_full_simt_t<__nv_bfloat16, 64>(p, q, k, v, o, lse, idx, cnt, sel, do_attn, st);
-    return launch_full_simt_t<__nv_bfloat16, 128>(p, q, k, v, o, lse, idx, cnt, sel, do_attn, st);
+                             float* sel, int do_attn, cudaStream_t st, const int32_t* seq_len) {
+    if (dtype == HS_FP32)
+        return launch_full_simt_d<float>(p, q, k, v, o, lse, idx, cnt, sel, do_attn, seq_len, st);
+    return launch_full_simt_d<__nv_bfloat16>(p, q, k, v, o, lse, idx, cnt, sel, do_attn, seq_len,
+                                             st);
 }
 
 }  // namespace hs

@@ -301,7 +301,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 bool full_tc_supported(const KParams& p, int dtype) {
     if (dtype != HS_BF16 || p.head_dim != 128) return false;
     if (128 % p.group != 0) return false;
-    if (p.mode == 0) return p.block_size == tc::kBN && p.ksel <= tc::kList;
+    // block mode: the group merge runs on g consecutive lanes of a warp
+    if (p.mode == 0) return p.block_size == tc::kBN && p.ksel <= tc::kList && p.group <= 16;
     return true;
 }
 

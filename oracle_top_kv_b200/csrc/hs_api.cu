@@ -65,8 +65,8 @@ hs_status resolve(const hs_params* p, bool decode, KParams* kp) {
     if (big > 4.0e15) return HS_ERR_INVALID_ARG;
     // what this build implements
     const int g = p->hq / p->hkv;
-    if (p->head_dim != 64 && p->head_dim != 128) return HS_ERR_UNSUPPORTED;
-    if (g > 16) return HS_ERR_UNSUPPORTED;
+    if (p->head_dim != 64 && p->head_dim != 128 && p->head_dim != 256) return HS_ERR_UNSUPPORTED;
+    if (g > 64) return HS_ERR_UNSUPPORTED;
     if (p->mode == HS_SEL_BLOCK) {
         const int B = p->block_size;
         if (B != 16 && B != 32 && B != 64 && B != 128) return HS_ERR_UNSUPPORTED;
@@ -93,6 +93,10 @@ hs_status resolve(const hs_params* p, bool decode, KParams* kp) {
 }
 
 hs_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HS_OK : HS_ERR_CUDA; }
+
+// The mma.sync gather and decode kernels: groups of up to 16 heads, d <= 128.
+// Wider groups and d = 256 (the MQA 64/1, d = 256 shape) take the SIMT kernels.
+bool mma_shape(const KParams& kp) { return kp.group <= 16 && kp.head_dim <= 128; }
 
 // Launch a sequence through fn() and count its kernels when it succeeds.
 template <typename Fn>
@@ -169,6 +173,12 @@ hs_status hs_sparse_attn_reuse(const hs_params* p, const void* q_sparse, const v
                                           local ? k_local : nullptr, v_local, o_global,
                                           lse_global, o_local, lse_local, st);
         });
+    if (!mma_shape(kp))
+        return launched(1, [&] {
+            return hs::launch_sparse_simt(kp, p->dtype, q_sparse, k_f, v_f, idx, idx_count,
+                                          local ? k_local : nullptr, v_local, o_global,
+                                          lse_global, o_local, lse_local, st);
+        });
     if (hs::sparse_tc_supported(kp, p->dtype)) {
         // global branch, then the window branch, on the tensor cores
         return launched(local ? 2 : 1, [&] {
@@ -191,6 +201,7 @@ size_t hs_workspace_size(const hs_params* p, int32_t which) {
     const bool decode = which == HS_WS_DECODE_FULL || which == HS_WS_DECODE_SPARSE;
     if (which < HS_WS_FULL || which > HS_WS_DECODE_SPARSE) return (size_t)-1;
     if (resolve(p, decode, &kp) != HS_OK) return (size_t)-1;
+    if (decode && !mma_shape(kp)) return 0;  // the SIMT decode kernels need none
     switch (which) {
         case HS_WS_FULL:
             return hs::full_tc_supported(kp, p->dtype) && hs::token_select_wide_applies(kp, p->dtype)
@@ -214,6 +225,20 @@ hs_status hs_decode_step(const hs_params* p, int32_t kind, const void* q, const 
     if (!ok_ptr(q) || !ok_ptr(k_cache) || !ok_ptr(v_cache) || !ok_ptr(seq_len) || !ok_ptr(idx) ||
         !ok_ptr(idx_count) || !ok_ptr(o) || !ok_opt(lse) || !ok_opt(sel_scores))
         return HS_ERR_INVALID_ARG;
+    if (!mma_shape(kp)) {  // wide groups / d = 256: one SIMT kernel per step, no workspace
+        cudaStream_t st = static_cast<cudaStream_t>(stream);
+        if (kind == HS_DECODE_FULL_INDEX) {
+            if (!lse) return HS_ERR_INVALID_ARG;
+            return launched(1, [&] {
+                return hs::launch_full_simt(kp, p->dtype, q, k_cache, v_cache, o, lse, idx,
+                                            idx_count, sel_scores, 1, st, seq_len);
+            });
+        }
+        return launched(1, [&] {
+            return hs::launch_sparse_simt(kp, p->dtype, q, k_cache, v_cache, idx, idx_count,
+                                          nullptr, nullptr, o, lse, nullptr, nullptr, st, seq_len);
+        });
+    }
     const size_t need = kind == HS_DECODE_FULL_INDEX ? hs::decode_full_workspace(kp)
                                                      : hs::decode_sparse_workspace(kp);
     if (need > 0 && (workspace == nullptr || ws_bytes < need || !aligned16(workspace)))
@@ -233,6 +258,79 @@ hs_status hs_decode_step(const hs_params* p, int32_t kind, const void* q, const 
     });
 }
 
+}  // extern "C"
+
+namespace {
+// Validates a block table description and records it in kp.
+hs_status set_pages(const hs_params* p, const hs_pages* pages, KParams* kp) {
+    if (!pages || !ok_ptr(pages->block_table)) return HS_ERR_INVALID_ARG;
+    if (pages->page_size < 1 || pages->max_pages < 1 || pages->n_pages < 1)
+        return HS_ERR_INVALID_ARG;
+    if ((long long)pages->max_pages * pages->page_size != p->t_kv) return HS_ERR_INVALID_ARG;
+    if ((long long)pages->n_pages * p->hkv * pages->page_size >= (1ll << 31))
+        return HS_ERR_INVALID_ARG;
+    kp->bt = pages->block_table;
+    kp->page_size = pages->page_size;
+    kp->max_pages = pages->max_pages;
+    kp->n_pages = pages->n_pages;
+    return HS_OK;
+}
+}  // namespace
+
+extern "C" {
+
+hs_status hs_sparse_attn_reuse_paged(const hs_params* p, const hs_pages* pages,
+                                     const void* q_sparse, const void* k_pool,
+                                     const void* v_pool, const int32_t* idx,
+                                     const int32_t* idx_count, void* o_global,
+                                     float* lse_global, void* stream) {
+    KParams kp;
+    hs_status s = resolve(p, false, &kp);
+    if (s != HS_OK) return s;
+    if ((s = set_pages(p, pages, &kp)) != HS_OK) return s;
+    if (!ok_ptr(q_sparse) || !ok_ptr(k_pool) || !ok_ptr(v_pool) || !ok_ptr(idx) ||
+        !ok_ptr(idx_count) || !ok_ptr(o_global) || !ok_ptr(lse_global))
+        return HS_ERR_INVALID_ARG;
+    if (p->dtype != HS_BF16 || !mma_shape(kp)) return HS_ERR_UNSUPPORTED;
+    if (kp.t_q == 0) return HS_OK;
+    return launched(1, [&] {
+        return hs::launch_sparse_mma(kp, q_sparse, k_pool, v_pool, idx, idx_count, nullptr,
+                                     nullptr, o_global, lse_global, nullptr, nullptr,
+                                     static_cast<cudaStream_t>(stream));
+    });
+}
+
+hs_status hs_decode_step_paged(const hs_params* p, const hs_pages* pages, int32_t kind,
+                               const void* q, const void* k_pool, const void* v_pool,
+                               const int32_t* seq_len, int32_t* idx, int32_t* idx_count,
+                               void* o, float* lse, float* sel_scores, void* workspace,
+                               size_t ws_bytes, void* stream) {
+    KParams kp;
+    hs_status s = resolve(p, true, &kp);
+    if (s != HS_OK) return s;
+    if ((s = set_pages(p, pages, &kp)) != HS_OK) return s;
+    if (kind != HS_DECODE_FULL_INDEX && kind != HS_DECODE_SPARSE) return HS_ERR_INVALID_ARG;
+    if (p->dtype != HS_BF16 || p->mode != HS_SEL_TOKEN || !mma_shape(kp)) return HS_ERR_UNSUPPORTED;
+    if (!ok_ptr(q) || !ok_ptr(k_pool) || !ok_ptr(v_pool) || !ok_ptr(seq_len) || !ok_ptr(idx) ||
+        !ok_ptr(idx_count) || !ok_ptr(o) || !ok_opt(lse) || !ok_opt(sel_scores))
+        return HS_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (kind == HS_DECODE_FULL_INDEX) {
+        const size_t need = hs::decode_full_workspace(kp);
+        if (need > 0 && (workspace == nullptr || ws_bytes < need || !aligned16(workspace)))
+            return HS_ERR_WORKSPACE;
+        if (!lse) return HS_ERR_INVALID_ARG;
+        return launched(hs::decode_full_kernel_count(kp), [&] {
+            return hs::launch_decode_full(kp, q, k_pool, v_pool, seq_len, idx, idx_count, o, lse,
+                                          sel_scores, workspace, st);
+        });
+    }
+    return launched(1, [&] {
+        return hs::launch_decode_sparse(kp, q, k_pool, v_pool, seq_len, idx, idx_count, o, lse,
+                                        nullptr, st);
+    });
+}
+
 hs_status hs_decode_sparse_noalloc(const hs_params* p, const void* q, const void* k_cache,
                                    const void* v_cache, const int32_t* seq_len,
                                    const int32_t* idx, const int32_t* idx_count, void* o,
@@ -240,7 +338,7 @@ hs_status hs_decode_sparse_noalloc(const hs_params* p, const void* q, const void
     KParams kp;
     hs_status s = resolve(p, true, &kp);
     if (s != HS_OK) return s;
-    if (p->dtype != HS_BF16 || p->mode != HS_SEL_TOKEN) return HS_ERR_UNSUPPORTED;
+    if (p->dtype != HS_BF16 || p->mode != HS_SEL_TOKEN || !mma_shape(kp)) return HS_ERR_UNSUPPORTED;
     if (!ok_ptr(q) || !ok_ptr(k_cache) || !ok_ptr(v_cache) || !ok_ptr(seq_len) || !ok_ptr(idx) ||
         !ok_ptr(idx_count) || !ok_ptr(o) || !ok_opt(lse))
         return HS_ERR_INVALID_ARG;

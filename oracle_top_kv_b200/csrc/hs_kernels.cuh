@@ -19,12 +19,21 @@ struct KParams {
     int k, window;
     int ksel;        // entries per index row
     float scale_log2;  // softmax scale * log2(e)
+    // Paged K^F/V^F (bt != nullptr): the cache is a pool of pages of
+    // page_size rows per kv head, [n_pages][hkv][page_size][d]; logical key i
+    // of sequence b lives in page bt[b * max_pages + i / page_size], row
+    // i % page_size.  t_kv is then max_pages * page_size.
+    const int32_t* bt = nullptr;
+    int page_size = 0, max_pages = 0, n_pages = 0;
 };
 
 // do_attn = 0: selection only, reading lse from a previous attention pass.
+// seq_len (decode, t_q = 1): each sequence's query is its newest token.
+// Groups of up to 64 heads, head_dim 64, 128 or 256.
 cudaError_t launch_full_simt(const KParams& p, int dtype, const void* q, const void* k,
                              const void* v, void* o, float* lse, int32_t* idx, int32_t* cnt,
-                             float* sel, int do_attn, cudaStream_t st);
+                             float* sel, int do_attn, cudaStream_t st,
+                             const int32_t* seq_len = nullptr);
 
 // tcgen05 flash attention (bf16, d = 128).  capture = 1: block-mode index.
 bool full_tc_supported(const KParams& p, int dtype);
@@ -32,10 +41,12 @@ cudaError_t launch_full_tc(const KParams& p, const void* q, const void* k, const
                            void* o, float* lse, int32_t* idx, int32_t* cnt, float* sel,
                            int capture, cudaStream_t st);
 
+// seq_len as for launch_full_simt.  Groups of up to 64 heads, head_dim 64,
+// 128 or 256.
 cudaError_t launch_sparse_simt(const KParams& p, int dtype, const void* q, const void* kf,
                                const void* vf, const int32_t* idx, const int32_t* cnt,
                                const void* kl, const void* vl, void* og, float* lseg, void* ol,
-                               float* lsel, cudaStream_t st);
+                               float* lsel, cudaStream_t st, const int32_t* seq_len = nullptr);
 
 // bf16 tensor-core paths (mma.sync fragments; d = 64 or 128).  global = false:
 // the window branch only (the global branch is computed by sparse_tc).

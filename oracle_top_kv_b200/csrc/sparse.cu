@@ -118,41 +118,46 @@ __device__ void simt_attend(const float* qh, const T* kbase, const T* vbase, int
     const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e) orow[lane * E + e] = from_f<T>(acc[e] * inv);
-    if (lane == 0) *lse_out = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+    if (lane == 0 && lse_out) *lse_out = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
 }
 
+// One CTA per (batch, kv group, query row) -- in decode per (sequence, kv
+// group) at the newest position -- whose warps take the group's heads in
+// turn (groups of up to 64 heads, head_dim up to 256).
 template <typename T, int D>
 __global__ void sparse_simt_kernel(KParams p, const T* __restrict__ q, const T* __restrict__ kf,
                                    const T* __restrict__ vf, const int32_t* __restrict__ idx,
                                    const int32_t* __restrict__ cnt, const T* __restrict__ kl,
                                    const T* __restrict__ vl, T* __restrict__ og,
                                    float* __restrict__ lseg, T* __restrict__ ol,
-                                   float* __restrict__ lsel) {
-    __shared__ float qs[16 * D];
+                                   float* __restrict__ lsel, const int32_t* __restrict__ seq_len) {
+    extern __shared__ float qs[];  // [g][D]
     const int j = blockIdx.x, u = blockIdx.y, b = blockIdx.z;
-    const int warp = threadIdx.x >> 5;
+    const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     const int g = p.group;
-    const int t = p.q_offset + j;
+    const int t = seq_len ? seq_len[b] - 1 : p.q_offset + j;
+    const bool valid = t >= 0 && t < p.t_kv;
+    if (!valid && threadIdx.x == 0) set_status(HS_ERR_BOUNDS);
     for (int x = threadIdx.x; x < g * D; x += blockDim.x) {
         const int h = u * g + x / D;
         qs[x] = to_f(q[(((size_t)b * p.hq + h) * p.t_q + j) * D + x % D]) * p.scale_log2;
     }
     __syncthreads();
-    if (warp >= g) return;
-    const int h = u * g + warp;
     const size_t row = ((size_t)b * p.hkv + u) * p.t_q + j;
-    const size_t orow = ((size_t)b * p.hq + h) * p.t_q + j;
     const size_t kvoff = ((size_t)b * p.hkv + u) * p.t_kv * D;
-    const int c = clamp_count(cnt[row], p.ksel);
+    const int c = valid ? clamp_count(cnt[row], p.ksel) : 0;
     const int n_rows = p.mode == 0 ? c * p.block_size : c;
-    GatherKeys keys{idx + row * p.ksel, n_rows, p.block_size, t, p.mode};
-    simt_attend<T, D>(qs + warp * D, kf + kvoff, vf + kvoff, n_rows, keys, og + orow * D,
-                      lseg + orow);
-    if (kl) {
-        const int first = max(0, t - p.window + 1);
-        simt_attend<T, D>(qs + warp * D, kl + kvoff, vl + kvoff, t - first + 1,
-                          [=](int r) { return first + r <= t ? first + r : -1; }, ol + orow * D,
-                          lsel + orow);
+    const GatherKeys keys{idx + row * p.ksel, n_rows, p.block_size, t, p.mode};
+    for (int hw = warp; hw < g; hw += nw) {
+        const size_t orow = ((size_t)b * p.hq + u * g + hw) * p.t_q + j;
+        simt_attend<T, D>(qs + hw * D, kf + kvoff, vf + kvoff, n_rows, keys, og + orow * D,
+                          lseg ? lseg + orow : nullptr);
+        if (kl) {
+            const int first = max(0, t - p.window + 1);
+            simt_attend<T, D>(qs + hw * D, kl + kvoff, vl + kvoff, valid ? t - first + 1 : 0,
+                              [=](int r) { return first + r <= t ? first + r : -1; },
+                              ol + orow * D, lsel + orow);
+        }
     }
 }
 
@@ -160,30 +165,46 @@ template <typename T, int D>
 static cudaError_t launch_sparse_simt_t(const KParams& p, const void* q, const void* kf,
                                         const void* vf, const int32_t* idx, const int32_t* cnt,
                                         const void* kl, const void* vl, void* og, float* lseg,
-                                        void* ol, float* lsel, cudaStream_t st) {
+                                        void* ol, float* lsel, const int32_t* seq_len,
+                                        cudaStream_t st) {
     dim3 grid(p.t_q, p.hkv, p.batch);
-    sparse_simt_kernel<T, D><<<grid, 32 * p.group, 0, st>>>(
-        p, (const T*)q, (const T*)kf, (const T*)vf, idx, cnt, (const T*)kl, (const T*)vl, (T*)og,
-        lseg, (T*)ol, lsel);
+    const int threads = 32 * (p.group < 16 ? p.group : 16);
+    const size_t smem = sizeof(float) * p.group * D;
+    auto kern = sparse_simt_kernel<T, D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, threads, smem, st>>>(p, (const T*)q, (const T*)kf, (const T*)vf, idx, cnt,
+                                       (const T*)kl, (const T*)vl, (T*)og, lseg, (T*)ol, lsel,
+                                       seq_len);
     return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_sparse_simt_d(const KParams& p, const void* q, const void* kf,
+                                        const void* vf, const int32_t* idx, const int32_t* cnt,
+                                        const void* kl, const void* vl, void* og, float* lseg,
+                                        void* ol, float* lsel, const int32_t* seq_len,
+                                        cudaStream_t st) {
+    if (p.head_dim == 64)
+        return launch_sparse_simt_t<T, 64>(p, q, kf, vf, idx, cnt, kl, vl, og, lseg, ol, lsel,
+                                           seq_len, st);
+    if (p.head_dim == 128)
+        return launch_sparse_simt_t<T, 128>(p, q, kf, vf, idx, cnt, kl, vl, og, lseg, ol, lsel,
+                                            seq_len, st);
+    return launch_sparse_simt_t<T, 256>(p, q, kf, vf, idx, cnt, kl, vl, og, lseg, ol, lsel,
+                                        seq_len, st);
 }
 
 cudaError_t launch_sparse_simt(const KParams& p, int dtype, const void* q, const void* kf,
                                const void* vf, const int32_t* idx, const int32_t* cnt,
                                const void* kl, const void* vl, void* og, float* lseg, void* ol,
-                               float* lsel, cudaStream_t st) {
-    if (dtype == HS_FP32) {
-        if (p.head_dim == 64)
-            return launch_sparse_simt_t<float, 64>(p, q, kf, vf, idx, cnt, kl, vl, og, lseg, ol,
-                                                   lsel, st);
-        return launch_sparse_simt_t<float, 128>(p, q, kf, vf, idx, cnt, kl, vl, og, lseg, ol,
-                                                lsel, st);
-    }
-    if (p.head_dim == 64)
-        return launch_sparse_simt_t<__nv_bfloat16, 64>(p, q, kf, vf, idx, cnt, kl, vl, og, lseg,
-                                                       ol, lsel, st);
-    return launch_sparse_simt_t<__nv_bfloat16, 128>(p, q, kf, vf, idx, cnt, kl, vl, og, lseg, ol,
-                                                    lsel, st);
+                               float* lsel, cudaStream_t st, const int32_t* seq_len) {
+    if (dtype == HS_FP32)
+        return launch_sparse_simt_d<float>(p, q, kf, vf, idx, cnt, kl, vl, og, lseg, ol, lsel,
+                                           seq_len, st);
+    return launch_sparse_simt_d<__nv_bfloat16>(p, q, kf, vf, idx, cnt, kl, vl, og, lseg, ol, lsel,
+                                               seq_len, st);
 }
 
 // ------------------------------------------------------------ tensor-core path
@@ -268,6 +289,11 @@ __global__ void __launch_bounds__(W * 32)
         AttnStateT<D> st;
         st.init();
         if (!do_global) {
+        } else if (p.bt) {  // paged K^F/V^F: every row through the block table
+            const PagedSrc<GatherKeys> keys{
+                GatherKeys{idx + row * p.ksel, n_rows, p.block_size, t, p.mode}, page_map(p, b, u)};
+            attend_rows_t<D, S>(st, qb, kf, vf, (n_rows + kChunk - 1) / kChunk, keys, sbase,
+                                p.scale_log2);
         } else if (p.mode == 0 && p.block_size % kChunk == 0) {
             BlockChunks src{idx + row * p.ksel, p.block_size, t};
             attend_rows_tma_t<D, S>(st, qb, &tm_kf, &tm_vf, unit, c * (p.block_size / kChunk),
@@ -295,6 +321,11 @@ __global__ void __launch_bounds__(W * 32)
     AttnState<D> st;
     st.init();
     if (!do_global) {
+    } else if (p.bt) {  // paged K^F/V^F: every row through the block table
+        const PagedSrc<GatherKeys> keys{
+            GatherKeys{idx + row * p.ksel, n_rows, p.block_size, t, p.mode}, page_map(p, b, u)};
+        attend_rows<D, S>(st, qf, kf, vf, (n_rows + kChunk - 1) / kChunk, keys, sbase,
+                          p.scale_log2, NoHook{});
     } else if (p.mode == 0 && p.block_size % kChunk == 0) {
         BlockChunks src{idx + row * p.ksel, p.block_size, t};
         attend_rows_tma<D, S>(st, qf, &tm_kf, &tm_vf, unit, c * (p.block_size / kChunk), src,
@@ -345,8 +376,11 @@ static cudaError_t launch_sparse_mma_t(const KParams& p, const void* q, const vo
     const int flags = (kl ? 1 : 0) | (global ? 0 : 2);
     CUtensorMap mk, mv, mkl, mvl;
     const long long units = (long long)p.batch * p.hkv;
-    if (!tc::encode_rows(&mk, kf, D, p.t_kv, units, kChunk) ||
-        !tc::encode_rows(&mv, vf, D, p.t_kv, units, kChunk))
+    // a paged pool is read by gathers only: its maps (unused) span the pool
+    const long long rows = p.bt ? (long long)p.n_pages * p.hkv * p.page_size : p.t_kv;
+    const long long mu = p.bt ? 1 : units;
+    if (!tc::encode_rows(&mk, kf, D, rows, mu, kChunk) ||
+        !tc::encode_rows(&mv, vf, D, rows, mu, kChunk))
         return cudaErrorInvalidValue;
     if (kl) {
         if (!tc::encode_rows(&mkl, kl, D, p.t_kv, units, kChunk) ||
@@ -608,9 +642,15 @@ __global__ void __launch_bounds__(kSparseWarps * 32)
         uint32_t qf[D / 16][4];
         load_q_frags<D>(qf, q + ((size_t)b * p.hq + u * g) * D, D, g);
         const StridedGather keys{idx + (size_t)unit * p.ksel, c, t, wg, W};
-        const size_t kvoff = (size_t)unit * p.t_kv * D;
-        attend_rows<D>(st, qf, kc + kvoff, vc + kvoff, mine, keys,
-                       base + warp * WarpSmem<D>::kBytes, p.scale_log2, NoHook{});
+        if (p.bt) {  // paged cache: every row through the block table
+            const PagedSrc<StridedGather> pkeys{keys, page_map(p, b, u)};
+            attend_rows<D>(st, qf, kc, vc, mine, pkeys, base + warp * WarpSmem<D>::kBytes,
+                           p.scale_log2, NoHook{});
+        } else {
+            const size_t kvoff = (size_t)unit * p.t_kv * D;
+            attend_rows<D>(st, qf, kc + kvoff, vc + kvoff, mine, keys,
+                           base + warp * WarpSmem<D>::kBytes, p.scale_log2, NoHook{});
+        }
     } else if (crank == 0 && threadIdx.x == 0) {
         set_status(HS_ERR_BOUNDS);
     }

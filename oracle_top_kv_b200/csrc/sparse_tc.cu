@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }  // namespace stc
 
 bool sparse_tc_supported(const KParams& p, int dtype) {
-    if (dtype != HS_BF16 || p.head_dim != stc::kD || p.mode != 0) return false;
+    if (dtype != HS_BF16 || p.head_dim != stc::kD || p.mode != 0 || p.group > 16) return false;
     if (p.block_size != stc::kBN || p.ksel > stc::kMaxSel || 128 % p.group != 0) return false;
     const int P = stc::kBM / p.group;
     if (stc::kNQ * P * p.ksel > stc::kMaxUnion) return false;  // the union always fits

@@ -26,7 +26,7 @@ HS_WS_FULL, HS_WS_SPARSE, HS_WS_DECODE_FULL, HS_WS_DECODE_SPARSE = 0, 1, 2, 3
 
 EXPORTS = ("hs_full_attn_index", "hs_sparse_attn_reuse", "hs_decode_step", "hs_workspace_size",
            "hs_device_status", "hs_status_string", "hs_launch_count", "hs_decode_sparse_noalloc",
-           "hs_set_wait_limit")
+           "hs_set_wait_limit", "hs_sparse_attn_reuse_paged", "hs_decode_step_paged")
 
 
 class HsError(RuntimeError):
@@ -45,6 +45,16 @@ class hs_params(ctypes.Structure):
     @property
     def ksel(self) -> int:
         return self.k // self.block_size if self.mode == HS_SEL_BLOCK else self.k
+
+
+class hs_pages(ctypes.Structure):
+    _fields_ = [("block_table", ctypes.c_void_p), ("page_size", ctypes.c_int32),
+                ("max_pages", ctypes.c_int32), ("n_pages", ctypes.c_int32)]
+
+
+def make_pages(block_table, page_size, n_pages) -> hs_pages:
+    """hs_pages for a [batch][max_pages] int32 device block table."""
+    return hs_pages(_ptr(block_table), int(page_size), int(block_table.shape[-1]), int(n_pages))
 
 
 def make_params(batch, hq, hkv, head_dim, t_q, t_kv, q_offset=0, dtype="bf16", mode="block",
@@ -78,6 +88,9 @@ def load(path: str = LIB_PATH):
     lib.hs_workspace_size.restype = S
     lib.hs_device_status.argtypes = [P, ctypes.POINTER(I32)]
     lib.hs_set_wait_limit.argtypes = [ctypes.c_int64]
+    PG = ctypes.POINTER(hs_pages)
+    lib.hs_sparse_attn_reuse_paged.argtypes = [PP, PG, P, P, P, P, P, P, P, P]
+    lib.hs_decode_step_paged.argtypes = [PP, PG, I32, P, P, P, P, P, P, P, P, P, P, S, P]
     lib.hs_status_string.argtypes = [I32]
     lib.hs_status_string.restype = ctypes.c_char_p
     lib.hs_launch_count.argtypes = []
@@ -162,6 +175,24 @@ def hs_decode_step(p, kind, q, k_cache, v_cache, seq_len, idx, idx_count, o, lse
     _check(lib.hs_decode_step(ctypes.byref(p), int(kind), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                               _ptr(seq_len), _ptr(idx), _ptr(idx_count), _ptr(o), _ptr(lse),
                               _ptr(sel_scores), wp, wb, _stream(stream)), "hs_decode_step")
+
+
+def hs_sparse_attn_reuse_paged(p, pages, q_sparse, k_pool, v_pool, idx, idx_count, o_global,
+                               lse_global, stream=None):
+    _check(load().hs_sparse_attn_reuse_paged(ctypes.byref(p), ctypes.byref(pages),
+                                             _ptr(q_sparse), _ptr(k_pool), _ptr(v_pool),
+                                             _ptr(idx), _ptr(idx_count), _ptr(o_global),
+                                             _ptr(lse_global), _stream(stream)),
+           "hs_sparse_attn_reuse_paged")
+
+
+def hs_decode_step_paged(p, pages, kind, q, k_pool, v_pool, seq_len, idx, idx_count, o,
+                         lse=None, sel_scores=None, workspace=None, stream=None):
+    wp, wb = _ws(workspace)
+    _check(load().hs_decode_step_paged(ctypes.byref(p), ctypes.byref(pages), int(kind), _ptr(q),
+                                       _ptr(k_pool), _ptr(v_pool), _ptr(seq_len), _ptr(idx),
+                                       _ptr(idx_count), _ptr(o), _ptr(lse), _ptr(sel_scores), wp,
+                                       wb, _stream(stream)), "hs_decode_step_paged")
 
 
 def hs_decode_sparse_noalloc(p, q, k_cache, v_cache, seq_len, idx, idx_count, o, lse=None,

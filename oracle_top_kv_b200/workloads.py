@@ -194,3 +194,29 @@ def decode_seq_lens(w: Workload, ragged: bool = False, device="cpu") -> torch.Te
     lens = torch.randint(w.t // 2, w.t + 1, (w.batch,), generator=gen, dtype=torch.int32)
     lens[0] = w.t
     return lens.to(device)
+
+
+def paged_pool(k: torch.Tensor, v: torch.Tensor, page_size: int, seed: int = 0,
+               extra_pages: int = 3):
+    """Scatter contiguous K, V [b, hkv, T, d] into page pools.
+
+    Pools are [n_pages, hkv, page_size, d]; the block table [b, ceil(T/ps)]
+    int32 maps logical page i of sequence b to a physical page drawn from a
+    seeded permutation, so consecutive logical pages land anywhere in the pool.
+    Unused pages (extra_pages of them, and the tail of a last partial page)
+    hold noise that a correct reader never sees.  Pure data movement.
+    """
+    b, hkv, T, d = k.shape
+    mp = -(-T // page_size)
+    n_pages = b * mp + extra_pages
+    gen = torch.Generator().manual_seed(7919 + seed)
+    perm = torch.randperm(n_pages, generator=gen)[: b * mp].view(b, mp)
+    kp = (torch.randn(n_pages, hkv, page_size, d, generator=gen) * 0.5).to(k.dtype)
+    vp = (torch.randn(n_pages, hkv, page_size, d, generator=gen) * 0.5).to(v.dtype)
+    kc, vc = k.cpu(), v.cpu()
+    for bb in range(b):
+        for lp in range(mp):
+            n = min(page_size, T - lp * page_size)
+            kp[perm[bb, lp], :, :n] = kc[bb, :, lp * page_size: lp * page_size + n]
+            vp[perm[bb, lp], :, :n] = vc[bb, :, lp * page_size: lp * page_size + n]
+    return kp.to(k.device), vp.to(v.device), perm.to(torch.int32).to(k.device)

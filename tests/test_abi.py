@@ -65,7 +65,8 @@ def _full(p, **ptrs):
     (dict(block_size=8, k=1024), hs.HS_ERR_UNSUPPORTED),  # B not in {16..128}
     (dict(k=8192), hs.HS_ERR_UNSUPPORTED),            # k/B > 64
     (dict(head_dim=96), hs.HS_ERR_UNSUPPORTED),
-    (dict(hq=64, hkv=2), hs.HS_ERR_UNSUPPORTED),      # group of 32 heads
+    (dict(hq=128, hkv=1), hs.HS_ERR_UNSUPPORTED),     # group of 128 heads
+    (dict(head_dim=512), hs.HS_ERR_UNSUPPORTED),
     (dict(q_offset=1), hs.HS_ERR_INVALID_ARG),        # rows beyond t_kv
     (dict(mode="token", window=2000, k=1024), hs.HS_ERR_INVALID_ARG),  # w > k
     (dict(mode="token", k=8192, window=128), hs.HS_ERR_UNSUPPORTED),
@@ -138,3 +139,36 @@ def test_gate_sink_argument_checks(lib):
     assert _gate_sink(p, z_g=FAKE + 4) == bad
     assert _gate_sink(_p(head_dim=96)) == hs.HS_ERR_UNSUPPORTED
     assert _gate_sink(_p(t_q=0, t_kv=4)) == hs.HS_OK       # nothing to do, nothing launched
+
+
+def test_paged_entry_points_check_the_table(lib):
+    p = _p(mode="token", block_size=1, t_kv=1024)
+    ok = hs.hs_pages(FAKE, 16, 64, 10)
+    for bad in (hs.hs_pages(None, 16, 64, 10), hs.hs_pages(FAKE, 0, 64, 10),
+                hs.hs_pages(FAKE, 16, 63, 10), hs.hs_pages(FAKE, 16, 64, 0),
+                hs.hs_pages(FAKE, 16, 64, 1 << 27)):
+        assert lib.hs_sparse_attn_reuse_paged(ctypes.byref(p), ctypes.byref(bad), FAKE, FAKE,
+                                              FAKE, FAKE, FAKE, FAKE, FAKE, None) == \
+            hs.HS_ERR_INVALID_ARG
+    assert lib.hs_sparse_attn_reuse_paged(ctypes.byref(p), None, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                          FAKE, FAKE, None) == hs.HS_ERR_INVALID_ARG
+    pf = _p(mode="token", block_size=1, t_kv=1024, dtype="fp32")
+    assert lib.hs_sparse_attn_reuse_paged(ctypes.byref(pf), ctypes.byref(ok), FAKE, FAKE, FAKE,
+                                          FAKE, FAKE, FAKE, FAKE, None) == hs.HS_ERR_UNSUPPORTED
+    pd = _p(mode="token", block_size=1, t_kv=1024, t_q=1)
+    assert lib.hs_decode_step_paged(ctypes.byref(pd), ctypes.byref(ok), 0, FAKE, FAKE, FAKE,
+                                    FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 0, None) == \
+        hs.HS_ERR_WORKSPACE
+
+
+def test_wide_groups_and_head_dim_256_take_no_decode_workspace(lib):
+    p = _p(hq=64, hkv=1, head_dim=256, t_q=1, t_kv=4096, mode="token", block_size=1)
+    assert hs.hs_workspace_size(p, hs.HS_WS_DECODE_FULL) == 0
+    p = _p(hq=64, hkv=1, head_dim=256, t_q=1, t_kv=4096, mode="token", block_size=1)
+    pages = hs.hs_pages(FAKE, 16, 256, 10)
+    # paged and allocation-free entry points: groups of <= 16 heads, d <= 128
+    assert lib.hs_decode_step_paged(ctypes.byref(p), ctypes.byref(pages), 1, FAKE, FAKE, FAKE,
+                                    FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 0, None) == \
+        hs.HS_ERR_UNSUPPORTED
+    assert lib.hs_decode_sparse_noalloc(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                        FAKE, None, None) == hs.HS_ERR_UNSUPPORTED

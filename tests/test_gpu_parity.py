@@ -144,6 +144,17 @@ SMALL = {
     "bf16_token_long_scan": wl.scaled(wl.WORKLOADS["long_1m_chunk"], name="bf16_token_long_scan",
                                       hq=16, hkv=1, t=266240, t_q=40, q_offset=266200, k=1024,
                                       window=128, needles="loguniform:16"),
+    # HySparse2's MQA 64/1 at head dim 256 (SIMT kernels), and 64/1 at d = 128
+    # (tensor-core attention pass, SIMT selection); a 32-head block-mode group
+    # at d = 256 with the window branch
+    "bf16_token_mqa64_d256": wl.scaled(wl.WORKLOADS["hysparse2_prefill"],
+                                       name="bf16_token_mqa64_d256", hq=64, hkv=1, head_dim=256,
+                                       t=600, k=256, window=64),
+    "bf16_token_mqa64_d128": wl.scaled(wl.WORKLOADS["hysparse2_prefill"],
+                                       name="bf16_token_mqa64_d128", hq=64, hkv=1, t=700, k=256,
+                                       window=64),
+    "bf16_block_g32_d256": wl.scaled(wl.WORKLOADS["hysparse_7b_block"], name="bf16_block_g32_d256",
+                                     batch=1, hq=32, hkv=1, head_dim=256, t=400, k=256, window=64),
     "bf16_select_all": wl.scaled(wl.WORKLOADS["hysparse2_prefill"], name="bf16_select_all",
                                  hq=4, hkv=2, t=100, k=128, window=16),
     "bf16_single_token": wl.scaled(wl.WORKLOADS["hysparse2_prefill"], name="bf16_single_token",
@@ -327,6 +338,13 @@ def test_decode_small_g4_d64():
     w = wl.scaled(wl.WORKLOADS["hysparse2_decode"], name="decode_g4", batch=2, hq=8, hkv=2,
                   head_dim=64, t=3000, k=100, window=10)
     run_decode(w, torch.tensor([2999, 3000], dtype=torch.int32))
+
+
+def test_decode_mqa64_d256():
+    """HySparse2's MQA 64/1 at head dim 256 (SIMT decode kernels)."""
+    w = wl.scaled(wl.WORKLOADS["hysparse2_decode"], name="decode_mqa64_d256", batch=3, hq=64,
+                  hkv=1, head_dim=256, t=2500, k=256, window=64)
+    run_decode(w, torch.tensor([2500, 1, 1300], dtype=torch.int32))
 
 
 def test_decode_bad_length_sets_status():

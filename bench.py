@@ -187,7 +187,14 @@ class DecodeBlock:
         q, kc, vc, _ = wl.full_layer_inputs(w, device=device)
         self.q, self.k, self.v = q, kc, vc
         self.seq = wl.decode_seq_lens(w, ragged=False, device=device)
-        self.p = hs.make_params(w.batch, w.hq, w.hkv, w.head_dim, 1, w.t, 0, w.dtype, w.mode,
+        t_kv = w.t
+        self.pages = None
+        if w.page_size:  # the cache as a pool of pages with a shuffled block table
+            self.k, self.v, self.bt = wl.paged_pool(kc, vc, w.page_size)
+            del kc, vc
+            self.pages = hs.make_pages(self.bt, w.page_size, self.k.shape[0])
+            t_kv = self.bt.shape[1] * w.page_size
+        self.p = hs.make_params(w.batch, w.hq, w.hkv, w.head_dim, 1, t_kv, 0, w.dtype, w.mode,
                                 w.block_size, w.k, w.window)
         ks = self.p.ksel
         self.idx = torch.empty(w.batch, w.hkv, ks, dtype=torch.int32, device=device)
@@ -202,11 +209,22 @@ class DecodeBlock:
                    for _ in self.qs]
 
     def full(self, stream):
+        if self.pages is not None:
+            self.hs.hs_decode_step_paged(self.p, self.pages, self.hs.HS_DECODE_FULL_INDEX, self.q,
+                                         self.k, self.v, self.seq, self.idx, self.cnt, self.o,
+                                         self.lse, None, self.ws_full, stream)
+            return
         self.hs.hs_decode_step(self.p, self.hs.HS_DECODE_FULL_INDEX, self.q, self.k, self.v,
                                self.seq, self.idx, self.cnt, self.o, self.lse, None, self.ws_full,
                                stream)
 
     def sparse(self, layer, stream):
+        if self.pages is not None:
+            self.hs.hs_decode_step_paged(self.p, self.pages, self.hs.HS_DECODE_SPARSE,
+                                         self.qs[layer], self.k, self.v, self.seq, self.idx,
+                                         self.cnt, self.os[layer], self.ls[layer], None, None,
+                                         stream)
+            return
         self.hs.hs_decode_step(self.p, self.hs.HS_DECODE_SPARSE, self.qs[layer], self.k, self.v,
                                self.seq, self.idx, self.cnt, self.os[layer], self.ls[layer], None,
                                self.ws_sp, stream)
@@ -286,6 +304,9 @@ def workload_of(args):
         kw["batch"] = args.batch
     if args.seq:
         kw["t"] = args.seq
+    if args.tq:  # a shorter query chunk at the end of the same prefix
+        kw["t_q"] = args.tq
+        kw["q_offset"] = (args.seq or w.t) - args.tq
     if kw:
         w = wl.scaled(w, name=w.name + "".join(f"_{k}{v}" for k, v in kw.items()), **kw)
     return w
@@ -322,7 +343,8 @@ def config_of(w, world, launch):
             "hkv": w.hkv, "head_dim": w.head_dim, "mode": w.mode,
             "block_size": w.block_size, "k": w.k, "window": w.window,
             "decode": w.decode, "t_q": w.tq, "q_offset": w.q_offset,
-            "sparse_layers": w.n_sparse, "parallelism": f"replicas{world}",
+            "sparse_layers": w.n_sparse, "page_size": w.page_size or None,
+            "parallelism": f"replicas{world}",
             "l2": "inputs larger than L2 (K^F+V^F alone exceed 126 MB)",
             "launch": launch}
 
@@ -773,6 +795,8 @@ def main():
     ap.add_argument("--workload", default="long_1m_chunk", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--batch", type=int, default=0, help="override the batch (reduced replica)")
     ap.add_argument("--seq", type=int, default=0, help="override the sequence length")
+    ap.add_argument("--tq", type=int, default=0,
+                    help="prefill: only the last TQ query rows of the sequence (reduced replica)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="time per-call launches instead of CUDA graph replays")

@@ -47,6 +47,7 @@ class Workload:
     t_q: int = 0           # query rows (0: = t);  chunked prefill uses fewer
     q_offset: int = 0
     config_id: int = 0
+    page_size: int = 0     # > 0: the K^F/V^F cache is paged (decode workloads)
     extra: dict = field(default_factory=dict)
 
     @property
@@ -94,6 +95,19 @@ WORKLOADS = {
     "long_1m_decode": Workload("long_1m_decode", 1, 64, 4, 128, 1 << 20, "bf16", "token", 1,
                                1024, 128, 11, False, _S128, 8.0 / _S128, "loguniform:64",
                                decode=True, config_id=5),
+    # The HySparse2 decode case over a paged cache: 64-token pages, shuffled
+    # block table ("HySparse 混合稀疏注意力（一）", 工程实现中的关键约束 item 2).
+    "hysparse2_decode_paged": Workload("hysparse2_decode_paged", 32, 64, 4, 128, 131072, "bf16",
+                                       "token", 1, 1024, 128, 11, False, _S128, 8.0 / _S128,
+                                       "decode:16", decode=True, config_id=4, page_size=64),
+    # HySparse2's MQA 64/1 at head dim 256 ("HySparse2 ...", 6.4): a prefill
+    # and a decode case at reduced lengths (CUDA-core kernels).
+    "mqa64_d256_prefill": Workload("mqa64_d256_prefill", 1, 64, 1, 256, 8192, "bf16", "token",
+                                   1, 1024, 128, 11, False, 1.0 / 16.0, 8.0 * 16.0, "frac:0.01",
+                                   config_id=6),
+    "mqa64_d256_decode": Workload("mqa64_d256_decode", 8, 64, 1, 256, 32768, "bf16", "token", 1,
+                                  1024, 128, 11, False, 1.0 / 16.0, 8.0 * 16.0, "decode:16",
+                                  decode=True, config_id=7),
 }
 
 
@@ -209,14 +223,24 @@ def paged_pool(k: torch.Tensor, v: torch.Tensor, page_size: int, seed: int = 0,
     b, hkv, T, d = k.shape
     mp = -(-T // page_size)
     n_pages = b * mp + extra_pages
+    dev = k.device
     gen = torch.Generator().manual_seed(7919 + seed)
     perm = torch.randperm(n_pages, generator=gen)[: b * mp].view(b, mp)
-    kp = (torch.randn(n_pages, hkv, page_size, d, generator=gen) * 0.5).to(k.dtype)
-    vp = (torch.randn(n_pages, hkv, page_size, d, generator=gen) * 0.5).to(v.dtype)
-    kc, vc = k.cpu(), v.cpu()
-    for bb in range(b):
-        for lp in range(mp):
-            n = min(page_size, T - lp * page_size)
-            kp[perm[bb, lp], :, :n] = kc[bb, :, lp * page_size: lp * page_size + n]
-            vp[perm[bb, lp], :, :n] = vc[bb, :, lp * page_size: lp * page_size + n]
-    return kp.to(k.device), vp.to(v.device), perm.to(torch.int32).to(k.device)
+    noise = torch.Generator(device=dev).manual_seed(104729 + seed)
+    kp = (torch.randn(n_pages, hkv, page_size, d, generator=noise, device=dev) * 0.5).to(k.dtype)
+    vp = (torch.randn(n_pages, hkv, page_size, d, generator=noise, device=dev) * 0.5).to(v.dtype)
+    pad = mp * page_size - T
+    for pool, src in ((kp, k), (vp, v)):
+        x = torch.nn.functional.pad(src, (0, 0, 0, pad)) if pad else src
+        # [b, hkv, mp, ps, d] -> one [hkv, ps, d] page per (b, logical page)
+        pages = x.reshape(b, hkv, mp, page_size, d).permute(0, 2, 1, 3, 4).reshape(b * mp, hkv,
+                                                                                 page_size, d)
+        if pad:  # the tail of a last partial page keeps its noise
+            keep = pool[perm[:, -1].to(dev)].clone()
+            pool[perm.reshape(-1).to(dev)] = pages
+            tail = pool[perm[:, -1].to(dev)]
+            tail[:, :, page_size - pad:] = keep[:, :, page_size - pad:]
+            pool[perm[:, -1].to(dev)] = tail
+        else:
+            pool[perm.reshape(-1).to(dev)] = pages
+    return kp, vp, perm.to(torch.int32).to(dev)

@@ -294,6 +294,19 @@ hs_status hs_decode_step_paged(const hs_params* p, const hs_pages* pages, int32_
  * bound of a few hundred cycles to make waits run out on purpose. */
 hs_status hs_set_wait_limit(int64_t cycles);
 
+/* Token-selection tuning (HySparse2 token mode, hs_full_attn_index with a
+ * workspace; the selection itself is unchanged).  Before a long scan the
+ * selector scores 2048 keys spread evenly over the range every position of a
+ * work item ranks and starts from the rank-th best of them as its admission
+ * threshold, so far fewer keys enter its candidate buffers.  If fewer than
+ * k - w keys of a position pass that threshold (the threshold was too high,
+ * which the automatic rank makes a below-1e-5 event) the work item is scanned
+ * again without one, so the result never depends on this setting.
+ * rank < 0: automatic (the default; a rank from the sample density), 0: off,
+ * rank > 0: always that rank (tests use 1 to force the rescan).  Applies to
+ * kernels launched afterwards on the current device; synchronous. */
+hs_status hs_set_select_sampling(int32_t rank);
+
 #ifdef __cplusplus
 }
 #endif

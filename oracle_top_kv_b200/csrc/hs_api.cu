@@ -392,6 +392,12 @@ hs_status hs_set_wait_limit(int64_t cycles) {
                                                                                : HS_ERR_CUDA;
 }
 
+hs_status hs_set_select_sampling(int32_t rank) {
+    const int v = rank < 0 ? -1 : (int)rank;
+    return cudaMemcpyToSymbol(hs::g_sel_sample, &v, sizeof(v)) == cudaSuccess ? HS_OK
+                                                                               : HS_ERR_CUDA;
+}
+
 const char* hs_status_string(int32_t status) {
     switch (status) {
         case HS_OK: return "HS_OK";

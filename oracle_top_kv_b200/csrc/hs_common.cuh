@@ -25,6 +25,27 @@ __device__ __forceinline__ void set_status(int code) { atomicCAS(&g_status, 0, c
 // host sets it through hs_set_wait_limit, a failure-detection diagnostic).
 __device__ long long g_wait_limit = 2000000000ll;
 
+// Sampled start threshold of the token selectors (per device; set by the
+// host through hs_set_select_sampling): -1 = rank chosen from the sample
+// density, 0 = off, r > 0 = always the r-th best sampled score.
+__device__ int g_sel_sample = -1;
+
+// Rank, among `n_samples` keys drawn evenly from `range_keys` keys, of the
+// sampled score a selector may start from as its admission threshold when it
+// ranks the best `kc` keys of at least those `range_keys`.  The number of
+// samples that fall among the true best kc is about Poisson(lambda), lambda =
+// kc * n_samples / range_keys; the threshold is too high only if at least r of
+// them do, so r = lambda + 4.3 sqrt(lambda) + 3 keeps that below 1e-5 (the
+// selector then detects it and rescans without a threshold).  0 = do not
+// sample (off, or samples too dense to save admissions).
+__device__ __forceinline__ int sample_rank(int kc, int n_samples, long long range_keys) {
+    const int mode = g_sel_sample;
+    if (mode >= 0) return mode < n_samples ? mode : 0;
+    const float lam = (float)kc * (float)n_samples / (float)range_keys;
+    if (!(lam <= 200.f)) return 0;
+    return (int)ceilf(lam + 4.3f * sqrtf(lam) + 3.f);
+}
+
 // ---------------------------------------------------------------- element I/O
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }

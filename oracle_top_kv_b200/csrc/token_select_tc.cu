@@ -75,9 +75,13 @@ struct Cfg {
     static constexpr uint32_t kBarOff = kHistOff + kPos * 1024;
     enum { BQ = 0, BKF = 1, BKE = BKF + kStages, BSF = BKE + kStages, BSE = BSF + kSBufs,
            BDRAIN = BSE + kSBufs, BCOUNT = BDRAIN + 1 };
-    // tmem slot (4) | abort (4) | count[kPos] (32) | threshold key[kPos] (64)
+    // tmem slot (4) | abort (4) | count[kPos] (32) | threshold key[kPos] (64) | rescan (4)
     static constexpr uint32_t kMiscOff = kBarOff + BCOUNT * 8;
-    static constexpr uint32_t kSmemBytes = kMiscOff + 8 + 4 * kPos + 8 * kPos + 1024;
+    static constexpr uint32_t kFailOff = kMiscOff + 8 + 4 * kPos + 8 * kPos;
+    static constexpr uint32_t kSmemBytes = kFailOff + 16 + 1024;
+    // sampled tiles: an even count fills most of a buffer (the sampled
+    // threshold is taken at a check, which falls on odd tiles)
+    static constexpr int kSampleTiles = (kCap / kKeys) / kCheck * kCheck;
     static_assert(kSmemBytes <= 232448, "shared memory");
     static_assert(kStages * 32768 >= kPos * kMaxRanked * 8, "sort scratch fits in the K ring");
     static_assert(kStages * 32768 >= kPos * (kBitmapKeys / 8), "id bitmaps fit in the K ring");
@@ -122,10 +126,21 @@ __device__ __forceinline__ float group_max16(const uint32_t* r, float sl2, const
                  max3f(max3f(v[9], v[10], v[11]), max3f(v[12], v[13], v[14]), v[15]));
 }
 
+// Key tile that pipeline step j of a sampled pass loads: the first
+// kSampleTiles steps visit tiles spread evenly over 0 .. n_rt-1.
 template <class C>
-__global__ void __launch_bounds__(C::kThreads, 1)
-    token_select_kernel(const __grid_constant__ CUtensorMap tmap_q,
-                        const __grid_constant__ CUtensorMap tmap_k, Args a) {
+__device__ __forceinline__ int sample_tile(int j, int n_rt) {
+    return ((2 * j + 1) * n_rt) / (2 * C::kSampleTiles);
+}
+
+// One scan of the CTA's key tiles and the finalize.  kSampled: the first
+// kSampleTiles pipeline steps score sampled tiles straight into the buffers
+// and set each position's threshold to the rank-th best sample; the
+// finalize then flags (*s_fail) a position that saw fewer than k - w keys
+// pass it.  reinit: the barriers of an earlier pass are invalidated first.
+template <class C, bool kSampled>
+__device__ __forceinline__ void select_pass(const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,
+                                            const Args& a, int rank, int n_rt, bool reinit) {
     constexpr int kStages = C::kStagesN, kCap = C::kCapN, kPP = C::kPP;
     constexpr int kSets = C::kSets, kScorers = C::kScorers;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -150,19 +165,21 @@ __global__ void __launch_bounds__(C::kThreads, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + C::kMiscOff + 4);
     int* s_cnt = reinterpret_cast<int*>(gb + C::kMiscOff + 8);
     unsigned long long* s_th = reinterpret_cast<unsigned long long*>(gb + C::kMiscOff + 8 + 4 * kPos);
+    volatile int* s_fail = reinterpret_cast<volatile int*>(gb + C::kFailOff);
+    constexpr int ns = kSampled ? C::kSampleTiles : 0;  // sampled pipeline steps
+    (void)s_fail;
+    (void)rank;
 
     if (threadIdx.x == 0) {
+        if (reinit)
+            for (int i = 0; i < C::BCOUNT; ++i)
+                asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(bar(i)) : "memory");
         mbar_init(bar(C::BQ), 1);
         for (int i = 0; i < kStages; ++i) { mbar_init(bar(C::BKF + i), 1); mbar_init(bar(C::BKE + i), 1); }
         for (int i = 0; i < kSBufs; ++i) { mbar_init(bar(C::BSF + i), 1); mbar_init(bar(C::BSE + i), kScorers); }
         mbar_init(bar(C::BDRAIN), 1);
-        *abort_flag = 0;
         for (int i = 0; i < kPos; ++i) { s_cnt[i] = 0; s_th[i] = 0ull; }
         fence_mbar_init();
-    }
-    if (warp == 1) {
-        tmem_alloc(base + C::kMiscOff, kTmemCols);
-        tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
@@ -171,13 +188,12 @@ __global__ void __launch_bounds__(C::kThreads, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            prefetch_tmap(&tmap_q);
-            prefetch_tmap(&tmap_k);
+            if (!reinit) { prefetch_tmap(&tmap_q); prefetch_tmap(&tmap_k); }
             mbar_arrive_expect_tx(bar(C::BQ), 32768);
             tma_load_4d(base + C::kQOff, &tmap_q, bar(C::BQ), 0, u * kG, row0, b);
             tma_load_4d(base + C::kQOff + 16384, &tmap_q, bar(C::BQ), 64, u * kG, row0, b);
             int issued = 0;
-            for (int j = 0; j < nt; ++j) {
+            for (int j = 0; j < ns + nt; ++j) {
                 const int st = j % kStages;
                 if (j >= kStages &&
                     !mbar_wait(bar(C::BKE + st), ((j / kStages) - 1) & 1, abort_flag))
@@ -185,8 +201,9 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                 const uint32_t f = bar(C::BKF + st);
                 mbar_arrive_expect_tx(f, 32768);
                 const uint32_t kd = base + C::kKOff + st * 32768;
-                tma_load_3d(kd, &tmap_k, f, 0, j * kKeys, bu);
-                tma_load_3d(kd + 16384, &tmap_k, f, 64, j * kKeys, bu);
+                const int key0 = (kSampled && j < ns ? sample_tile<C>(j, n_rt) : j - ns) * kKeys;
+                tma_load_3d(kd, &tmap_k, f, 0, key0, bu);
+                tma_load_3d(kd + 16384, &tmap_k, f, 64, key0, bu);
                 issued = j + 1;
             }
             drain(bar(C::BQ), 0);
@@ -202,7 +219,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             const uint64_t dq = sw128_desc(base + C::kQOff, 16, 1024);
             bool ok = mbar_wait(bar(C::BQ), 0, abort_flag);
             tc_fence_after();
-            for (int j = 0; ok && j < nt; ++j) {
+            for (int j = 0; ok && j < ns + nt; ++j) {
                 const int st = j % kStages, s = j % kSBufs;
                 if (!mbar_wait(bar(C::BKF + st), (j / kStages) & 1, abort_flag)) break;
                 if (j >= kSBufs &&
@@ -263,9 +280,10 @@ __global__ void __launch_bounds__(C::kThreads, 1)
         for (int i = 0; i < kPP; ++i) thf[i] = -INFINITY;
         const uint32_t lt_mask = (1u << lane) - 1u;
         bool ok = true;
-        // Every warp runs every iteration (the set meets at named barriers);
-        // after an abort the waits fail at once and the work is skipped.
-        for (int j = 0; j < nt; ++j) {
+        // Pipeline step j scores key tile key0 (a sampled tile while sample).
+        // Every warp runs every step (the set meets at named barriers); after
+        // an abort the waits fail at once and the work is skipped.
+        auto step = [&](const int j, const int key0, const bool sample) {
             const int s = j % kSBufs;
             bool got = ok && mbar_wait(bar(C::BSF + s), (j / kSBufs) & 1, abort_flag);
             got = __all_sync(0xffffffffu, got);
@@ -280,7 +298,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(C::BSE + s));
-                const int key = j * kKeys + quad * 32 + lane;
+                const int key = key0 + quad * 32 + lane;
                 float sc[kPP];
                 bool any = false;
 #pragma unroll
@@ -305,7 +323,7 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                         }
                     }
                 }
-                if (a.sel) {
+                if (!sample && a.sel) {
                     // scores of the keys selected without ranking (tests ask for them)
 #pragma unroll
                     for (int i = 0; i < kPP; ++i) {
@@ -323,7 +341,19 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             if (j % kCheck == kCheck - 1) {
                 asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
                 const int n = s_cnt[my_pos];
-                if (ok && cutter && n > kCap - kCheck * kKeys) {
+                if (sample) {
+                    if (j == ns - 1 && cutter) {
+                        // the samples are in: start from the rank-th best of
+                        // them and empty the buffer (the scan proper sees
+                        // them again)
+                        const uint64_t th = (ok && n >= rank)
+                            ? warp_kth_largest(bufs + (size_t)my_pos * kCap, n, rank, hist) : 0ull;
+                        if (lane == 0) {
+                            s_th[my_pos] = th ? th - 1ull : 0ull;
+                            s_cnt[my_pos] = 0;
+                        }
+                    }
+                } else if (ok && cutter && n > kCap - kCheck * kKeys) {
                     // keep at most halfway between k - w and the trigger
                     const int target = Kc + (kCap - kCheck * kKeys - Kc) / 2;
                     uint64_t th;
@@ -344,7 +374,10 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                     thf[i] = (th == 0ull || x != x) ? -INFINITY : x;
                 }
             }
-        }
+        };
+        if constexpr (kSampled)
+            for (int j = 0; j < ns; ++j) step(j, sample_tile<C>(j, n_rt) * kKeys, true);
+        for (int jj = 0; jj < nt; ++jj) step(jj + ns, jj * kKeys, false);
         // ---- finalize: one warp per position (K stages are free: all MMAs done)
         asm volatile("bar.sync %0, %1;" ::"r"(1 + kSets), "r"(32 * kScorers) : "memory");
         const int pos = wid;
@@ -362,6 +395,11 @@ __global__ void __launch_bounds__(C::kThreads, 1)
                 uint64_t* buf = bufs + (size_t)pos * kCap;
                 int n = Kc > 0 ? min(s_cnt[pos], kCap) : 0;
                 uint32_t* fhist = reinterpret_cast<uint32_t*>(gb + C::kHistOff + pos * 1024);
+                // Every key above the threshold was admitted; with a sampled
+                // start the k-w best are all among them only if at least k-w
+                // of the buffer's keys reach it -- otherwise the CTA rescans.
+                if (kSampled && warp_count_at_least(buf, n, s_th[pos]) < Kc && lane == 0)
+                    *s_fail = 1;
                 if (n > Kc) { warp_cut_to_k(buf, n, Kc, fhist); n = Kc; }
                 __syncwarp();
                 if (!srow && t < kBitmapKeys) {
@@ -418,13 +456,56 @@ __global__ void __launch_bounds__(C::kThreads, 1)
             if (lane == 0) a.cnt[orow] = n_out;
         }
     }
+    tc_fence_before();
+    __syncthreads();  // the pass is done: every wait, load and MMA has drained
+    tc_fence_after();
+}
+
+// One CTA = kPos positions of one (batch, KV group).  A scan whose ranked
+// range is long enough starts from a sampled threshold: kSampleTiles key
+// tiles spread evenly over the n_rt tiles that every position of the CTA
+// ranks are scored first, and the rank-th best of each position's samples
+// becomes its admission threshold (a few thousand admissions and a few cuts
+// per position instead of ~2 (k-w) ln(T/(k-w))).  If the finalize finds a
+// position for which fewer than k-w keys reach it, the CTA scans again
+// without one.
+template <class C>
+__global__ void __launch_bounds__(C::kThreads, 1)
+    token_select_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                        const __grid_constant__ CUtensorMap tmap_k, Args a) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    unsigned char* gb = smem_raw + (base - raw);
+    const int warp = threadIdx.x >> 5;
+    const KParams& p = a.p;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gb + C::kMiscOff);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + C::kMiscOff + 4);
+    volatile int* s_fail = reinterpret_cast<volatile int*>(gb + C::kFailOff);
+    if (threadIdx.x == 0) { *abort_flag = 0; *s_fail = 0; }
+    if (warp == 1) {
+        tmem_alloc(base + C::kMiscOff, kTmemCols);
+        tmem_relinquish();
+    }
+    const int Kc = p.k - p.window;
+    const int row0 = (a.n_ptiles - 1 - (int)(blockIdx.x / (p.batch * p.hkv))) * kPos;
+    const int n_rt = (p.q_offset + row0 - p.window + 1) / kKeys;  // tiles every position ranks
+    const int rank = (Kc > 0 && n_rt >= 8 * C::kSampleTiles)
+                         ? sample_rank(Kc, C::kSampleTiles * kKeys, (long long)n_rt * kKeys)
+                         : 0;
+    bool plain = true;
+    if (rank > 0) {
+        select_pass<C, true>(tmap_q, tmap_k, a, rank, n_rt, false);
+        plain = *s_fail != 0 && *abort_flag == 0;  // read after the pass's barrier
+    }
+    if (plain) select_pass<C, false>(tmap_q, tmap_k, a, 0, n_rt, rank > 0);
 
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(*tmem_slot, kTmemCols);
     }
 }
 

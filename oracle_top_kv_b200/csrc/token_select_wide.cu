@@ -67,6 +67,8 @@ constexpr int kSBufs = 2;
 constexpr int kCheck = 2;
 constexpr int kCap = 2048;       // workspace entries per position
 constexpr int kMaxRanked = 1024;
+constexpr int kSampleTiles = kCap / kKeys;  // sampled tiles fill a buffer exactly
+constexpr int kMinSampleTiles = 64;         // ranked range worth sampling
 constexpr uint32_t kTmemCols = kN * kSBufs;  // 512
 
 constexpr uint32_t kQOff = 0;                          // 2 d halves x 32 KB
@@ -80,10 +82,11 @@ constexpr uint32_t kBarOff = kHistOff + kPos * 1024;
 enum { BQ = 0, BKF = 1, BKE = BKF + kStages, BSF = BKE + kStages, BSE = BSF + kSBufs,
        BDRAIN = BSE + kSBufs, BCOUNT = BDRAIN + 1 };
 // tmem slot (4) | abort (4) | count[kPos] (64) | threshold key[kPos] (128) |
-// admission threshold / scale [kPos] (64, 16-byte aligned)
+// admission threshold / scale [kPos] (64, 16-byte aligned) | rescan (4)
 constexpr uint32_t kMiscOff = kBarOff + BCOUNT * 8;
 constexpr uint32_t kThrOff = (kMiscOff + 8 + 4 * kPos + 8 * kPos + 15) & ~15u;
-constexpr uint32_t kSmemBytes = kThrOff + 4 * kPos + 1024;
+constexpr uint32_t kFailOff = kThrOff + 4 * kPos;
+constexpr uint32_t kSmemBytes = kFailOff + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory");
 static_assert(kKOff + kStages * 32768 >= (uint32_t)kPos * kMaxRanked * 8,
               "finalize sort scratch fits in the Q and K regions");
@@ -115,9 +118,20 @@ __device__ __forceinline__ void mbar_inval(uint32_t bar) {
     asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
-    token_select_wide_kernel(const __grid_constant__ CUtensorMap tmap_q,
-                             const __grid_constant__ CUtensorMap tmap_k, Args a) {
+// Key tile that pipeline step j of a sampled scan loads: the first
+// kSampleTiles steps visit tiles spread evenly over 0 .. n_rt-1.
+__device__ __forceinline__ int sample_tile(int j, int n_rt) {
+    return ((2 * j + 1) * n_rt) / (2 * kSampleTiles);
+}
+
+// One scan of work item `it` and its finalize.  kSampled: the first
+// kSampleTiles pipeline steps score sampled tiles straight into the buffers
+// and set each position's threshold to the rank-th best sample; the
+// finalize then flags (*s_fail = it + 1) a position that saw fewer than
+// k - w keys reach it.  first: the CTA's first scan (no barriers to invalidate yet).
+template <bool kSampled>
+__device__ __forceinline__ void scan_item(const CUtensorMap& tmap_q, const CUtensorMap& tmap_k,
+                                          const Args& a, int it, int rank, int n_rt, bool first) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -133,25 +147,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     int* s_cnt = reinterpret_cast<int*>(gb + kMiscOff + 8);
     unsigned long long* s_th = reinterpret_cast<unsigned long long*>(gb + kMiscOff + 8 + 4 * kPos);
     float* s_thr = reinterpret_cast<float*>(gb + kThrOff);
+    volatile int* s_fail = reinterpret_cast<volatile int*>(gb + kFailOff);
     uint64_t* slot = a.ws + (size_t)blockIdx.x * kPos * kCap;
+    constexpr int ns = kSampled ? kSampleTiles : 0;  // sampled pipeline steps
+    (void)s_fail;
+    (void)rank;
 
-    if (warp == 1) {
-        tmem_alloc(base + kMiscOff, kTmemCols);
-        tmem_relinquish();
-    }
-    if (threadIdx.x == 0) *abort_flag = 0;
-    // zero the extra operand buffer once, then the ones column of the keys
-    // (logical 16-byte chunk 2 of rows 0..127: columns 16..18 = 1.0)
-    for (int x = (int)threadIdx.x; x < kN * 8; x += kThreads)
-        *reinterpret_cast<uint4*>(gb + kXOff + x * 16) = make_uint4(0u, 0u, 0u, 0u);
-    __syncthreads();
-    for (int r = (int)threadIdx.x; r < kKeys; r += kThreads) {
-        const uint32_t one = 0x3f80u;  // bf16 1.0
-        *reinterpret_cast<uint4*>(gb + kXOff + r * 128 + ((2 ^ (r & 7)) << 4)) =
-            make_uint4(one | (one << 16), one, 0u, 0u);
-    }
-
-    for (int it = blockIdx.x; it < a.n_items; it += gridDim.x) {
+    {
         const int pt = a.n_ptiles - 1 - it / bu_n;  // latest positions first
         const int bu = it % bu_n;
         const int b = bu / p.hkv, u = bu % p.hkv;
@@ -161,7 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         // ---- set-up of the item (the previous one has fully drained)
         if (threadIdx.x == 0) {
-            if (it != (int)blockIdx.x)
+            if (!first)
                 for (int i = 0; i < BCOUNT; ++i) mbar_inval(bar(i));
             mbar_init(bar(BQ), 1);
             for (int i = 0; i < kStages; ++i) { mbar_init(bar(BKF + i), 1); mbar_init(bar(BKE + i), 1); }
@@ -192,16 +194,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncthreads();
         tc_fence_after();
         const uint32_t tmem = *tmem_slot;
-        if (*abort_flag) break;  // a wait of an earlier item gave up
+        if (*abort_flag) return;  // a wait of an earlier scan gave up
 
         if (warp == 0) {
             if (lane == 0) {
-                if (it == (int)blockIdx.x) { prefetch_tmap(&tmap_q); prefetch_tmap(&tmap_k); }
+                if (first) { prefetch_tmap(&tmap_q); prefetch_tmap(&tmap_k); }
                 mbar_arrive_expect_tx(bar(BQ), 65536);
                 tma_load_4d(base + kQOff, &tmap_q, bar(BQ), 0, u * kG, row0, b);
                 tma_load_4d(base + kQOff + 32768, &tmap_q, bar(BQ), 64, u * kG, row0, b);
                 int issued = 0;
-                for (int j = 0; j < nt; ++j) {
+                for (int j = 0; j < ns + nt; ++j) {
                     const int st = j % kStages;
                     if (j >= kStages &&
                         !mbar_wait(bar(BKE + st), ((j / kStages) - 1) & 1, abort_flag, false))
@@ -209,8 +211,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t f = bar(BKF + st);
                     mbar_arrive_expect_tx(f, 32768);
                     const uint32_t kd = base + kKOff + st * 32768;
-                    tma_load_3d(kd, &tmap_k, f, 0, j * kKeys, bu);
-                    tma_load_3d(kd + 16384, &tmap_k, f, 64, j * kKeys, bu);
+                    const int key0 = (kSampled && j < ns ? sample_tile(j, n_rt) : j - ns) * kKeys;
+                    tma_load_3d(kd, &tmap_k, f, 0, key0, bu);
+                    tma_load_3d(kd + 16384, &tmap_k, f, 64, key0, bu);
                     issued = j + 1;
                 }
                 drain(bar(BQ), 0);
@@ -225,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t dx = sw128_desc(base + kXOff, 16, 1024);
                 bool ok = mbar_wait(bar(BQ), 0, abort_flag, false);
                 tc_fence_after();
-                for (int j = 0; ok && j < nt; ++j) {
+                for (int j = 0; ok && j < ns + nt; ++j) {
                     const int st = j % kStages, s = j % kSBufs;
                     if (!mbar_wait(bar(BKF + st), (j / kStages) & 1, abort_flag, false)) break;
                     if (j >= kSBufs &&
@@ -281,7 +284,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < kPP; ++i) thr[i] = -INFINITY;
             const uint32_t lt_mask = (1u << lane) - 1u;
             bool ok = true;
-            for (int j = 0; j < nt; ++j) {
+            // pipeline step j scores key tile key0 (a sampled tile while sample)
+            auto step = [&](const int j, const int key0, const bool sample) {
                 const int s = j % kSBufs;
                 bool got = ok && mbar_wait(bar(BSF + s), (j / kSBufs) & 1, abort_flag);
                 got = __all_sync(0xffffffffu, got);
@@ -295,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar(BSE + s));
-                    const int key = j * kKeys + quad * 32 + lane;
+                    const int key = key0 + quad * 32 + lane;
                     float m[kPP];
                     uint32_t cmask = 0u;  // positions with this key as a candidate
 #pragma unroll
@@ -325,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             else set_status(HS_ERR_BOUNDS);  // not reached: the cuts keep room
                         }
                     }
-                    if (a.sel) {
+                    if (!sample && a.sel) {
                         // scores of the keys selected without ranking (tests ask for them)
 #pragma unroll
                         for (int i = 0; i < kPP; ++i) {
@@ -341,7 +345,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (j % kCheck == kCheck - 1) {
                     asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
                     const int n = min(s_cnt[my_pos], kCap);
-                    if (ok && n > kCap - kCheck * kKeys) {
+                    if (sample) {
+                        if (j == ns - 1) {
+                            // the samples are in: start from the rank-th best
+                            // of them and empty the buffer (the scan proper
+                            // sees them again)
+                            const uint64_t th =
+                                (ok && n >= rank) ? warp_kth_largest(my_buf, n, rank, hist) : 0ull;
+                            if (lane == 0) {
+                                s_th[my_pos] = th ? th - 1ull : 0ull;
+                                s_cnt[my_pos] = 0;
+                                const float x = order_float((uint32_t)(th >> 32)) / sl2;
+                                s_thr[my_pos] =
+                                    (th == 0ull || x != x) ? -INFINITY : x - fabsf(x) * 0x1p-20f;
+                            }
+                        }
+                    } else if (ok && n > kCap - kCheck * kKeys) {
                         const int target = Kc + (kCap - kCheck * kKeys - Kc) / 2;
                         uint64_t th;
                         const int mm = warp_cut_sampled(my_buf, n, Kc, n - target, hist, &th);
@@ -357,7 +376,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float4 t4 = *reinterpret_cast<const float4*>(s_thr + set * kPP);
                     thr[0] = t4.x; thr[1] = t4.y; thr[2] = t4.z; thr[3] = t4.w;
                 }
-            }
+            };
+            if constexpr (kSampled)
+                for (int j = 0; j < ns; ++j) step(j, sample_tile(j, n_rt) * kKeys, true);
+            for (int jj = 0; jj < nt; ++jj) step(jj + ns, jj * kKeys, false);
             // ---- finalize: one warp per position; the Q and K regions are free
             asm volatile("bar.sync %0, %1;" ::"r"(1 + kSets), "r"(32 * kScorers) : "memory");
             const int pos = wid;
@@ -375,6 +397,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint64_t* buf = slot + (size_t)pos * kCap;
                     int n = Kc > 0 ? min(s_cnt[pos], kCap) : 0;
                     uint32_t* fhist = reinterpret_cast<uint32_t*>(gb + kHistOff + pos * 1024);
+                    // Every key above the threshold was admitted; with a
+                    // sampled start the k-w best are all among them only if
+                    // at least k-w of the buffer's keys reach it -- otherwise
+                    // the item is scanned again.
+                    if (kSampled && warp_count_at_least(buf, n, s_th[pos]) < Kc && lane == 0)
+                        *s_fail = it + 1;  // tagged with the item: never stale
                     if (n > Kc) { warp_cut_to_k(buf, n, Kc, fhist); n = Kc; }
                     __syncwarp();
                     const int sort_n = next_pow2(Kc > 0 ? Kc : 1);
@@ -399,8 +427,66 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         tc_fence_before();
-        __syncthreads();  // the item is done: every wait, load and MMA has drained
+        __syncthreads();  // the scan is done: every wait, load and MMA has drained
         tc_fence_after();
+    }
+}
+
+// Persistent: CTA c scans work items c, c + gridDim.x, ...  An item whose
+// ranked range is long enough starts from a sampled threshold: kSampleTiles
+// key tiles spread evenly over the n_rt tiles that every position of the
+// item ranks are scored first, and the rank-th best of each position's
+// samples becomes its admission threshold, so the scan admits a few thousand
+// keys per position instead of ~(k-w) ln(T/(k-w)) times two.  If the
+// finalize finds a position for which fewer than k-w keys reach it, the item
+// is scanned again without one.
+__global__ void __launch_bounds__(kThreads, 1)
+    token_select_wide_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                             const __grid_constant__ CUtensorMap tmap_k, Args a) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    unsigned char* gb = smem_raw + (base - raw);
+    const int warp = threadIdx.x >> 5;
+    const KParams& p = a.p;
+    const int Kc = p.k - p.window;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gb + kMiscOff);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(gb + kMiscOff + 4);
+    volatile int* s_fail = reinterpret_cast<volatile int*>(gb + kFailOff);
+
+    if (warp == 1) {
+        tmem_alloc(base + kMiscOff, kTmemCols);
+        tmem_relinquish();
+    }
+    if (threadIdx.x == 0) { *abort_flag = 0; *s_fail = 0; }
+    // zero the extra operand buffer once, then the ones column of the keys
+    // (logical 16-byte chunk 2 of rows 0..127: columns 16..18 = 1.0)
+    for (int x = (int)threadIdx.x; x < kN * 8; x += kThreads)
+        *reinterpret_cast<uint4*>(gb + kXOff + x * 16) = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+    for (int r = (int)threadIdx.x; r < kKeys; r += kThreads) {
+        const uint32_t one = 0x3f80u;  // bf16 1.0
+        *reinterpret_cast<uint4*>(gb + kXOff + r * 128 + ((2 ^ (r & 7)) << 4)) =
+            make_uint4(one | (one << 16), one, 0u, 0u);
+    }
+
+    bool first = true;
+    for (int it = blockIdx.x; it < a.n_items && !*abort_flag; it += gridDim.x) {
+        const int row0 = (a.n_ptiles - 1 - it / (p.batch * p.hkv)) * kPos;
+        const int n_rt = (p.q_offset + row0 - p.window + 1) / kKeys;  // tiles every position ranks
+        const int rank = (Kc > 0 && n_rt >= kMinSampleTiles)
+                             ? sample_rank(Kc, kSampleTiles * kKeys, (long long)n_rt * kKeys)
+                             : 0;
+        bool plain = true;
+        if (rank > 0) {
+            scan_item<true>(tmap_q, tmap_k, a, it, rank, n_rt, first);
+            first = false;
+            plain = *s_fail == it + 1 && *abort_flag == 0;  // read after the scan's barrier
+        }
+        if (plain) {
+            scan_item<false>(tmap_q, tmap_k, a, it, 0, n_rt, first);
+            first = false;
+        }
     }
 
     tc_fence_before();

@@ -26,7 +26,8 @@ HS_WS_FULL, HS_WS_SPARSE, HS_WS_DECODE_FULL, HS_WS_DECODE_SPARSE = 0, 1, 2, 3
 
 EXPORTS = ("hs_full_attn_index", "hs_sparse_attn_reuse", "hs_decode_step", "hs_workspace_size",
            "hs_device_status", "hs_status_string", "hs_launch_count", "hs_decode_sparse_noalloc",
-           "hs_set_wait_limit", "hs_sparse_attn_reuse_paged", "hs_decode_step_paged")
+           "hs_set_wait_limit", "hs_sparse_attn_reuse_paged", "hs_decode_step_paged",
+           "hs_set_select_sampling")
 
 
 class HsError(RuntimeError):
@@ -88,6 +89,7 @@ def load(path: str = LIB_PATH):
     lib.hs_workspace_size.restype = S
     lib.hs_device_status.argtypes = [P, ctypes.POINTER(I32)]
     lib.hs_set_wait_limit.argtypes = [ctypes.c_int64]
+    lib.hs_set_select_sampling.argtypes = [I32]
     PG = ctypes.POINTER(hs_pages)
     lib.hs_sparse_attn_reuse_paged.argtypes = [PP, PG, P, P, P, P, P, P, P, P]
     lib.hs_decode_step_paged.argtypes = [PP, PG, I32, P, P, P, P, P, P, P, P, P, P, S, P]
@@ -220,6 +222,11 @@ def hs_device_status(stream=None) -> int:
 def hs_set_wait_limit(cycles: int) -> None:
     """Bound, in SM cycles, of the kernels' waits (<= 0: the default)."""
     _check(load().hs_set_wait_limit(int(cycles)), "hs_set_wait_limit")
+
+
+def hs_set_select_sampling(rank: int) -> None:
+    """Sampled start threshold of the token selector: -1 automatic, 0 off, r > 0 that rank."""
+    _check(load().hs_set_select_sampling(int(rank)), "hs_set_select_sampling")
 
 
 def hs_status_string(code) -> str:

@@ -27,6 +27,15 @@ CASES = {
 }
 
 
+# Many more work items than SMs (2 groups x 150 items of 16 positions): the
+# persistent wide selector takes several items per CTA, so forced rescans
+# land in the middle of a CTA's item sequence.  Compared across sampling
+# ranks only (the oracle check of the same kernel runs on the cases above).
+MANY_ITEMS = wl.scaled(wl.WORKLOADS["long_1m_chunk"], name="sample_wide_many", hq=32, hkv=2,
+                       t=266240, t_q=2400, q_offset=263840, k=1024, window=128,
+                       needles="loguniform:16")
+
+
 @pytest.fixture(autouse=True)
 def _restore():
     hs.load()
@@ -61,3 +70,25 @@ def test_sampled_threshold_never_changes_the_selection(case):
     orc = P.oracle_full_rows(w, q, k, v, rws, w.q_offset + rws[:, 2])
     P.check_index(P.gpu_rows(ref[0].numpy(), rws, False), P.gpu_rows(ref[1].numpy(), rws, False),
                   orc, w.mode, w.window, w.k, f"{case} index (sampled threshold)")
+
+
+def test_sampled_threshold_many_items_per_cta():
+    w = MANY_ITEMS
+    q, k, v, _ = wl.full_layer_inputs(w, device=DEV)
+    p = P.abi_params(w)
+    ws = hs.workspace(p, hs.HS_WS_FULL)
+    assert ws is not None
+    outs = {}
+    for rank in (-1, 0, 1, 9):
+        hs.hs_set_select_sampling(rank)
+        o, lse, idx, cnt, _ = hs.full_outputs(p)
+        idx.fill_(-7)
+        cnt.fill_(-7)
+        hs.hs_full_attn_index(p, q, k, v, o, lse, idx, cnt, None, ws)
+        torch.cuda.synchronize()
+        assert hs.hs_device_status() == 0, f"rank {rank}"
+        outs[rank] = (idx.cpu(), cnt.cpu())
+    for rank, got in outs.items():
+        assert torch.equal(got[0], outs[0][0]) and torch.equal(got[1], outs[0][1]), \
+            f"index with sampling rank {rank} differs from the unsampled scan"
+    assert int(outs[0][1].min()) == w.k  # every position ranks (t + 1 > k)

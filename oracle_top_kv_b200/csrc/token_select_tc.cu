@@ -14,7 +14,9 @@
 // of its positions in registers: the group max is in-thread packed FMA plus
 // three-input max with the fp32 lse.  Each position keeps an exact streaming
 // top-(k-w) buffer in shared memory (admission threshold = a key at or below
-// the (k-w)-th best seen so far, raised by each cut of the buffer).
+// the (k-w)-th best seen so far, raised by each cut of the buffer; a long scan
+// starts from the rank-th best of a sample of its keys instead of from
+// nothing, see token_select_kernel).
 //
 // What bounds it: per 128-key tile the tensor core reads its operands from
 // shared memory (K 32 KB + Q^T 32 KB over the 8 MMAs) while TMA writes the

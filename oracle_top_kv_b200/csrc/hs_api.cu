@@ -21,6 +21,7 @@
 #include "token_select_wide.cu"
 #include "noalloc.cu"
 #include "sparse.cu"
+#include "decode_simt.cu"
 #include "gate_sink.cu"
 
 namespace hs {
@@ -201,7 +202,10 @@ size_t hs_workspace_size(const hs_params* p, int32_t which) {
     const bool decode = which == HS_WS_DECODE_FULL || which == HS_WS_DECODE_SPARSE;
     if (which < HS_WS_FULL || which > HS_WS_DECODE_SPARSE) return (size_t)-1;
     if (resolve(p, decode, &kp) != HS_OK) return (size_t)-1;
-    if (decode && !mma_shape(kp)) return 0;  // the SIMT decode kernels need none
+    if (decode && !mma_shape(kp))  // wide groups / d = 256: the split-k CUDA-core steps
+        return hs::decode_simt_split_supported(kp)
+                   ? hs::decode_simt_workspace(kp, which == HS_WS_DECODE_FULL)
+                   : 0;
     switch (which) {
         case HS_WS_FULL:
             return hs::full_tc_supported(kp, p->dtype) && hs::token_select_wide_applies(kp, p->dtype)
@@ -225,8 +229,18 @@ hs_status hs_decode_step(const hs_params* p, int32_t kind, const void* q, const 
     if (!ok_ptr(q) || !ok_ptr(k_cache) || !ok_ptr(v_cache) || !ok_ptr(seq_len) || !ok_ptr(idx) ||
         !ok_ptr(idx_count) || !ok_ptr(o) || !ok_opt(lse) || !ok_opt(sel_scores))
         return HS_ERR_INVALID_ARG;
-    if (!mma_shape(kp)) {  // wide groups / d = 256: one SIMT kernel per step, no workspace
+    if (!mma_shape(kp)) {
+        // wide groups / d = 256: split-k CUDA-core kernels with the workspace,
+        // else one CTA per sequence and group (no workspace)
         cudaStream_t st = static_cast<cudaStream_t>(stream);
+        const bool full = kind == HS_DECODE_FULL_INDEX;
+        if (full && !lse) return HS_ERR_INVALID_ARG;
+        if (hs::decode_simt_split_supported(kp) && workspace != nullptr && aligned16(workspace) &&
+            ws_bytes >= hs::decode_simt_workspace(kp, full))
+            return launched(hs::decode_simt_kernel_count(full), [&] {
+                return hs::launch_decode_simt(kp, full, q, k_cache, v_cache, seq_len, idx,
+                                              idx_count, o, lse, sel_scores, workspace, st);
+            });
         if (kind == HS_DECODE_FULL_INDEX) {
             if (!lse) return HS_ERR_INVALID_ARG;
             return launched(1, [&] {

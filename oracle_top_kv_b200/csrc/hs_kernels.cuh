@@ -41,6 +41,17 @@ cudaError_t launch_full_tc(const KParams& p, const void* q, const void* k, const
                            void* o, float* lse, int32_t* idx, int32_t* cnt, float* sel,
                            int capture, cudaStream_t st);
 
+// Split-k decode steps on the CUDA cores for groups of up to 64 heads and
+// head_dim 64/128/256 (contiguous cache): full = full step with the index,
+// else the sparse step.  Needs decode_simt_workspace(p, full) bytes.
+bool decode_simt_split_supported(const KParams& p);
+size_t decode_simt_workspace(const KParams& p, bool full);
+int decode_simt_kernel_count(bool full);
+cudaError_t launch_decode_simt(const KParams& p, bool full, const void* q, const void* kc,
+                               const void* vc, const int32_t* seq_len, int32_t* idx,
+                               int32_t* cnt, void* o, float* lse, float* sel, void* ws,
+                               cudaStream_t st);
+
 // seq_len as for launch_full_simt.  Groups of up to 64 heads, head_dim 64,
 // 128 or 256.
 cudaError_t launch_sparse_simt(const KParams& p, int dtype, const void* q, const void* kf,

@@ -272,7 +272,7 @@ def test_block_sparse_bounds_status():
 
 
 # -------------------------------------------------------------------- decode
-def run_decode(w, seq_len, layers=2, gen_device="cpu", units=None):
+def run_decode(w, seq_len, layers=2, gen_device="cpu", units=None, use_ws=True):
     q, kc, vc, _ = wl.full_layer_inputs(w, device=gen_device)
     q, kc, vc = _cuda(q, kc, vc)
     sl = seq_len.to(DEV).to(torch.int32)
@@ -283,7 +283,7 @@ def run_decode(w, seq_len, layers=2, gen_device="cpu", units=None):
     sel = torch.empty(w.batch, w.hkv, ksel, dtype=torch.float32, device=DEV)
     o = torch.empty_like(q)
     lse = torch.empty(w.batch, w.hq, 1, dtype=torch.float32, device=DEV)
-    ws = hs.workspace(p, hs.HS_WS_DECODE_FULL)
+    ws = hs.workspace(p, hs.HS_WS_DECODE_FULL) if use_ws else None
     hs.hs_decode_step(p, hs.HS_DECODE_FULL_INDEX, q, kc, vc, sl, idx, cnt, o, lse, sel, ws)
     torch.cuda.synchronize()
     assert hs.hs_device_status() == 0
@@ -305,7 +305,7 @@ def run_decode(w, seq_len, layers=2, gen_device="cpu", units=None):
     for n in range(len(g_cnt)):
         ids = g_idx[n, :g_cnt[n]]
         np.testing.assert_allclose(g_sel[n, :g_cnt[n]], orc["scores"][n][ids], rtol=2e-3)
-    wss = hs.workspace(p, hs.HS_WS_DECODE_SPARSE)
+    wss = hs.workspace(p, hs.HS_WS_DECODE_SPARSE) if use_ws else None
     for layer in range(layers):
         qs = wl.sparse_layer_query(w, layer, device=gen_device).to(DEV)
         os_ = torch.empty_like(qs)
@@ -341,10 +341,33 @@ def test_decode_small_g4_d64():
 
 
 def test_decode_mqa64_d256():
-    """HySparse2's MQA 64/1 at head dim 256 (SIMT decode kernels)."""
+    """HySparse2's MQA 64/1 at head dim 256 (split-k CUDA-core decode)."""
     w = wl.scaled(wl.WORKLOADS["hysparse2_decode"], name="decode_mqa64_d256", batch=3, hq=64,
                   hkv=1, head_dim=256, t=2500, k=256, window=64)
     run_decode(w, torch.tensor([2500, 1, 1300], dtype=torch.int32))
+
+
+def test_decode_mqa64_d256_without_workspace():
+    """The same shape without a workspace: one CTA per sequence and group."""
+    w = wl.scaled(wl.WORKLOADS["hysparse2_decode"], name="decode_mqa64_d256_nows", batch=2, hq=64,
+                  hkv=1, head_dim=256, t=1500, k=256, window=64)
+    run_decode(w, torch.tensor([1500, 700], dtype=torch.int32), layers=1, use_ws=False)
+
+
+def test_decode_wide_groups_split():
+    """Groups of 64 heads at d = 128, 32 at d = 64 and 18 at d = 128 (split-k
+    CUDA-core decode; splits of 512 keys with a ragged last one, short and
+    1-key caches)."""
+    w = wl.scaled(wl.WORKLOADS["hysparse2_decode"], name="decode_g64_d128", batch=2, hq=128,
+                  hkv=2, head_dim=128, t=1700, k=300, window=32)
+    run_decode(w, torch.tensor([1700, 513], dtype=torch.int32), layers=1)
+    w = wl.scaled(wl.WORKLOADS["hysparse2_decode"], name="decode_g32_d64", batch=2, hq=32,
+                  hkv=1, head_dim=64, t=900, k=128, window=16)
+    run_decode(w, torch.tensor([1, 900], dtype=torch.int32), layers=1)
+    # 18 heads: warps own 3 or 2 heads, logit rows not 16-byte multiples
+    w = wl.scaled(wl.WORKLOADS["hysparse2_decode"], name="decode_g18", batch=1, hq=18, hkv=1,
+                  head_dim=128, t=600, k=128, window=16)
+    run_decode(w, torch.tensor([600], dtype=torch.int32), layers=1)
 
 
 def test_decode_bad_length_sets_status():

@@ -183,6 +183,13 @@ typedef enum { HS_DECODE_FULL_INDEX = 0, HS_DECODE_SPARSE = 1 } hs_decode_kind;
  *           HS_DECODE_SPARSE needs none (its size is 0; NULL allowed): one
  *           kernel per step, each (sequence, group) on a cluster of CTAs that
  *           merge their partial results in distributed shared memory.
+ *           Groups of more than 16 heads and head_dim 256 (CUDA-core
+ *           kernels): with hs_workspace_size(p, HS_WS_DECODE_FULL /
+ *           HS_WS_DECODE_SPARSE) bytes both steps run split-k over many CTAs
+ *           (the full step holds every key's head logits, 4 * group bytes per
+ *           cache row, plus per-split partials); with a smaller workspace, or
+ *           NULL, one CTA per (sequence, group) runs each step instead: same
+ *           results, far slower on long caches.
  * The caller keeps k_cache, v_cache and idx alive until the last sparse layer
  * of the block has run.
  */

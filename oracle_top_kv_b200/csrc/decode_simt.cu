@@ -89,15 +89,19 @@ static size_t ws_bytes(const KParams& p, bool full) {
     return b;
 }
 
-// kGather = false: keys sp*kFullKeys .. of the cache (full step, keys <= t);
-// true: entries sp*kSparseKeys .. of the sequence-group's index row (sparse
-// step).  Paged caches are not taken here.
-template <int D, bool kGather>
+// kMode 0: keys sp*kFullKeys .. of the cache (decode full step, keys <= t);
+// 1: entries sp*kSparseKeys .. of the sequence-group's index row (decode
+// sparse step); 2: a sparse layer in prefill -- CTA (query row) takes all
+// of the row's index entries and writes o and lse itself (no split, no
+// workspace).  Paged caches are not taken here.
+template <int D, int kMode>
 __global__ void __launch_bounds__(kThreads)
     dsm_split_kernel(KParams p, const __nv_bfloat16* __restrict__ q,
                      const __nv_bfloat16* __restrict__ kc, const __nv_bfloat16* __restrict__ vc,
                      const int32_t* __restrict__ seq_len, const int32_t* __restrict__ idx,
-                     const int32_t* __restrict__ cnt, Ws ws) {
+                     const int32_t* __restrict__ cnt, Ws ws, __nv_bfloat16* __restrict__ o_out,
+                     float* __restrict__ lse_out) {
+    constexpr bool kGather = kMode != 0, kPrefill = kMode == 2;
     using S = Smem<D>;
     constexpr int E = D / 32;  // d elements per lane in the PV accumulation
     extern __shared__ __align__(16) unsigned char smem[];
@@ -105,19 +109,23 @@ __global__ void __launch_bounds__(kThreads)
     unsigned char* ks = smem + S::kK;
     __nv_bfloat16* vs = reinterpret_cast<__nv_bfloat16*>(smem + S::kV);
     int* ids = reinterpret_cast<int*>(smem + S::kIds);
-    const int sp = blockIdx.x, unit = blockIdx.y;
+    // row: the index row / query row (prefill), else the sequence-group
+    const int sp = kPrefill ? 0 : (int)blockIdx.x;
+    const int row = kPrefill ? (int)blockIdx.x : (int)blockIdx.y;
+    const int j = kPrefill ? row % p.t_q : 0;
+    const int unit = kPrefill ? row / p.t_q : row;
     const int u = unit % p.hkv, b = unit / p.hkv;
     const int g = p.group;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int L = seq_len[b];
+    const int L = kPrefill ? p.q_offset + j + 1 : seq_len[b];
     const bool valid = L >= 1 && L <= p.t_kv;
     const int t = L - 1;
     int n_keys = 0, first = 0;
     if (valid) {
         if (kGather) {
-            const int c = clamp_count(cnt[unit], p.ksel);
-            first = sp * kSparseKeys;
-            n_keys = max(0, min(c, first + kSparseKeys) - first);
+            const int c = clamp_count(cnt[row], p.ksel);
+            first = kPrefill ? 0 : sp * kSparseKeys;
+            n_keys = kPrefill ? c : max(0, min(c, first + kSparseKeys) - first);
         } else {
             first = sp * kFullKeys;
             n_keys = max(0, min(L, first + kFullKeys) - first);
@@ -125,10 +133,11 @@ __global__ void __launch_bounds__(kThreads)
     }
     for (int x = threadIdx.x; x < g * D; x += kThreads) {
         const int h = u * g + x / D;
-        qs[x] = __bfloat162float(q[((size_t)b * p.hq + h) * D + x % D]) * p.scale_log2;
+        qs[x] = __bfloat162float(q[(((size_t)b * p.hq + h) * p.t_q + j) * D + x % D]) *
+                p.scale_log2;
     }
     const size_t kvoff = (size_t)unit * p.t_kv * D;
-    const int32_t* irow = idx + (size_t)unit * p.ksel;
+    const int32_t* irow = idx + (size_t)row * p.ksel;
     const int my_n = g > warp ? (g - 1 - warp) / kWarps + 1 : 0;  // heads of this warp
     float m[kHeadsPerWarp], l[kHeadsPerWarp], o[kHeadsPerWarp][E];
 #pragma unroll
@@ -233,6 +242,21 @@ __global__ void __launch_bounds__(kThreads)
                 for (int e = 0; e < E; ++e) o[hh][e] += pj * vf[e];
             }
         }
+    }
+    if (kPrefill) {  // the row's whole index set: final outputs
+        if (!valid) return;
+#pragma unroll
+        for (int hh = 0; hh < kHeadsPerWarp; ++hh) {
+            if (hh >= my_n) break;
+            const size_t orow = ((size_t)b * p.hq + u * g + warp + hh * kWarps) * p.t_q + j;
+            const float inv = l[hh] > 0.f ? 1.f / l[hh] : 0.f;
+#pragma unroll
+            for (int e = 0; e < E; e += 2)
+                *reinterpret_cast<uint32_t*>(o_out + orow * D + lane * E + e) =
+                    pack_bf16(o[hh][e] * inv, o[hh][e + 1] * inv);
+            if (lane == 0) lse_out[orow] = l[hh] > 0.f ? (m[hh] + log2f(l[hh])) * kLn2 : -INFINITY;
+        }
+        return;
     }
     // partial of each of the warp's heads: m, l (log2 domain), O
     float* part = ws.part + ((size_t)unit * ws.n_split + sp) * g * (D + 2);
@@ -386,13 +410,14 @@ static cudaError_t launch_t(const KParams& p, bool full, const void* q, const vo
                             void* o, float* lse, float* sel, void* ws_base, cudaStream_t st) {
     Ws w = ws_layout(p, ws_base, full);
     const dim3 grid((unsigned)w.n_split, (unsigned)(p.batch * p.hkv));
-    auto kern = full ? dsm_split_kernel<D, false> : dsm_split_kernel<D, true>;
+    auto kern = full ? dsm_split_kernel<D, 0> : dsm_split_kernel<D, 1>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)Smem<D>::kBytes);
     if (e != cudaSuccess) return e;
     kern<<<grid, kThreads, Smem<D>::kBytes, st>>>(p, (const __nv_bfloat16*)q,
                                                    (const __nv_bfloat16*)kc,
-                                                   (const __nv_bfloat16*)vc, seq_len, idx, cnt, w);
+                                                   (const __nv_bfloat16*)vc, seq_len, idx, cnt, w,
+                                                   nullptr, nullptr);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     dsm_combine_kernel<D><<<p.batch * p.hq, D, 0, st>>>(p, w, seq_len, (__nv_bfloat16*)o, lse);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -408,7 +433,41 @@ static cudaError_t launch_t(const KParams& p, bool full, const void* q, const vo
     return cudaGetLastError();
 }
 
+template <int D>
+static cudaError_t launch_prefill_t(const KParams& p, const void* q, const void* kc,
+                                   const void* vc, const int32_t* idx, const int32_t* cnt,
+                                   void* o, float* lse, cudaStream_t st) {
+    Ws w{};
+    auto kern = dsm_split_kernel<D, 2>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Smem<D>::kBytes);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)((long long)p.batch * p.hkv * p.t_q);
+    kern<<<grid, kThreads, Smem<D>::kBytes, st>>>(p, (const __nv_bfloat16*)q,
+                                                   (const __nv_bfloat16*)kc,
+                                                   (const __nv_bfloat16*)vc, nullptr, idx, cnt, w,
+                                                   (__nv_bfloat16*)o, lse);
+    return cudaGetLastError();
+}
+
 }  // namespace dsm
+
+// Token-mode sparse layer in prefill on the CUDA cores for wide groups and
+// head_dim 256 (bf16, contiguous K^F/V^F, no window branch): one CTA per
+// (query row, group), no workspace.
+bool sparse_simt_rows_supported(const KParams& p, int dtype) {
+    return dtype == HS_BF16 && p.mode == 1 && !p.bt && p.group <= dsm::kMaxGroup &&
+           (p.head_dim == 64 || p.head_dim == 128 || p.head_dim == 256) &&
+           (long long)p.batch * p.hkv * p.t_q < (1ll << 31);
+}
+
+cudaError_t launch_sparse_simt_rows(const KParams& p, const void* q, const void* kf,
+                                    const void* vf, const int32_t* idx, const int32_t* cnt,
+                                    void* o, float* lse, cudaStream_t st) {
+    if (p.head_dim == 64) return dsm::launch_prefill_t<64>(p, q, kf, vf, idx, cnt, o, lse, st);
+    if (p.head_dim == 128) return dsm::launch_prefill_t<128>(p, q, kf, vf, idx, cnt, o, lse, st);
+    return dsm::launch_prefill_t<256>(p, q, kf, vf, idx, cnt, o, lse, st);
+}
 
 // Shapes this path takes: bf16, contiguous cache, groups of up to 64 heads,
 // head_dim 64, 128 or 256.

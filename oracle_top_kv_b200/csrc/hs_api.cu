@@ -174,12 +174,20 @@ hs_status hs_sparse_attn_reuse(const hs_params* p, const void* q_sparse, const v
                                           local ? k_local : nullptr, v_local, o_global,
                                           lse_global, o_local, lse_local, st);
         });
-    if (!mma_shape(kp))
+    if (!mma_shape(kp)) {
+        // wide groups / d = 256: one CTA per query row and group with staged
+        // K/V tiles (token mode, no window branch), else the per-head SIMT kernel
+        if (!local && hs::sparse_simt_rows_supported(kp, p->dtype))
+            return launched(1, [&] {
+                return hs::launch_sparse_simt_rows(kp, q_sparse, k_f, v_f, idx, idx_count,
+                                                   o_global, lse_global, st);
+            });
         return launched(1, [&] {
             return hs::launch_sparse_simt(kp, p->dtype, q_sparse, k_f, v_f, idx, idx_count,
                                           local ? k_local : nullptr, v_local, o_global,
                                           lse_global, o_local, lse_local, st);
         });
+    }
     if (hs::sparse_tc_supported(kp, p->dtype)) {
         // global branch, then the window branch, on the tensor cores
         return launched(local ? 2 : 1, [&] {

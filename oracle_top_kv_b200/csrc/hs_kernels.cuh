@@ -52,6 +52,13 @@ cudaError_t launch_decode_simt(const KParams& p, bool full, const void* q, const
                                int32_t* cnt, void* o, float* lse, float* sel, void* ws,
                                cudaStream_t st);
 
+// Token-mode sparse layer in prefill on the CUDA cores (wide groups, head_dim
+// 256; bf16, contiguous K^F/V^F, no window branch): one CTA per query row.
+bool sparse_simt_rows_supported(const KParams& p, int dtype);
+cudaError_t launch_sparse_simt_rows(const KParams& p, const void* q, const void* kf,
+                                    const void* vf, const int32_t* idx, const int32_t* cnt,
+                                    void* o, float* lse, cudaStream_t st);
+
 // seq_len as for launch_full_simt.  Groups of up to 64 heads, head_dim 64,
 // 128 or 256.
 cudaError_t launch_sparse_simt(const KParams& p, int dtype, const void* q, const void* kf,

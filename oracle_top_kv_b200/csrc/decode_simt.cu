@@ -30,7 +30,7 @@ constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kTile = 32;            // keys staged per step
 constexpr int kFullKeys = 512;       // cache keys per split (full step)
-constexpr int kSparseKeys = 128;     // index entries per split (sparse step)
+constexpr int kSparseKeys = 32;      // index entries per split (sparse step): one tile
 constexpr int kMaxGroup = 64;
 constexpr int kHeadsPerWarp = kMaxGroup / kWarps;  // 8
 constexpr int kSelThreads = 512;

@@ -355,9 +355,9 @@ def test_decode_mqa64_d256_without_workspace():
 
 
 def test_decode_wide_groups_split():
-    """Groups of 64 heads at d = 128, 32 at d = 64 and 18 at d = 128 (split-k
-    CUDA-core decode; splits of 512 keys with a ragged last one, short and
-    1-key caches)."""
+    """Groups of 64 heads at d = 128, 32 at d = 64, 18 at d = 128 and 4 at d =
+    256 (split-k CUDA-core decode; splits of 512 keys with a ragged last one,
+    short and 1-key caches)."""
     w = wl.scaled(wl.WORKLOADS["hysparse2_decode"], name="decode_g64_d128", batch=2, hq=128,
                   hkv=2, head_dim=128, t=1700, k=300, window=32)
     run_decode(w, torch.tensor([1700, 513], dtype=torch.int32), layers=1)
@@ -368,6 +368,10 @@ def test_decode_wide_groups_split():
     w = wl.scaled(wl.WORKLOADS["hysparse2_decode"], name="decode_g18", batch=1, hq=18, hkv=1,
                   head_dim=128, t=600, k=128, window=16)
     run_decode(w, torch.tensor([600], dtype=torch.int32), layers=1)
+    # 4 heads at d = 256: half the warps own no head
+    w = wl.scaled(wl.WORKLOADS["hysparse2_decode"], name="decode_g4_d256", batch=2, hq=8, hkv=2,
+                  head_dim=256, t=800, k=128, window=16)
+    run_decode(w, torch.tensor([800, 129], dtype=torch.int32), layers=1)
 
 
 def test_decode_bad_length_sets_status():

@@ -20,6 +20,11 @@ CASES = {
     "wide": (wl.scaled(wl.WORKLOADS["long_1m_chunk"], name="sample_wide", hq=16, hkv=1,
                        t=266240, t_q=40, q_offset=266200, k=1024, window=128,
                        needles="loguniform:16"), True),
+    # the same long scan without a workspace: the shared-memory selector's
+    # deep-ring configuration (1408-entry buffers, 10 sampled tiles)
+    "smem_long": (wl.scaled(wl.WORKLOADS["long_1m_chunk"], name="sample_smem_long", hq=16, hkv=1,
+                            t=266240, t_q=40, q_offset=266200, k=1024, window=128,
+                            needles="loguniform:16"), False),
     # a shorter scan without a workspace: the shared-memory selector
     "smem": (wl.scaled(wl.WORKLOADS["hysparse2_prefill"], name="sample_smem", hq=32, hkv=2,
                        t=40000, t_q=40, q_offset=39960, k=1024, window=128,
